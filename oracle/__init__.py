@@ -1,0 +1,157 @@
+"""fp64 oracle of the MoRE low-rank router — TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import this package.  The routing library (``mixture_experts_rank_b200``) never
+does, and shares no code with it.  The arithmetic lives in ``more_oracle.c``
+(plain C loops in double precision); this module only marshals numpy arrays.
+
+Source: "MoRE: Scaling mixture of experts with hardware-aware low-rank routing"
+(arXiv 2609.36301), §2 "MoRE layer", App. F eq. (5) and Algorithm 1.
+Parity status of every function: pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "more_oracle.c")
+_LIB = os.path.join(_HERE, "libmore_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile ``libmore_oracle.so`` next to its source.
+
+    -O2 without -ffast-math, so the loops keep IEEE double arithmetic in source order.
+    """
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def _bind(lib):
+    lib.oracle_route.restype = ctypes.c_int
+    lib.oracle_route.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 ctypes.c_int, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P,
+                                 ctypes.c_int]
+    lib.oracle_logits.restype = ctypes.c_int
+    lib.oracle_logits.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  _P, ctypes.c_int64, _P]
+    lib.oracle_projection.restype = ctypes.c_int
+    lib.oracle_projection.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _P,
+                                      ctypes.c_int64, _P]
+    lib.oracle_logits_at.restype = ctypes.c_int
+    lib.oracle_logits_at.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int64, _P, _P, _P]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _u16(a, shape):
+    a = np.ascontiguousarray(a, dtype=np.uint16)
+    if a.size != int(np.prod(shape)):
+        raise ValueError(f"expected {shape} bf16 elements, got {a.shape}")
+    return a
+
+
+def _rows(rows, N):
+    if rows is None:
+        return None, N
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    return rows, rows.size
+
+
+@dataclass
+class OracleResult:
+    idx: np.ndarray      # (n, k) int32, routing order
+    gate: np.ndarray     # (n, k) float64
+    logit: np.ndarray    # (n, k) float64, logits of idx
+    margin: np.ndarray   # (n,) l_(k) - l_(k+1); inf when k == M
+    gaps: np.ndarray     # (n, k) l_(j) - l_(j+1); gaps[:, k-1] == margin
+    rms: np.ndarray      # (n,) sqrt(mean_e l_e^2)
+    counts: np.ndarray   # (M,) int64 selections per expert over these rows
+
+
+def route(X, R1, R2, N: int, h: int, r: int, M: int, k: int, rows=None,
+          threads: int | None = None) -> OracleResult:
+    """Route tokens ``rows`` (default: all N) of bf16 X (N x h) with R1 (h x r), R2 (r x M)."""
+    X = _u16(X, (N, h))
+    R1 = _u16(R1, (h, r))
+    R2 = _u16(R2, (r, M))
+    rows, n = _rows(rows, N)
+    idx = np.empty((n, k), np.int32)
+    gate = np.empty((n, k))
+    logit = np.empty((n, k))
+    margin = np.empty(n)
+    gaps = np.empty((n, k))
+    rms = np.empty(n)
+    counts = np.empty(M, np.int64)
+    rc = _load().oracle_route(X.ctypes.data, R1.ctypes.data, R2.ctypes.data, N, h, r, M, k,
+                              None if rows is None else rows.ctypes.data, n, idx.ctypes.data,
+                              gate.ctypes.data, logit.ctypes.data, margin.ctypes.data, gaps.ctypes.data,
+                              rms.ctypes.data, counts.ctypes.data,
+                              threads or max(1, min(64, os.cpu_count() or 1)))
+    if rc != 0:
+        raise ValueError("oracle_route: invalid arguments")
+    return OracleResult(idx, gate, logit, margin, gaps, rms, counts)
+
+
+def logits(X, R1, R2, N: int, h: int, r: int, M: int, rows=None) -> np.ndarray:
+    """All M logits of tokens ``rows`` (n x M, float64)."""
+    X = _u16(X, (N, h))
+    R1 = _u16(R1, (h, r))
+    R2 = _u16(R2, (r, M))
+    rows, n = _rows(rows, N)
+    out = np.empty((n, M))
+    rc = _load().oracle_logits(X.ctypes.data, R1.ctypes.data, R2.ctypes.data, N, h, r, M,
+                               None if rows is None else rows.ctypes.data, n, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_logits: invalid arguments")
+    return out
+
+
+def projection(X, R1, N: int, h: int, r: int, rows=None) -> np.ndarray:
+    """z = x . R1 of tokens ``rows`` (n x r, float64)."""
+    X = _u16(X, (N, h))
+    R1 = _u16(R1, (h, r))
+    rows, n = _rows(rows, N)
+    out = np.empty((n, r))
+    rc = _load().oracle_projection(X.ctypes.data, R1.ctypes.data, N, h, r,
+                                   None if rows is None else rows.ctypes.data, n, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_projection: invalid arguments")
+    return out
+
+
+def logits_at(X, R1, R2, N: int, h: int, r: int, M: int, rows, experts) -> np.ndarray:
+    """Logit of each (rows[p], experts[p]) pair (float64)."""
+    X = _u16(X, (N, h))
+    R1 = _u16(R1, (h, r))
+    R2 = _u16(R2, (r, M))
+    rows = np.ascontiguousarray(rows, dtype=np.int64).ravel()
+    experts = np.ascontiguousarray(experts, dtype=np.int32).ravel()
+    if rows.size != experts.size:
+        raise ValueError("rows and experts differ in length")
+    out = np.empty(rows.size)
+    rc = _load().oracle_logits_at(X.ctypes.data, R1.ctypes.data, R2.ctypes.data, N, h, r, M, rows.size,
+                                  rows.ctypes.data, experts.ctypes.data, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_logits_at: invalid arguments")
+    return out

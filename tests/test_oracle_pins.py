@@ -1,0 +1,267 @@
+"""Pins of the fp64 oracle against facts the MoRE pages and plain mathematics fix.
+
+Source: "MoRE: Scaling mixture of experts with hardware-aware low-rank routing"
+(arXiv 2609.36301).  Every check here is independent of the oracle's own code:
+explicit W = R1 R2 products, brute-force ranks, closed-form constructions from
+App. J, symmetry (Lemma 3), limiting cases of the softmax, and statistics
+(Proposition 1, Lemma 1).  ``test_oracle_mutations.py`` shows that plausible
+mistakes planted in a copy of the oracle fail these pins.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic as syn
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(values):
+    v = np.asarray(values, dtype=np.float64)
+    bits = syn.f32_to_bf16_bits(v.astype(np.float32))
+    assert np.array_equal(syn.bf16_bits_to_f64(bits), v), "value not exact in bf16"
+    return bits
+
+
+def identity_router(values):
+    """h = r = M and R1 = R2 = I, so the logits equal the (bf16-exact) inputs."""
+    X = bf16(np.atleast_2d(values))
+    M = X.shape[1]
+    eye = bf16(np.eye(M))
+    return X, eye, eye
+
+
+def route_values(values, k):
+    X, R1, R2 = identity_router(values)
+    N, M = X.shape
+    return oracle.route(X, R1, R2, N, M, M, M, k, threads=2)
+
+
+def brute_force_order(l):
+    """Routing order by counting, for each expert, the experts that beat it."""
+    M = len(l)
+    rank = np.array([sum(1 for b in range(M) if l[b] > l[a] or (l[b] == l[a] and b < a))
+                     for a in range(M)])
+    order = np.empty(M, dtype=np.int64)
+    order[rank] = np.arange(M)
+    return order
+
+
+def read_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([part.split() for part in line.split("|")])
+    return rows
+
+
+# --- factorisation: standard router with W = R1 R2 (MoRE §2, A1 == A2) -----------
+
+def test_logits_equal_explicit_W_product():
+    N, h, r, M = 37, 48, 16, 72
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=11)
+    Xf, R1f, R2f = (syn.bf16_bits_to_f64(a) for a in (X, R1, R2))
+    W = R1f @ R2f                                   # h x M, formed explicitly
+    expected = Xf @ W                               # standard router x W
+    got = oracle.logits(X, R1, R2, N, h, r, M)
+    np.testing.assert_allclose(got, expected, rtol=1e-11, atol=1e-12)
+    res = oracle.route(X, R1, R2, N, h, r, M, 5)
+    np.testing.assert_allclose(res.logit, np.take_along_axis(expected, res.idx.astype(np.int64), 1),
+                               rtol=1e-11, atol=1e-12)
+
+
+def test_projection_and_pairs_agree_with_matmul():
+    N, h, r, M = 9, 40, 24, 30
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=5)
+    Xf, R1f, R2f = (syn.bf16_bits_to_f64(a) for a in (X, R1, R2))
+    np.testing.assert_allclose(oracle.projection(X, R1, N, h, r), Xf @ R1f, rtol=1e-12, atol=1e-13)
+    rows = np.array([0, 3, 3, 8, 1])
+    experts = np.array([29, 0, 7, 15, 2])
+    np.testing.assert_allclose(oracle.logits_at(X, R1, R2, N, h, r, M, rows, experts),
+                               (Xf @ R1f @ R2f)[rows, experts], rtol=1e-11, atol=1e-12)
+    sub = oracle.logits(X, R1, R2, N, h, r, M, rows=rows)
+    np.testing.assert_allclose(sub, (Xf @ R1f @ R2f)[rows], rtol=1e-11, atol=1e-12)
+
+
+# --- selection: brute force, ties, relabelling ----------------------------------
+
+@pytest.mark.parametrize("M", [1, 2, 7, 13, 33])
+def test_topk_matches_brute_force_random(M):
+    rng = np.random.default_rng(M)
+    vals = syn.bf16_bits_to_f64(syn.f32_to_bf16_bits(rng.standard_normal((6, M)).astype(np.float32)))
+    for k in range(1, M + 1):
+        res = route_values(vals, k)
+        for n in range(vals.shape[0]):
+            assert list(res.idx[n]) == list(brute_force_order(vals[n])[:k])
+
+
+@pytest.mark.parametrize("M", [5, 16, 40])
+def test_topk_matches_brute_force_tie_heavy(M):
+    rng = np.random.default_rng(100 + M)
+    vals = rng.integers(-2, 3, size=(8, M)).astype(np.float64)   # many equal logits
+    for k in sorted({1, 2, M // 2, M - 1, M}):
+        if k < 1:
+            continue
+        res = route_values(vals, k)
+        for n in range(vals.shape[0]):
+            assert list(res.idx[n]) == list(brute_force_order(vals[n])[:k])
+
+
+def test_golden_tie_order():
+    for (mk, logits, expected) in read_golden("tie_order.txt"):
+        M, k = int(mk[0]), int(mk[1])
+        vals = [float(v) for v in logits]
+        assert len(vals) == M
+        res = route_values([vals], k)
+        assert list(res.idx[0]) == [int(e) for e in expected]
+
+
+def test_relabelling_equivariance():
+    """Lemma 3 (App. J): permuting the experts permutes the selected set (no ties)."""
+    N, h, r, M, k = 64, 32, 16, 96, 7
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=3)
+    base = oracle.route(X, R1, R2, N, h, r, M, k)
+    perm = np.random.default_rng(0).permutation(M)            # new column j is old expert perm[j]
+    R2p = np.ascontiguousarray(R2[:, perm])
+    moved = oracle.route(X, R1, R2p, N, h, r, M, k)
+    assert np.array_equal(perm[moved.idx], base.idx)
+    np.testing.assert_array_equal(moved.logit, base.logit)
+    np.testing.assert_array_equal(moved.counts[np.argsort(perm)], base.counts)
+
+
+# --- gates, margin, rms, counts --------------------------------------------------
+
+def test_k_equals_M_gives_full_softmax():
+    N, h, r, M = 20, 24, 16, 12
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=8)
+    res = oracle.route(X, R1, R2, N, h, r, M, M)
+    full = oracle.logits(X, R1, R2, N, h, r, M)
+    e = np.exp(full - full.max(axis=1, keepdims=True))
+    softmax = e / e.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(res.gate, np.take_along_axis(softmax, res.idx.astype(np.int64), 1),
+                               rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(res.gate.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+    assert np.all(np.isinf(res.margin))
+
+
+def test_gate_special_cases():
+    vals = np.array([[0.5, 3.0, -1.0, 2.25, 0.0]])
+    one = route_values(vals, 1)
+    assert one.gate[0, 0] == 1.0
+    two = route_values(vals, 2)
+    d = 3.0 - 2.25                                       # k = 2: softmax is the logistic function
+    np.testing.assert_allclose(two.gate[0], [1 / (1 + np.exp(-d)), 1 / (1 + np.exp(d))], rtol=1e-15)
+
+
+def test_margin_gaps_and_rms_against_sorted_logits():
+    N, h, r, M, k = 25, 32, 16, 50, 6
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=21)
+    res = oracle.route(X, R1, R2, N, h, r, M, k)
+    full = oracle.logits(X, R1, R2, N, h, r, M)
+    s = -np.sort(-full, axis=1)
+    np.testing.assert_allclose(res.logit, s[:, :k], rtol=0, atol=0)
+    np.testing.assert_allclose(res.margin, s[:, k - 1] - s[:, k], rtol=0, atol=0)
+    np.testing.assert_allclose(res.gaps, s[:, :k] - s[:, 1:k + 1], rtol=0, atol=0)
+    np.testing.assert_allclose(res.rms, np.linalg.norm(full, axis=1) / np.sqrt(M), rtol=1e-14)
+
+
+def test_counts_are_the_bincount_of_indices():
+    N, h, r, M, k = 300, 32, 16, 40, 3
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=2)
+    res = oracle.route(X, R1, R2, N, h, r, M, k, threads=3)
+    assert res.counts.sum() == N * k
+    np.testing.assert_array_equal(res.counts, np.bincount(res.idx.ravel(), minlength=M))
+    rows = np.array([7, 299, 0, 7])
+    part = oracle.route(X, R1, R2, N, h, r, M, k, rows=rows)
+    np.testing.assert_array_equal(part.idx, res.idx[rows])
+    np.testing.assert_array_equal(part.counts, np.bincount(res.idx[rows].ravel(), minlength=M))
+    # each row's selected experts are distinct
+    for n in range(N):
+        assert len(set(res.idx[n])) == k
+
+
+# --- closed forms from App. J -----------------------------------------------------
+
+def test_golden_jl_construction():
+    for (mk, S, margin, gate) in read_golden("jl_construction.txt"):
+        M, k = int(mk[0]), int(mk[1])
+        S = [int(s) for s in S]
+        x = np.full(M, -float(k))
+        x[S] = float(M - k)
+        X, R1, R2 = identity_router([x])
+        res = oracle.route(X, R1, R2, 1, M, M, M, k)
+        assert list(res.idx[0]) == S
+        assert res.margin[0] == float(margin[0])
+        np.testing.assert_allclose(res.gate[0], float(gate[0]), rtol=0, atol=1e-15)
+
+
+def hypercube_router(h, r):
+    """R1 selects the first r coordinates; column a of R2 is the sign vector of a."""
+    M = 2 ** r
+    R1 = np.zeros((h, r))
+    R1[:r, :r] = np.eye(r)
+    signs = np.array([[1.0 if (a >> l) & 1 else -1.0 for a in range(M)] for l in range(r)])
+    return bf16(R1), bf16(signs), M
+
+
+def test_golden_hypercube_top1_is_sign_pattern():
+    R1, R2, M = hypercube_router(8, 8)
+    for (z, expected) in read_golden("hypercube_k1.txt"):
+        x = bf16([[float(v) for v in z]])
+        res = oracle.route(x, R1, R2, 1, 8, 8, M, 1)
+        assert res.idx[0, 0] == int(expected[0])
+
+
+def test_hypercube_top1_random_inputs():
+    h, r = 12, 8
+    R1, R2, M = hypercube_router(h, r)
+    X = syn.normal_bf16(4, syn.TENSOR_X, 500, h)
+    xf = syn.bf16_bits_to_f64(X)[:, :r]
+    res = oracle.route(X, R1, R2, 500, h, r, M, 1)
+    expected = ((xf > 0) * (1 << np.arange(r))).sum(axis=1)
+    np.testing.assert_array_equal(res.idx[:, 0], expected)
+
+
+@pytest.mark.parametrize("k", [1, 4])
+def test_hypercube_load_balance_bound(k):
+    """Proposition 1: with M = 2^r sign-vector experts each is chosen w.p. exactly k/M,
+    and max_a |N_a - nk/M| <= sqrt(2 n k L / M) + (2/3) L, L = log(2M/delta), w.p. 1 - delta."""
+    h, r, n, delta = 10, 6, 20000, 1e-6
+    R1, R2, M = hypercube_router(h, r)
+    X = syn.normal_bf16(9, syn.TENSOR_X, n, h)
+    res = oracle.route(X, R1, R2, n, h, r, M, k)
+    L = np.log(2 * M / delta)
+    bound = np.sqrt(2 * n * k * L / M) + 2.0 / 3.0 * L
+    assert np.max(np.abs(res.counts - n * k / M)) <= bound
+    assert res.counts.sum() == n * k
+
+
+def test_logit_variance_matches_lemma_1():
+    """Lemma 1 (App. D.2): Var([R1 R2 x]_e) = r s1^2 s2^2 |x|^2; with R1 ~ N(0, 1/h) and
+    R2 ~ N(0, 1/r) this is |x|^2 / h.  Averaged over tokens, experts and three seeds."""
+    h, r, M, N = 128, 32, 192, 512
+    ratios = []
+    for seed in (0, 1, 2):
+        X, R1, R2 = syn.router_inputs(N, h, r, M, seed=seed)
+        l = oracle.logits(X, R1, R2, N, h, r, M)
+        xf = syn.bf16_bits_to_f64(X)
+        ratios.append(np.mean(l ** 2 / (np.sum(xf ** 2, axis=1, keepdims=True) / h)))
+    assert abs(np.mean(ratios) - 1.0) < 0.08
+
+
+# --- argument checks --------------------------------------------------------------
+
+def test_oracle_rejects_invalid_arguments():
+    X, R1, R2 = syn.router_inputs(4, 8, 4, 6)
+    with pytest.raises(ValueError):
+        oracle.route(X, R1, R2, 4, 8, 4, 6, 7)           # k > M
+    with pytest.raises(ValueError):
+        oracle.route(X, R1, R2, 4, 8, 4, 6, 0)           # k < 1
+    with pytest.raises(ValueError):
+        oracle.route(X, R1, R2, 4, 8, 4, 6, 2, rows=[4])  # row out of range
+    empty = oracle.route(X, R1, R2, 4, 8, 4, 6, 2, rows=np.zeros(0, np.int64))
+    assert empty.idx.shape == (0, 2) and empty.counts.sum() == 0
