@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Throughput of the fused low-rank MoE router (MoRE) on B200.
+
+One step = one routing call over the workload's N tokens: z = x.R1, the M logits
+z.R2, top-k with softmax gates, per-expert counts ("MoRE: Scaling mixture of
+experts with hardware-aware low-rank routing", App. F, Algorithm 1).  Default
+workload: prefill, N = 262,144 tokens (256 sequences x 1024), h = 2048, M = 4096,
+r = 32, k = 8, X rows at unit RMS, R1 ~ N(0, 1/h), R2 ~ N(0, 1/r), seed 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--variant auto|fused_tc|small_n|unfused] [--workload NAME]
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank routes its own
+N-token shard of a larger synthetic token set (weak scaling, no collective on the
+data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (N, h, r, M, k, x_unit_rms)
+    "prefill_r32": (262144, 2048, 32, 4096, 8, True),
+    "prefill_r16": (262144, 2048, 16, 4096, 8, True),
+    "prefill_r64": (262144, 2048, 64, 4096, 8, True),
+    "prefill_r128": (262144, 2048, 128, 4096, 8, True),
+    "many_experts": (32768, 4096, 64, 65536, 8, False),
+    "sweep_M1024": (65536, 512, 32, 1024, 8, False),
+    "sweep_M2048": (65536, 512, 32, 2048, 8, False),
+    "sweep_M4096": (65536, 512, 32, 4096, 8, False),
+    "sweep_M8192": (65536, 512, 32, 8192, 8, False),
+    "sweep_M16384": (65536, 512, 32, 16384, 8, False),
+    "tiny": (4096, 128, 32, 192, 4, False),
+}
+METRIC = "routed tokens/s (fused low-rank router + top-k)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def describe(name):
+    N, h, r, M, k, unit = WORKLOADS[name]
+    return (f"{name}: N={N} h={h} M={M} r={r} k={k}, X bf16 N(0,1)"
+            f"{' rows at unit RMS' if unit else ''}, R1 N(0,1/h), R2 N(0,1/r), seed 0")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)) or None, \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores, on a bounded sample of the workload per step."""
+    if rank != 0:
+        return 0
+    import oracle
+    import synthetic as syn
+    N, h, r, M, k, unit = WORKLOADS[args.workload]
+    cores = os.cpu_count() or 1
+    R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
+    R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+    # size the per-step sample from a short probe: about args.ref_step_seconds of CPU work
+    probe = max(cores, 16)
+    Xp = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, probe)
+    t = time.perf_counter()
+    oracle.route(Xp, R1, R2, probe, h, r, M, k, threads=cores)
+    per_tok = (time.perf_counter() - t) / probe
+    S = int(max(cores, min(N, args.ref_step_seconds / max(per_tok, 1e-9))))
+    X = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, S)
+    for _ in range(args.warmup):
+        oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+        times.append(time.perf_counter() - t)
+    step = sum(times) / len(times)
+    value = S / step
+    sample = f"first {S} tokens of the workload per step ({S / N:.4%} of N), all M experts"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": describe(args.workload), "N": N, "h": h, "r": r,
+                                            "M": M, "k": k, "tokens_per_step": S},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(workload, seconds):
+    import oracle
+    import synthetic as syn
+    N, h, r, M, k, unit = WORKLOADS[workload]
+    cores = os.cpu_count() or 1
+    R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
+    R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+    probe = max(cores, 16)
+    Xp = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, probe)
+    t = time.perf_counter()
+    oracle.route(Xp, R1, R2, probe, h, r, M, k, threads=cores)
+    per_tok = (time.perf_counter() - t) / probe
+    S = int(max(probe, min(N, seconds / max(per_tok, 1e-9))))
+    X = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, S)
+    t = time.perf_counter()
+    oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+    el = time.perf_counter() - t
+    return {"value": S / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {S} of the {N} tokens, all M experts, {el:.1f} s on {cores} threads"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="auto", choices=["auto", "fused_tc", "small_n", "unfused"])
+    ap.add_argument("--workload", default="prefill_r32", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample size, in CPU seconds")
+    ap.add_argument("--ref-step-seconds", type=float, default=3.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import mixture_experts_rank_b200 as more
+    import synthetic as syn
+
+    N, h, r, M, k, unit = WORKLOADS[args.workload]
+    # rank i routes tokens [i N, (i+1) N) of one synthetic token set (seed 0)
+    Xh = syn.normal_bf16(0, syn.TENSOR_X, N * world, h, 1.0, unit, rank * N, N)
+    R1h = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
+    R2h = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+
+    def dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+    X, R1, R2 = dev(Xh), dev(R1h), dev(R2h)
+    idx = torch.empty((N, k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((N, k), dtype=torch.float32, device="cuda")
+    cnt = torch.empty((M,), dtype=torch.int32, device="cuda")
+    logits = torch.empty((N, k), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    scratch = None
+    if args.variant == "unfused":
+        scratch = torch.empty(more.unfused_scratch_bytes(N, r, M), dtype=torch.uint8, device="cuda")
+
+    def step():
+        if args.variant == "unfused":
+            more.route_unfused(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate, out_expert_count=cnt,
+                               out_logits=logits, stream=stream)
+        else:
+            more.route(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
+                       variant=args.variant, stream=stream)
+
+    variant_used = args.variant
+    if args.variant == "auto":
+        variant_used = "fused_tc"
+        try:
+            more.route(X[:1024], R1, R2, k, variant="fused_tc")
+        except more.MoreError:
+            variant_used = "small_n"
+        variant_used = variant_used if N >= 512 else "small_n"
+    launches_per_step = 3 if args.variant == "unfused" else 1
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if more.device_status() != 0:
+        raise RuntimeError("a kernel recorded a device error during warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if more.device_status() != 0:
+        raise RuntimeError("a kernel recorded a device error during the timed steps")
+    ms = total_ms / args.steps
+    value = N * world / (ms / 1e3)
+
+    # end to end: pinned host X in, route through the public API, results out
+    e2e = None
+    if not args.no_e2e:
+        router = more.Router(R1, R2, k, N)
+        Xpin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
+        for _ in range(2):
+            router.route_host(Xpin)
+        barrier()
+        torch.cuda.synchronize()
+        e_steps = max(3, min(args.steps, 10))
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(e_steps):
+            router.route_host(Xpin, synchronize=False)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = t0.elapsed_time(t1) / e_steps
+        if dist is not None:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        bi, bo = router.bytes_per_call(N)
+        e2e = {"value": N * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": e_ms}
+
+    if rank == 0:
+        hbm, tc, tc_sus, src = peaks()
+        x_bytes = 2.0 * N * h                        # algorithmic bytes of one launch: X read once
+        flops = 2.0 * N * r * (h + M)                # z = x.R1 and l = z.R2
+        launch_ms = statistics.mean(per_launch) if launches_per_step == 1 else None
+        kernel_ms = launch_ms if launch_ms is not None else ms
+        achieved = x_bytes / (kernel_ms / 1e3) / 1e9
+        traffic = None
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
+                else "fallback 6.65 TB/s",
+                "tensor": {"achieved_tflops": flops / (kernel_ms / 1e3) / 1e12, "peak_tflops": tc,
+                           "frac": flops / (kernel_ms / 1e3) / 1e12 / tc}}
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": describe(args.workload), "N_per_gpu": N, "h": h, "r": r, "M": M, "k": k,
+                           "variant": variant_used, "parallelism": f"token shards x{world}",
+                           "l2": f"inputs larger than L2 (X = {x_bytes / 1e9:.2f} GB per GPU)"
+                           if x_bytes > L2_BYTES else "inputs fit in L2; no flush (L2-warm)"},
+                "roofline": roof, "gpu_launches": launches_per_step * args.steps, "clocks": clocks}
+        if e2e is not None:
+            line["e2e"] = e2e
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

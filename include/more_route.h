@@ -1,0 +1,129 @@
+/*
+ * more_route.h - C ABI of the fused low-rank MoE router for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the MoRE router of "MoRE: Scaling mixture of experts with
+ * hardware-aware low-rank routing" (arXiv 2609.36301):
+ *   §2 "MoRE layer":  g(x; R1, R2) = softmax(TopK(R1 R2 x)), the standard router
+ *                     softmax(TopK(R x)) with R replaced by a rank-r product;
+ *   App. F, eq. (5):  logits l = X R_2^T R_1^T, one B_N x B_M tile at a time;
+ *   App. F, Algorithm 1 (inference, prefilling): z = X R_2^T accumulated in
+ *                     fp32 and narrowed to bf16, one sweep over the experts with a
+ *                     running top-k, out-of-range experts at -infinity, and the
+ *                     (N, k) TopVals/TopIdxs written instead of the (N, M) logits;
+ *   App. F, Fig. 12:  gate weights = softmax over the k selected logits;
+ *   App. F, eq. (9):  f = bincount of TopIdxs (here: out_expert_count).
+ *
+ * Naming: R1 here is h x r (the paper's R_2 transposed) and R2 is r x M (the
+ * paper's R_1 transposed), so z = x . R1 and l = z . R2.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are row-major and live in device memory owned by the caller.
+ *     bf16 tensors are raw 16-bit patterns.  Nothing is retained after a call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise the host, except more_device_status.
+ *   - Per token the k experts are returned in routing order: larger logit
+ *     first, lower expert index first on equal logits (Algorithm 1 keeps the
+ *     earlier expert on equal values).  out_logits[n][j] is the fp32 logit of
+ *     expert out_idx[n][j]; out_gate[n][] is the softmax of those k logits.
+ *   - The logits are computed as in Algorithm 1: z accumulated in fp32 and
+ *     rounded to bf16 (nearest even), then z . R2 accumulated in fp32.
+ *   - out_expert_count[e] is set (not accumulated) to the number of (token,
+ *     slot) pairs of this call that name expert e; the call zeroes it first.
+ *   - Inputs must be finite; results for NaN or infinite inputs are unspecified.
+ *
+ * Argument requirements (checked before anything is launched; a violation
+ * returns an error and launches nothing):
+ *   N >= 0; h >= 8 and h % 8 == 0; M >= 8 and M % 8 == 0; r % 16 == 0 and
+ *   16 <= r <= 128; 1 <= k <= M; k <= MORE_KMAX; M <= MORE_MMAX;
+ *   X (unless N == 0), R1, R2, out_idx, out_gate and out_expert_count non-NULL;
+ *   every pointer 16-byte aligned.  Violations of the shape limits that are
+ *   not errors of meaning (k > MORE_KMAX, r outside 16..128 or not a multiple
+ *   of 16, M > MORE_MMAX) return MORE_ERR_UNSUPPORTED; the rest return
+ *   MORE_ERR_INVALID_ARG.
+ */
+#ifndef MORE_ROUTE_H
+#define MORE_ROUTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MORE_ROUTE_ABI_VERSION 1
+#define MORE_KMAX 16
+#define MORE_MMAX 262144
+
+typedef enum more_status {
+  MORE_OK = 0,
+  MORE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, impossible shape          */
+  MORE_ERR_UNSUPPORTED = 2, /* legal request outside this library's limits        */
+  MORE_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed        */
+  MORE_ERR_DEVICE = 4       /* a kernel recorded an error (see more_device_status) */
+} more_status;
+
+/* Kernel variants of more_route_variant.  All compute the same function. */
+typedef enum more_variant {
+  MORE_VARIANT_AUTO = 0,     /* the fused tensor-core kernel for large N, the small-N kernel otherwise */
+  MORE_VARIANT_FUSED_TC = 1, /* persistent kernel: TMA-staged X, tcgen05 MMAs into TMEM             */
+  MORE_VARIANT_SMALL_N = 2   /* CUDA-core kernel, one warp per token (decode-sized batches)         */
+} more_variant;
+
+/*
+ * Route N tokens.  [MoRE §2 "MoRE layer"; App. F, Algorithm 1 and Fig. 12]
+ *   X                bf16 [N][h]      token hidden vectors
+ *   R1               bf16 [h][r]      first router factor
+ *   R2               bf16 [r][M]      second router factor (one column per expert)
+ *   out_idx          int32 [N][k]     selected experts, routing order
+ *   out_gate         fp32 [N][k]      softmax over the k selected logits
+ *   out_expert_count int32 [M]        selections per expert (zeroed, then counted)
+ *   out_logits       fp32 [N][k]      selected logits, or NULL to skip
+ * No N x M tensor is written: the logits exist only on chip.
+ */
+more_status more_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                       int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
+                       float* out_logits, void* stream);
+
+/* more_route with an explicit kernel variant (more_variant); same contract. */
+more_status more_route_variant(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                               int M, int k, int32_t* out_idx, float* out_gate,
+                               int32_t* out_expert_count, float* out_logits, int variant,
+                               void* stream);
+
+/*
+ * Materialise-then-top-k comparison path (the unfused router of MoRE App. H.6,
+ * Fig. 24): z = X . R1 is written to scratch as bf16 [N][r], the full logits as
+ * fp32 [N][M], then a row-wise top-k and softmax read them back.  Same
+ * arguments and results as more_route, plus caller-owned device scratch of at
+ * least more_route_unfused_scratch_bytes(N, r, M) bytes (16-byte aligned).
+ * Too little scratch returns MORE_ERR_INVALID_ARG.
+ */
+size_t more_route_unfused_scratch_bytes(int64_t N, int r, int M);
+more_status more_route_unfused(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                               int M, int k, int32_t* out_idx, float* out_gate,
+                               int32_t* out_expert_count, float* out_logits, void* scratch,
+                               size_t scratch_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then return and clear the library's device error word
+ * on the current device: MORE_OK if no kernel recorded an error since the last
+ * call, MORE_ERR_DEVICE if one did (e.g. a bounded wait gave up), or
+ * MORE_ERR_CUDA if synchronising failed.  `detail` (may be NULL) receives the
+ * raw error word (an OR of the MORE_DEVERR_* bits).
+ */
+#define MORE_DEVERR_WAIT_TIMEOUT 0x1u  /* a bounded barrier wait ran out            */
+#define MORE_DEVERR_BAD_CONFIG 0x2u    /* a kernel saw a configuration it rejects  */
+more_status more_device_status(void* stream, uint32_t* detail);
+
+/* Static description of a status code. */
+const char* more_status_string(more_status status);
+
+/* MORE_ROUTE_ABI_VERSION of the built library. */
+int more_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MORE_ROUTE_H */

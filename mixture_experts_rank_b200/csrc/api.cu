@@ -1,0 +1,169 @@
+// C ABI of the router: argument validation, variant choice, the device error word.
+#include <mutex>
+
+#include "more_internal.cuh"
+
+namespace more {
+
+// Device error word of this library (one per device; MORE_DEVERR_* bits).
+__device__ unsigned int g_device_status;
+
+namespace {
+
+unsigned int* status_word() {
+  // The symbol address differs per device; cache it per device ordinal.
+  static std::mutex mu;
+  static unsigned int* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+more_status validate(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                     int k, const int32_t* out_idx, const float* out_gate,
+                     const int32_t* out_count, const float* out_logits) {
+  if (N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1)
+    return MORE_ERR_INVALID_ARG;
+  if (!R1 || !R2 || !out_idx || !out_gate || !out_count || (N > 0 && !X)) return MORE_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || !aligned16(R1) || !aligned16(R2) || !aligned16(out_idx) ||
+      !aligned16(out_gate) || !aligned16(out_count) || (out_logits && !aligned16(out_logits)))
+    return MORE_ERR_INVALID_ARG;
+  if (N > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
+  if (k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX) return MORE_ERR_UNSUPPORTED;
+  return MORE_OK;
+}
+
+RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                    int k, int32_t* out_idx, float* out_gate, int32_t* out_count,
+                    float* out_logits, void* stream) {
+  RouteArgs a;
+  a.X = static_cast<const __nv_bfloat16*>(X);
+  a.R1 = static_cast<const __nv_bfloat16*>(R1);
+  a.R2 = static_cast<const __nv_bfloat16*>(R2);
+  a.N = N;
+  a.h = h;
+  a.r = r;
+  a.M = M;
+  a.k = k;
+  a.out_idx = out_idx;
+  a.out_gate = out_gate;
+  a.out_count = out_count;
+  a.out_logits = out_logits;
+  a.status = nullptr;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return a;
+}
+
+// Below this many tokens the small-N kernel wins: the fused kernel works on
+// 128-token tiles, one per SM, and a handful of tiles leaves the GPU idle.
+constexpr int64_t kSmallNThreshold = 512;
+
+}  // namespace
+}  // namespace more
+
+using namespace more;
+
+extern "C" {
+
+int more_abi_version(void) { return MORE_ROUTE_ABI_VERSION; }
+
+const char* more_status_string(more_status s) {
+  switch (s) {
+    case MORE_OK:
+      return "MORE_OK";
+    case MORE_ERR_INVALID_ARG:
+      return "MORE_ERR_INVALID_ARG: null or misaligned pointer, or impossible shape";
+    case MORE_ERR_UNSUPPORTED:
+      return "MORE_ERR_UNSUPPORTED: request outside the library's limits";
+    case MORE_ERR_CUDA:
+      return "MORE_ERR_CUDA: a CUDA call or kernel launch failed";
+    case MORE_ERR_DEVICE:
+      return "MORE_ERR_DEVICE: a kernel recorded an error";
+  }
+  return "unknown more_status";
+}
+
+more_status more_route_variant(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                               int M, int k, int32_t* out_idx, float* out_gate,
+                               int32_t* out_expert_count, float* out_logits, int variant,
+                               void* stream) {
+  more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  if (st != MORE_OK) return st;
+  if (variant < MORE_VARIANT_AUTO || variant > MORE_VARIANT_SMALL_N) return MORE_ERR_INVALID_ARG;
+  RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
+                          stream);
+  a.status = status_word();
+  if (!a.status) return MORE_ERR_CUDA;
+  if (cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
+    return MORE_ERR_CUDA;
+  if (N == 0) return MORE_OK;
+  if (variant == MORE_VARIANT_AUTO)
+    variant = (N >= kSmallNThreshold && fused_tc_supports(a)) ? MORE_VARIANT_FUSED_TC
+                                                              : MORE_VARIANT_SMALL_N;
+  cudaError_t err;
+  if (variant == MORE_VARIANT_FUSED_TC) {
+    if (!fused_tc_supports(a)) return MORE_ERR_UNSUPPORTED;
+    err = launch_fused_tc(a);
+  } else {
+    err = launch_small_n(a);
+  }
+  return err == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
+more_status more_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                       int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
+                       float* out_logits, void* stream) {
+  return more_route_variant(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
+                            MORE_VARIANT_AUTO, stream);
+}
+
+size_t more_route_unfused_scratch_bytes(int64_t N, int r, int M) {
+  if (N < 0 || r < 1 || M < 1) return 0;
+  return unfused_scratch_bytes(N, r, M);
+}
+
+more_status more_route_unfused(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                               int M, int k, int32_t* out_idx, float* out_gate,
+                               int32_t* out_expert_count, float* out_logits, void* scratch,
+                               size_t scratch_bytes, void* stream) {
+  more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  if (st != MORE_OK) return st;
+  if (N > 0 && (!scratch || !aligned16(scratch) || scratch_bytes < unfused_scratch_bytes(N, r, M)))
+    return MORE_ERR_INVALID_ARG;
+  RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
+                          stream);
+  a.status = status_word();
+  if (!a.status) return MORE_ERR_CUDA;
+  if (cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
+    return MORE_ERR_CUDA;
+  if (N == 0) return MORE_OK;
+  return launch_unfused(a, scratch) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
+more_status more_device_status(void* stream, uint32_t* detail) {
+  if (detail) *detail = 0;
+  unsigned int* word = status_word();
+  if (!word) return MORE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MORE_ERR_CUDA;
+  unsigned int value = 0;
+  if (cudaMemcpy(&value, word, sizeof(value), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MORE_ERR_CUDA;
+  if (value != 0) {
+    unsigned int zero = 0;
+    if (cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MORE_ERR_CUDA;
+  }
+  if (detail) *detail = value;
+  return value ? MORE_ERR_DEVICE : MORE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal declarations shared by the router's translation units (not part of the ABI).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "more_route.h"
+
+namespace more {
+
+// Arguments of one routing call after validation.
+struct RouteArgs {
+  const __nv_bfloat16* X;
+  const __nv_bfloat16* R1;
+  const __nv_bfloat16* R2;
+  int64_t N;
+  int h, r, M, k;
+  int32_t* out_idx;
+  float* out_gate;
+  int32_t* out_count;
+  float* out_logits;  // may be null
+  unsigned int* status;  // device error word (MORE_DEVERR_* bits)
+  cudaStream_t stream;
+};
+
+// Launchers; each returns cudaSuccess or the launch error.
+cudaError_t launch_small_n(const RouteArgs& a);
+cudaError_t launch_fused_tc(const RouteArgs& a);
+bool fused_tc_supports(const RouteArgs& a);
+cudaError_t launch_unfused(const RouteArgs& a, void* scratch);
+size_t unfused_scratch_bytes(int64_t N, int r, int M);
+
+// ---- small device helpers -------------------------------------------------
+
+__device__ __forceinline__ float bf16_round(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// Routing order on (value, expert): a goes first iff it has the larger value,
+// or the same value and the lower expert index.
+__device__ __forceinline__ bool goes_first(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+}  // namespace more

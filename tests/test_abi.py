@@ -1,0 +1,93 @@
+"""The C ABI library loads, exports every declared symbol, and rejects bad arguments
+before touching a GPU (these calls return before any CUDA runtime call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(more_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import mixture_experts_rank_b200 as m
+    return m._lib
+
+
+def test_header_declares_the_route_entry_points():
+    names = declared_functions()
+    for required in ("more_route", "more_route_variant", "more_route_unfused",
+                     "more_route_unfused_scratch_bytes", "more_device_status", "more_status_string",
+                     "more_abi_version"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.more_abi_version() == 1
+    for code in range(5):
+        assert lib.more_status_string(code).startswith(b"MORE_")
+    assert lib.more_status_string(99) == b"unknown more_status"
+
+
+def call(lib, N=16, h=64, r=32, M=64, k=4, X=16, R1=16, R2=16, idx=16, gate=16, cnt=16, logits=None,
+         variant=0):
+    P = ctypes.c_void_p
+    return lib.more_route_variant(P(X) if X else None, P(R1) if R1 else None, P(R2) if R2 else None, N, h,
+                                  r, M, k, P(idx) if idx else None, P(gate) if gate else None,
+                                  P(cnt) if cnt else None, P(logits) if logits else None, variant, None)
+
+
+@pytest.mark.parametrize("kwargs,expected", [
+    (dict(k=0), 1), (dict(k=65), 1), (dict(N=-1), 1), (dict(h=4), 1), (dict(h=66), 1),
+    (dict(M=4), 1), (dict(M=70), 1), (dict(X=0), 1), (dict(R1=0), 1), (dict(R2=0), 1),
+    (dict(idx=0), 1), (dict(gate=0), 1), (dict(cnt=0), 1), (dict(X=24), 1), (dict(gate=40), 1),
+    (dict(logits=8), 1), (dict(variant=7), 1),
+    (dict(k=17, M=64), 2), (dict(r=24), 2), (dict(r=8), 2), (dict(r=144), 2), (dict(M=262152), 2),
+])
+def test_invalid_arguments_are_rejected(lib, kwargs, expected):
+    assert call(lib, **kwargs) == expected
+
+
+def test_unfused_scratch_size_and_checks(lib):
+    n = lib.more_route_unfused_scratch_bytes(1000, 32, 256)
+    assert n >= 1000 * 32 * 2 + 1000 * 256 * 4
+    assert lib.more_route_unfused_scratch_bytes(-1, 32, 256) == 0
+    P = ctypes.c_void_p
+    # too little scratch
+    st = lib.more_route_unfused(P(16), P(16), P(16), 1000, 64, 32, 256, 4, P(16), P(16), P(16), None, P(16),
+                                n - 1, None)
+    assert st == 1
+
+
+def test_package_refuses_to_run_without_the_library(monkeypatch, tmp_path):
+    """The binding has no fallback: a missing nvcc and library means import fails."""
+    import importlib
+    import sys
+    import mixture_experts_rank_b200._build as b
+    monkeypatch.setattr(b, "LIB", str(tmp_path / "missing.so"))
+    monkeypatch.setenv("NVCC", str(tmp_path / "no-nvcc"))
+    monkeypatch.setattr(b.shutil, "which", lambda _: None)
+    monkeypatch.setattr(b.os.path, "exists", lambda p: False)
+    saved = sys.modules.pop("mixture_experts_rank_b200")
+    try:
+        with pytest.raises(RuntimeError):
+            importlib.import_module("mixture_experts_rank_b200")
+    finally:
+        sys.modules["mixture_experts_rank_b200"] = saved
