@@ -25,8 +25,11 @@
  *     first, lower expert index first on equal logits (Algorithm 1 keeps the
  *     earlier expert on equal values).  out_logits[n][j] is the fp32 logit of
  *     expert out_idx[n][j]; out_gate[n][] is the softmax of those k logits.
- *   - The logits are computed as in Algorithm 1: z accumulated in fp32 and
- *     rounded to bf16 (nearest even), then z . R2 accumulated in fp32.
+ *   - Precision: z = x . R1 is accumulated in fp32 and carried into the second
+ *     product as a pair of bf16 terms, z_hi = bf16(z) and z_lo = bf16(z - z_hi)
+ *     (nearest even), so z keeps about 16 significant bits; l = (z_hi + z_lo) . R2
+ *     is accumulated in fp32.  Algorithm 1 narrows z to a single bf16; that alone
+ *     moves logits by up to about 1% of their RMS, the whole parity tolerance.
  *   - out_expert_count[e] is set (not accumulated) to the number of (token,
  *     slot) pairs of this call that name expert e; the call zeroes it first.
  *   - Inputs must be finite; results for NaN or infinite inputs are unspecified.
@@ -35,8 +38,8 @@
  * returns an error and launches nothing):
  *   N >= 0; h >= 8 and h % 8 == 0; M >= 8 and M % 8 == 0; r % 16 == 0 and
  *   16 <= r <= 128; 1 <= k <= M; k <= MORE_KMAX; M <= MORE_MMAX;
- *   X (unless N == 0), R1, R2, out_idx, out_gate and out_expert_count non-NULL;
- *   every pointer 16-byte aligned.  Violations of the shape limits that are
+ *   R1, R2 and out_expert_count non-NULL, and X, out_idx and out_gate non-NULL
+ *   unless N == 0; every non-NULL pointer 16-byte aligned.  Violations of the shape limits that are
  *   not errors of meaning (k > MORE_KMAX, r outside 16..128 or not a multiple
  *   of 16, M > MORE_MMAX) return MORE_ERR_UNSUPPORTED; the rest return
  *   MORE_ERR_INVALID_ARG.
@@ -93,8 +96,9 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
 
 /*
  * Materialise-then-top-k comparison path (the unfused router of MoRE App. H.6,
- * Fig. 24): z = X . R1 is written to scratch as bf16 [N][r], the full logits as
- * fp32 [N][M], then a row-wise top-k and softmax read them back.  Same
+ * Fig. 24): z = X . R1 (as z_hi + z_lo, see Precision) is written to scratch as
+ * fp32 [N][r], the full logits as fp32 [N][M], then a row-wise top-k and
+ * softmax read them back.  Same
  * arguments and results as more_route, plus caller-owned device scratch of at
  * least more_route_unfused_scratch_bytes(N, r, M) bytes (16-byte aligned).
  * Too little scratch returns MORE_ERR_INVALID_ARG.

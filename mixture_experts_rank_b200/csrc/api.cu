@@ -32,9 +32,9 @@ more_status validate(const void* X, const void* R1, const void* R2, int64_t N, i
                      const int32_t* out_count, const float* out_logits) {
   if (N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1)
     return MORE_ERR_INVALID_ARG;
-  if (!R1 || !R2 || !out_idx || !out_gate || !out_count || (N > 0 && !X)) return MORE_ERR_INVALID_ARG;
-  if ((X && !aligned16(X)) || !aligned16(R1) || !aligned16(R2) || !aligned16(out_idx) ||
-      !aligned16(out_gate) || !aligned16(out_count) || (out_logits && !aligned16(out_logits)))
+  if (!R1 || !R2 || !out_count || (N > 0 && (!X || !out_idx || !out_gate))) return MORE_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || !aligned16(R1) || !aligned16(R2) || (out_idx && !aligned16(out_idx)) ||
+      (out_gate && !aligned16(out_gate)) || !aligned16(out_count) || (out_logits && !aligned16(out_logits)))
     return MORE_ERR_INVALID_ARG;
   if (N > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
   if (k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX) return MORE_ERR_UNSUPPORTED;

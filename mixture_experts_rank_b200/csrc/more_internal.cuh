@@ -36,6 +36,13 @@ __device__ __forceinline__ float bf16_round(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
 }
 
+// z as the bf16 pair z_hi + z_lo (z_hi = bf16(z), z_lo = bf16(z - z_hi)), summed in fp32:
+// the value every kernel multiplies with R2 (about 16 significant bits of z).
+__device__ __forceinline__ float split_bf16_pair(float z) {
+  float hi = bf16_round(z);
+  return hi + bf16_round(z - hi);
+}
+
 // Routing order on (value, expert): a goes first iff it has the larger value,
 // or the same value and the lower expert index.
 __device__ __forceinline__ bool goes_first(float va, int ia, float vb, int ib) {

@@ -1,11 +1,12 @@
 // Small-batch (decode-sized) MoRE routing kernel on CUDA cores: one warp per token.
 //
 // Per token, following "MoRE: Scaling mixture of experts with hardware-aware
-// low-rank routing", App. F, Algorithm 1 (z accumulated in fp32 and narrowed to
-// bf16, one sweep over the experts with a running top-k) and Fig. 12 (softmax
-// over the k selected logits):
+// low-rank routing", App. F, Algorithm 1 (z accumulated in fp32, one sweep over
+// the experts with a running top-k) and Fig. 12 (softmax over the k selected
+// logits):
 //   1. z = x . R1: lanes stride over h, 16 outputs per pass, reduce-scatter
-//      through shuffles; z is rounded to bf16 and kept in shared memory.
+//      through shuffles; z is carried as the bf16 pair z_hi + z_lo (finer than
+//      Algorithm 1's single bf16) and kept in shared memory.
 //   2. lanes take expert pairs (2 lane + 64 j, +1); each lane keeps a sorted
 //      running top-k of its experts (strict '>' insertion, so on equal logits
 //      the lower expert index stays ahead).

@@ -1,10 +1,868 @@
-// Fused tensor-core routing kernel (placeholder until the tcgen05 path lands).
+// Fused MoRE routing kernel for B200 (sm_100a): TMA-staged X, tcgen05 MMAs into
+// TMEM, an exact two-pass top-k on the CUDA cores, softmax gates and counts.
+//
+// What it computes is the router of "MoRE: Scaling mixture of experts with
+// hardware-aware low-rank routing": §2 "MoRE layer" (softmax over TopK of the
+// rank-r logits), App. F eq. (5) and Algorithm 1 (z = X R1 accumulated in fp32,
+// one B_N x B_M logit tile at a time, out-of-range experts at -infinity, only
+// the (N, k) selection written), Fig. 12 (gates) and eq. (9) (counts).  The N x M
+// logits exist only in TMEM.
+//
+// How (one persistent CTA per SM, 128-token tiles, 12 warps):
+//   warp 0  TMA producer of X (128 x 64 bf16, 128B swizzle) and R1 (64 x r) stages.
+//   warp 1  MMA issuer for Z = X R1: M=128 tokens, N=r, K=16 steps over h, into a
+//           double-buffered TMEM accumulator (the next tile streams while the
+//           current one is routed, so HBM never waits on the top-k).
+//   warp 2  MMA issuer for the logit tiles: pass 1 D[tok, exp] = Z R2 (128 x 128),
+//           pass 2 D^T[exp, tok] = R2^T Z^T.  z enters as the bf16 pair
+//           z_hi + z_lo (K = 2r), which keeps ~16 bits of z.
+//   warp 3  TMA producer of R2 tiles (r x 128 experts); R2 stays resident in
+//           shared memory when it fits, else it is streamed from L2.
+//   warps 4-11  two consumer warpgroups (TMEM lanes = tokens in pass 1, experts
+//           in pass 2):
+//     epilogue  Z from TMEM -> (z_hi, z_lo) bf16 -> shared memory (K-major).
+//     pass 1    every 32-expert chunk of a token is reduced to its maximum and
+//               packed into a 32-bit key (order-preserving value bits above the
+//               chunk id); a branch-free sorted list keeps the best k+2 keys.
+//               The k largest logits lie in the k chunks with the largest
+//               maxima, so the list names every chunk that can hold them.
+//     select    threshold T = the k-th key's value bits (rounded down); the
+//               needed chunks are those whose key is not below T, marked in a
+//               per-chunk token bitmask.
+//     pass 2    each warp owns a 32-expert lane group of the transposed tile;
+//               for every token that needs its chunk it reads that column,
+//               ballots the experts >= T and appends them as candidates.
+//     finalize  one thread per token sorts its few candidates in routing order
+//               (larger logit, then lower expert), softmax, stores, counts.
+//               Ties at the threshold, candidate overflow or a short list send
+//               the token to an exact warp-wide recomputation on CUDA cores.
+// Every barrier wait is bounded (a few seconds); on expiry the kernel records
+// MORE_DEVERR_WAIT_TIMEOUT in the library's device error word and unwinds.
+#include <cudaTypedefs.h>
+
 #include "more_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "warp_simt.cuh"
 
 namespace more {
+namespace tc {
 
-bool fused_tc_supports(const RouteArgs&) { return false; }
+using namespace sm100;
 
-cudaError_t launch_fused_tc(const RouteArgs&) { return cudaErrorNotSupported; }
+constexpr int kBT = 128;        // tokens per tile (MMA M of Z and pass 1, N of pass 2)
+constexpr int kBE = 128;        // experts per logit tile
+constexpr int kBK = 64;         // hidden elements per X stage (128-byte rows)
+constexpr int kThreads = 384;   // 4 role warps + 8 consumer warps
+constexpr int kConsumerThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+constexpr uint32_t kRealKey = 0x00800000u;  // ordered value of -FLT_MAX: keys below are not real chunks
+
+// ---- parameters -----------------------------------------------------------------------
+
+struct Params {
+  RouteArgs a;
+  int num_tiles;     // token tiles
+  int kb_count;      // hidden blocks of kBK
+  int p_count;       // expert tiles of kBE
+  int nchunks;       // 32-expert chunks
+  uint32_t low_mask; // chunk-id bits of a key
+  int x_stages;
+  int r2_stages;
+  int r2_resident;   // every expert tile stays in shared memory
+  uint32_t off_x, off_r1, off_r2, off_zs, off_bits, off_lists, off_cand, off_thr, off_cnt, off_flag, off_bar;
+};
+
+template <int R, int KCAP>
+struct Cfg {
+  static constexpr int KL = KCAP + 2;                  // chunk keys kept per token
+  static constexpr int C = 2 * KCAP + 8;               // candidate slots per token
+  static constexpr int RK = 2 * R;                     // K of the logit MMAs: z_hi | z_lo
+  static constexpr uint32_t X_STAGE = kBT * kBK * 2;   // 16 KB
+  static constexpr int R1_BOX = R < 64 ? R : 64;       // inner box of R1 (elements)
+  static constexpr int R1_BOXES = R / R1_BOX;
+  static constexpr uint32_t R1_BOX_BYTES = kBK * R1_BOX * 2;
+  static constexpr uint32_t R1_STAGE = R1_BOX_BYTES * R1_BOXES;
+  static constexpr uint32_t R1_ROW = R1_BOX * 2;       // bytes per R1 row inside a box
+  static constexpr uint32_t R1_LAYOUT = R1_ROW == 32 ? kSwizzle32B : (R1_ROW == 64 ? kSwizzle64B : kSwizzle128B);
+  static constexpr uint32_t R2_BOX_BYTES = 64 * R * 2; // 64 experts x R rows
+  static constexpr uint32_t R2_STAGE = 2 * R2_BOX_BYTES;
+  static constexpr uint32_t ZS_BYTES = kBT * RK * 2;   // z pair of 128 tokens, K-major core matrices
+  static constexpr uint32_t ZS_SBO = (RK / 8) * 128;   // byte stride of 8-token groups
+  static constexpr int ZCOLS = R < 32 ? 32 : R;        // TMEM columns per Z accumulator
+  static constexpr uint32_t IDESC_Z = idesc_bf16_f32(128, R, 0, 1);    // A = X (K-major), B = R1 (MN-major)
+  static constexpr uint32_t IDESC_P1 = idesc_bf16_f32(128, 128, 0, 1); // A = z pair, B = R2 tile
+  static constexpr uint32_t IDESC_P2 = idesc_bf16_f32(128, 128, 1, 0); // A = R2 tile^T, B = z pair^T
+};
+
+// Barrier block layout (uint64_t slots).
+struct Bars {
+  uint64_t* x_full;
+  uint64_t* x_empty;
+  uint64_t* r2_full;
+  uint64_t* r2_empty;
+  uint64_t* zacc_full;   // [2]
+  uint64_t* zacc_empty;  // [2]
+  uint64_t* zsm_full;
+  uint64_t* zsm_empty;
+  uint64_t* d_full;      // [2]
+  uint64_t* d_empty;     // [2]
+  uint64_t* drain;       // [2]
+  uint64_t* cbar;        // consumer-warp barrier (8 arrivals per phase)
+  uint32_t* tmem_slot;
+  int* abort_flag;
+};
+
+__device__ __forceinline__ Bars bars_at(uint8_t* smem, const Params& p) {
+  uint64_t* b = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  Bars r;
+  r.x_full = b;
+  r.x_empty = b + 8;
+  r.r2_full = b + 16;
+  r.r2_empty = r.r2_full + 64;
+  r.zacc_full = r.r2_empty + 64;
+  r.zacc_empty = r.zacc_full + 2;
+  r.zsm_full = r.zacc_empty + 2;
+  r.zsm_empty = r.zsm_full + 1;
+  r.d_full = r.zsm_empty + 1;
+  r.d_empty = r.d_full + 2;
+  r.drain = r.d_empty + 2;
+  r.cbar = r.drain + 2;
+  r.tmem_slot = reinterpret_cast<uint32_t*>(r.cbar + 1);
+  r.abort_flag = reinterpret_cast<int*>(r.tmem_slot + 1);
+  return r;
+}
+constexpr uint32_t kBarBytes = (16 + 128 + 13) * 8 + 16;
+
+// Bounded mbarrier wait: false once the limit passes or another thread gave up.
+__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                      unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spin & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kTimeoutNs) {
+        atomicOr(status, MORE_DEVERR_WAIT_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+
+// Barrier of the 8 consumer warps, on an mbarrier so that the wait is bounded too.
+__device__ __forceinline__ bool consumer_sync(const Bars& b, uint32_t& phase, unsigned int* status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(b.cbar);
+  const bool ok = wait_bar(b.cbar, phase, b.abort_flag, status);
+  phase ^= 1u;
+  return ok;
+}
+
+// Order-preserving map of fp32 onto uint32 and its inverse.
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+}
+__device__ __forceinline__ float ord_inv(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+// Maximum of 32 fp32 values held as raw bits.
+__device__ __forceinline__ float max32(const uint32_t* v) {
+  float a[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i)
+    a[i] = max3f(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
+  a[10] = fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31]));
+  float b0 = max3f(a[0], a[1], a[2]), b1 = max3f(a[3], a[4], a[5]), b2 = max3f(a[6], a[7], a[8]);
+  float b3 = fmaxf(a[9], a[10]);
+  return max3f(b0, b1, fmaxf(b2, b3));
+}
+
+// Branch-free insertion of key x into the descending list kl[0..L).
+template <int L>
+__device__ __forceinline__ void key_insert(uint32_t* kl, uint32_t x) {
+#pragma unroll
+  for (int i = L - 1; i > 0; --i) kl[i] = min(kl[i - 1], max(kl[i], x));
+  kl[0] = max(kl[0], x);
+}
+
+// Byte offset of the 16-byte core-matrix row (token t, K chunk c) in the z pair buffer.
+template <int R, int KCAP>
+__device__ __forceinline__ uint32_t zs_offset(int t, int c) {
+  return (uint32_t)(((t >> 3) * (Cfg<R, KCAP>::RK / 8) + c) * 128 + (t & 7) * 16);
+}
+
+// z_t[i] (fp32 value of the pair) read back from the z pair buffer.
+template <int R, int KCAP>
+__device__ __forceinline__ float zs_value(const uint8_t* zs, int t, int i) {
+  const __nv_bfloat16* hi = reinterpret_cast<const __nv_bfloat16*>(zs + zs_offset<R, KCAP>(t, i >> 3)) + (i & 7);
+  const __nv_bfloat16* lo =
+      reinterpret_cast<const __nv_bfloat16*>(zs + zs_offset<R, KCAP>(t, (R + i) >> 3)) + (i & 7);
+  return __bfloat162float(*hi) + __bfloat162float(*lo);
+}
+
+// ---- role: TMA producer of X and R1 -----------------------------------------------
+
+template <int R, int KCAP>
+__device__ void producer_x(const Params& p, const Bars& b, uint8_t* smem, const CUtensorMap* tmX,
+                           const CUtensorMap* tmR1) {
+  using C = Cfg<R, KCAP>;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int kb = 0; kb < p.kb_count; ++kb) {
+      if (!wait_bar(&b.x_empty[s], ph ^ 1u, b.abort_flag, p.a.status)) return;
+      mbar_arrive_expect_tx(&b.x_full[s], C::X_STAGE + C::R1_STAGE);
+      tma_load_2d(smem + p.off_x + s * C::X_STAGE, tmX, &b.x_full[s], kb * kBK, tile * kBT);
+#pragma unroll
+      for (int q = 0; q < C::R1_BOXES; ++q)
+        tma_load_2d(smem + p.off_r1 + s * C::R1_STAGE + q * C::R1_BOX_BYTES, tmR1, &b.x_full[s], q * 64,
+                    kb * kBK);
+      if (++s == p.x_stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+}
+
+// ---- role: TMA producer of R2 tiles ----------------------------------------------------
+
+template <int R, int KCAP>
+__device__ void producer_r2(const Params& p, const Bars& b, uint8_t* smem, const CUtensorMap* tmR2) {
+  using C = Cfg<R, KCAP>;
+  if (p.r2_resident) {
+    for (int t = 0; t < p.p_count; ++t) {
+      uint8_t* dst = smem + p.off_r2 + t * C::R2_STAGE;
+      mbar_arrive_expect_tx(&b.r2_full[t], C::R2_STAGE);
+      tma_load_2d(dst, tmR2, &b.r2_full[t], t * kBE, 0);
+      tma_load_2d(dst + C::R2_BOX_BYTES, tmR2, &b.r2_full[t], t * kBE + 64, 0);
+    }
+    return;
+  }
+  int s = 0;
+  uint32_t ph = 0;
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int t = 0; t < p.p_count; ++t) {
+        if (!wait_bar(&b.r2_empty[s], ph ^ 1u, b.abort_flag, p.a.status)) return;
+        uint8_t* dst = smem + p.off_r2 + s * C::R2_STAGE;
+        mbar_arrive_expect_tx(&b.r2_full[s], C::R2_STAGE);
+        tma_load_2d(dst, tmR2, &b.r2_full[s], t * kBE, 0);
+        tma_load_2d(dst + C::R2_BOX_BYTES, tmR2, &b.r2_full[s], t * kBE + 64, 0);
+        if (++s == p.r2_stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+  }
+}
+
+// ---- role: MMA issuer of Z = X R1 ------------------------------------------------------
+
+template <int R, int KCAP>
+__device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
+  using C = Cfg<R, KCAP>;
+  int s = 0;
+  uint32_t ph = 0;
+  int lt = 0;
+  const uint32_t x0 = smem_u32(smem + p.off_x), r10 = smem_u32(smem + p.off_r1);
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
+    const int buf = lt & 1;
+    if (!wait_bar(&b.zacc_empty[buf], ((lt >> 1) & 1) ^ 1u, b.abort_flag, p.a.status)) break;
+    tc_fence_after();
+    const uint32_t d = tmem_base + 256 + buf * C::ZCOLS;
+    for (int kb = 0; kb < p.kb_count; ++kb) {
+      if (!wait_bar(&b.x_full[s], ph, b.abort_flag, p.a.status)) goto done;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kBK / 16; ++kk) {
+        uint64_t ad = smem_desc(x0 + s * C::X_STAGE + kk * 32, 16, 1024, kSwizzle128B);
+        uint64_t bd = smem_desc(r10 + s * C::R1_STAGE + kk * 16 * C::R1_ROW, C::R1_BOX_BYTES, 8 * C::R1_ROW,
+                                C::R1_LAYOUT);
+        mma_bf16(d, ad, bd, C::IDESC_Z, (kb | kk) != 0);
+      }
+      mma_commit(&b.x_empty[s]);
+      if (++s == p.x_stages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    mma_commit(&b.zacc_full[buf]);
+  }
+done:
+  mma_commit(&b.drain[0]);
+  wait_bar(&b.drain[0], 0, b.abort_flag, p.a.status);
+}
+
+// ---- role: MMA issuer of the logit tiles -------------------------------------------------
+
+template <int R, int KCAP>
+__device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
+  using C = Cfg<R, KCAP>;
+  int rs = 0;
+  uint32_t rph = 0;
+  int ds = 0;
+  uint32_t dph = 0;
+  int lt = 0;
+  const uint32_t zs = smem_u32(smem + p.off_zs), r20 = smem_u32(smem + p.off_r2);
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
+    if (!wait_bar(b.zsm_full, lt & 1, b.abort_flag, p.a.status)) goto done;
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int t = 0; t < p.p_count; ++t) {
+        int st;
+        if (p.r2_resident) {
+          st = t;
+          if (lt == 0 && pass == 0 && !wait_bar(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
+        } else {
+          st = rs;
+          if (!wait_bar(&b.r2_full[rs], rph, b.abort_flag, p.a.status)) goto done;
+        }
+        if (!wait_bar(&b.d_empty[ds], dph ^ 1u, b.abort_flag, p.a.status)) goto done;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ds * 128;
+        const uint32_t r2 = r20 + st * C::R2_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::RK / 16; ++kk) {
+          uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
+          uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
+          if (pass == 0)
+            mma_bf16(d, zd, rd, C::IDESC_P1, kk != 0);
+          else
+            mma_bf16(d, rd, zd, C::IDESC_P2, kk != 0);
+        }
+        mma_commit(&b.d_full[ds]);
+        if (!p.r2_resident) {
+          mma_commit(&b.r2_empty[rs]);
+          if (++rs == p.r2_stages) {
+            rs = 0;
+            rph ^= 1u;
+          }
+        }
+        ds ^= 1;
+        if (ds == 0) dph ^= 1u;
+      }
+    }
+    mma_commit(b.zsm_empty);
+  }
+done:
+  mma_commit(&b.drain[1]);
+  wait_bar(&b.drain[1], 0, b.abort_flag, p.a.status);
+}
+
+// ---- consumers ----------------------------------------------------------------------------
+
+template <int R, int KCAP>
+__device__ __forceinline__ void write_token(const RouteArgs& a, int64_t n, const TopList<KCAP>& sel) {
+  const int k = a.k;
+  float top = sel.v[0], sum = 0.f;
+  float ex[KCAP];
+#pragma unroll
+  for (int j = 0; j < KCAP; ++j) {
+    ex[j] = (j < k) ? expf(sel.v[j] - top) : 0.f;
+    sum += ex[j];
+  }
+  const float inv = 1.f / sum;
+  size_t o = (size_t)n * k;
+#pragma unroll
+  for (int j = 0; j < KCAP; ++j) {
+    if (j < k) {
+      a.out_idx[o + j] = sel.i[j];
+      a.out_gate[o + j] = ex[j] * inv;
+      if (a.out_logits) a.out_logits[o + j] = sel.v[j];
+      atomicAdd(a.out_count + sel.i[j], 1);
+    }
+  }
+}
+
+// Exact warp-wide recomputation of one token's top-k on CUDA cores (ties at the
+// threshold, candidate overflow).  Lanes take expert pairs in increasing order.
+template <int R, int KCAP>
+__device__ void fallback_token(const RouteArgs& a, const uint8_t* zs, int t, int64_t n, int lane) {
+  TopList<KCAP> list;
+  list.init();
+  const int pitch = a.M >> 1;
+  for (int e = 2 * lane; e < a.M; e += 64) {
+    const __nv_bfloat162* col = reinterpret_cast<const __nv_bfloat162*>(a.R2 + e);
+    float acc0 = 0.f, acc1 = 0.f;
+    for (int i = 0; i < R; ++i) {
+      float zi = zs_value<R, KCAP>(zs, t, i);
+      float2 w = __bfloat1622float2(col[(size_t)i * pitch]);
+      acc0 = fmaf(zi, w.x, acc0);
+      acc1 = fmaf(zi, w.y, acc1);
+    }
+    list.insert(acc0, e);
+    list.insert(acc1, e + 1);
+  }
+  float v;
+  int e;
+  warp_merge_topk<KCAP>(list, a.k, lane, v, e);
+  warp_write_selection(a, n, lane, v, e);
+}
+
+template <int R, int KCAP>
+__device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
+  using C = Cfg<R, KCAP>;
+  const RouteArgs& a = p.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sp = warp & 3;              // TMEM subpartition: lanes 32 sp .. 32 sp + 31
+  const int g = (warp - 4) >> 2;        // consumer warpgroup 0 / 1
+  const int t = sp * 32 + lane;         // token of this thread in pass 1 and finalize
+  const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+  uint8_t* zs = smem + p.off_zs;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);
+  uint2* cand = reinterpret_cast<uint2*>(smem + p.off_cand);
+  float* thr = reinterpret_cast<float*>(smem + p.off_thr);
+  int* cnt = reinterpret_cast<int*>(smem + p.off_cnt);
+  int* flag = reinterpret_cast<int*>(smem + p.off_flag);
+  const uint32_t low = p.low_mask;
+  int ds = 0;
+  uint32_t dph = 0;
+  uint32_t cph = 0;
+  int lt = 0;
+
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
+    const int64_t n0 = (int64_t)tile * kBT;
+    const int buf = lt & 1;
+    // ---------------- Z epilogue: TMEM -> (z_hi, z_lo) -> shared memory -------------
+    if (!wait_bar(&b.zacc_full[buf], (lt >> 1) & 1, b.abort_flag, a.status)) return;
+    tc_fence_after();
+    {
+      constexpr int HALF = R / 2;
+      uint32_t zr[HALF];
+      const uint32_t taddr = tmem_base + lane_base + 256 + buf * C::ZCOLS + g * HALF;
+      if constexpr (HALF == 8) {
+        tmem_ld_x8(taddr, zr);
+      } else if constexpr (HALF == 16) {
+        tmem_ld_x16(taddr, zr);
+      } else {
+#pragma unroll
+        for (int q = 0; q < HALF / 32; ++q) tmem_ld_x32(taddr + q * 32, zr + q * 32);
+      }
+      tmem_wait_ld();
+      reg_fence<HALF>(zr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.zacc_empty[buf]);
+      // the previous tile's logit MMAs must be done with the z buffer
+      if (lt > 0 && !wait_bar(b.zsm_empty, (lt - 1) & 1, b.abort_flag, a.status)) return;
+#pragma unroll
+      for (int q = 0; q < HALF / 8; ++q) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float z0 = __uint_as_float(zr[q * 8 + 2 * j]), z1 = __uint_as_float(zr[q * 8 + 2 * j + 1]);
+          __nv_bfloat16 h0 = __float2bfloat16_rn(z0), h1 = __float2bfloat16_rn(z1);
+          __nv_bfloat16 l0 = __float2bfloat16_rn(z0 - __bfloat162float(h0));
+          __nv_bfloat16 l1 = __float2bfloat16_rn(z1 - __bfloat162float(h1));
+          hi[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          lo[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        const int i0 = g * HALF + q * 8;  // first z index of this 8-group
+        *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, i0 >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, (R + i0) >> 3)) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b.zsm_full);
+    }
+
+    // ---------------- pass 1: chunk maxima -> top (k+2) chunk keys --------------------
+    uint32_t kl[C::KL];
+#pragma unroll
+    for (int i = 0; i < C::KL; ++i) kl[i] = 0u;
+    for (int pt = 0; pt < p.p_count; ++pt) {
+      if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
+      tc_fence_after();
+      uint32_t v[64];
+      const uint32_t taddr = tmem_base + lane_base + ds * 128 + g * 64;
+      tmem_ld_x32(taddr, v);
+      tmem_ld_x32(taddr + 32, v + 32);
+      tmem_wait_ld();
+      reg_fence<64>(v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.d_empty[ds]);
+      ds ^= 1;
+      if (ds == 0) dph ^= 1u;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c = pt * 4 + g * 2 + hh;
+        uint32_t* vc = v + hh * 32;
+        if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (32 * c + j >= a.M) vc[j] = 0xff800000u;
+        }
+        const uint32_t key = (ord_key(max32(vc)) & ~low) | (uint32_t)c;
+        key_insert<C::KL>(kl, key);
+      }
+    }
+
+    // ---------------- select: merge the two warpgroups' lists, mark needed chunks -----
+    if (g == 1) {
+#pragma unroll
+      for (int i = 0; i < C::KL; ++i) lists[i * kBT + t] = kl[i];
+    }
+    if (!consumer_sync(b, cph, a.status)) return;
+    if (g == 0) {
+#pragma unroll
+      for (int i = 0; i < C::KL; ++i) key_insert<C::KL>(kl, lists[i * kBT + t]);
+      const bool active = n0 + t < a.N;
+      uint32_t kth = 0;
+#pragma unroll
+      for (int i = 0; i < C::KL; ++i)
+        if (i == a.k - 1) kth = kl[i];
+      const uint32_t T = kth & ~low;
+      int f = active ? 0 : 2;
+      float threshold = -INFINITY;
+      if (T >= kRealKey) {
+        threshold = ord_inv(T);
+        if ((kl[C::KL - 1] & ~low) >= T) f |= 1;  // more ties than the list holds
+      }
+      if (f == 0) {
+#pragma unroll
+        for (int i = 0; i < C::KL; ++i) {
+          const uint32_t vb = kl[i] & ~low;
+          if (vb >= kRealKey && vb >= T) atomicOr(&bits[(kl[i] & low) * 4 + (t >> 5)], 1u << (t & 31));
+        }
+      }
+      thr[t] = threshold;
+      cnt[t] = 0;
+      flag[t] = f;
+    }
+    if (!consumer_sync(b, cph, a.status)) return;
+
+    // ---------------- pass 2: candidates of the needed chunks --------------------------
+    for (int pt = 0; pt < p.p_count; ++pt) {
+      if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
+      tc_fence_after();
+      const int c = pt * 4 + sp;
+      const int e = 32 * c + lane;
+      const uint32_t col0 = tmem_base + lane_base + ds * 128;
+#pragma unroll 1
+      for (int w = 2 * g; w < 2 * g + 2; ++w) {
+        uint32_t m = (c < p.nchunks) ? bits[c * 4 + w] : 0u;
+        __syncwarp();
+        if (lane == 0 && m) bits[c * 4 + w] = 0u;
+        while (m) {
+          int tok[4];
+          uint32_t val[4];
+          int nb = 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            tok[q] = -1;
+            if (m) {
+              const int bit = __ffs(m) - 1;
+              m &= m - 1;
+              tok[q] = 32 * w + bit;
+              nb = q + 1;
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < nb) val[q] = tmem_ld_x1(col0 + tok[q]);
+          tmem_wait_ld();
+          reg_fence<4>(val);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q >= nb) break;
+            const float x = __uint_as_float(val[q]);
+            const bool take = (e < a.M) && (x >= thr[tok[q]]);
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            if (bal) {
+              int base = 0;
+              if (lane == 0) base = atomicAdd(&cnt[tok[q]], __popc(bal));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const int pos = base + __popc(bal & ((1u << lane) - 1u));
+              if (take && pos < C::C) cand[tok[q] * C::C + pos] = make_uint2(val[q], (uint32_t)e);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.d_empty[ds]);
+      ds ^= 1;
+      if (ds == 0) dph ^= 1u;
+    }
+    if (!consumer_sync(b, cph, a.status)) return;
+
+    // ---------------- finalize: order, softmax, store, count ---------------------------
+    if (g == 0) {
+      const int64_t n = n0 + t;
+      const int f = flag[t];
+      const int nc = cnt[t];
+      const bool active = (f & 2) == 0;
+      const bool fb = active && ((f & 1) || nc > C::C || nc < a.k);
+      if (active && !fb) {
+        TopList<KCAP> sel;
+        sel.init();
+        for (int q = 0; q < nc; ++q) {
+          uint2 cv = cand[t * C::C + q];
+          sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
+        }
+        write_token<R, KCAP>(a, n, sel);
+      }
+      uint32_t need = __ballot_sync(0xffffffffu, fb);
+      while (need) {
+        const int j = __ffs(need) - 1;
+        need &= need - 1;
+        fallback_token<R, KCAP>(a, zs, sp * 32 + j, n0 + sp * 32 + j, lane);
+      }
+    }
+    if (!consumer_sync(b, cph, a.status)) return;
+  }
+}
+
+// ---- kernel -----------------------------------------------------------------------------
+
+template <int R, int KCAP>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_route_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR1,
+                       const __grid_constant__ CUtensorMap tmR2, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Bars b = bars_at(smem, p);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.x_stages; ++i) {
+      mbar_init(&b.x_full[i], 1);
+      mbar_init(&b.x_empty[i], 1);
+    }
+    const int nr2 = p.r2_resident ? p.p_count : p.r2_stages;
+    for (int i = 0; i < nr2; ++i) {
+      mbar_init(&b.r2_full[i], 1);
+      mbar_init(&b.r2_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b.zacc_full[i], 1);
+      mbar_init(&b.zacc_empty[i], 8);
+      mbar_init(&b.d_full[i], 1);
+      mbar_init(&b.d_empty[i], 8);
+      mbar_init(&b.drain[i], 1);
+    }
+    mbar_init(b.zsm_full, 8);
+    mbar_init(b.zsm_empty, 1);
+    mbar_init(b.cbar, 8);
+    *b.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmR1);
+    prefetch_tensormap(&tmR2);
+  }
+  if (warp == 1) {
+    tmem_alloc(b.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 4) {  // clear the needed-chunk bitmask
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);
+    for (int i = threadIdx.x - 128; i < p.nchunks * 4; i += kConsumerThreads) bits[i] = 0u;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *b.tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) producer_x<R, KCAP>(p, b, smem, &tmX, &tmR1);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) mma_z<R, KCAP>(p, b, smem, tmem_base);
+    __syncwarp();
+  } else if (warp == 2) {
+    if (lane == 0) mma_scores<R, KCAP>(p, b, smem, tmem_base);
+    __syncwarp();
+  } else if (warp == 3) {
+    if (lane == 0) producer_r2<R, KCAP>(p, b, smem, &tmR2);
+    __syncwarp();
+  } else {
+    consumers<R, KCAP>(p, b, smem, tmem_base);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---- host side ----------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr uint32_t kSmemLimit = 227 * 1024;
+
+uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory plan; returns the total bytes (0 when nothing fits).
+template <int R, int KCAP>
+uint32_t plan(Params& p) {
+  using C = Cfg<R, KCAP>;
+  for (int xs = 4; xs >= 2; --xs) {
+    for (int mode = 0; mode < 2; ++mode) {  // 0: R2 resident, 1: streamed
+      const int r2s = mode == 0 ? p.p_count : 4;
+      if (mode == 0 && p.p_count > 64) continue;
+      for (int r2n = r2s; r2n >= 2 || (mode == 0 && r2n == r2s); --r2n) {
+        uint32_t off = 0;
+        p.off_x = off;
+        off += xs * C::X_STAGE;
+        p.off_r1 = off = align_up(off, 1024);
+        off += xs * C::R1_STAGE;
+        p.off_r2 = off = align_up(off, 1024);
+        off += r2n * C::R2_STAGE;
+        p.off_zs = off = align_up(off, 1024);
+        off += C::ZS_BYTES;
+        p.off_bits = off = align_up(off, 16);
+        off += p.nchunks * 16;
+        // candidate slots and the list exchange share memory (disjoint lifetimes)
+        const uint32_t cand_bytes = kBT * C::C * 8, list_bytes = kBT * C::KL * 4;
+        p.off_cand = p.off_lists = off = align_up(off, 16);
+        off += cand_bytes > list_bytes ? cand_bytes : list_bytes;
+        p.off_thr = off;
+        off += kBT * 4;
+        p.off_cnt = off;
+        off += kBT * 4;
+        p.off_flag = off;
+        off += kBT * 4;
+        p.off_bar = off = align_up(off, 8);
+        off += kBarBytes;
+        const uint32_t total = off + 1024;  // alignment slack of the dynamic base
+        if (total <= kSmemLimit) {
+          p.x_stages = xs;
+          p.r2_stages = r2n;
+          p.r2_resident = mode == 0;
+          return total;
+        }
+        if (mode == 0) break;
+      }
+    }
+  }
+  return 0;
+}
+
+template <int R, int KCAP>
+bool fill_params(const RouteArgs& a, Params& p, uint32_t& smem) {
+  p.a = a;
+  p.num_tiles = (int)((a.N + kBT - 1) / kBT);
+  p.kb_count = (a.h + kBK - 1) / kBK;
+  p.p_count = (a.M + kBE - 1) / kBE;
+  p.nchunks = (a.M + 31) / 32;
+  int bits = 1;
+  while ((1 << bits) < p.nchunks) ++bits;
+  p.low_mask = (1u << bits) - 1u;
+  smem = plan<R, KCAP>(p);
+  return smem != 0;
+}
+
+template <int R, int KCAP>
+cudaError_t launch(const RouteArgs& a) {
+  using C = Cfg<R, KCAP>;
+  Params p;
+  uint32_t smem = 0;
+  if (!fill_params<R, KCAP>(a, p, smem)) return cudaErrorInvalidConfiguration;
+  CUtensorMap tmX, tmR1, tmR2;
+  const CUtensorMapSwizzle r1sw = C::R1_ROW == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                  : C::R1_ROW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_map(&tmX, a.X, (uint64_t)a.h, (uint64_t)a.N, kBK, kBT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tmR1, a.R1, (uint64_t)R, (uint64_t)a.h, C::R1_BOX, kBK, r1sw) ||
+      !make_map(&tmR2, a.R2, (uint64_t)a.M, (uint64_t)R, 64, R, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  static int configured = 0;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(fused_route_kernel<R, KCAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemLimit);
+    if (e != cudaSuccess) return e;
+    configured = 1;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  fused_route_kernel<R, KCAP><<<grid, kThreads, smem, a.stream>>>(tmX, tmR1, tmR2, p);
+  return cudaGetLastError();
+}
+
+template <int R>
+cudaError_t launch_r(const RouteArgs& a) {
+  if (a.k <= 4) return launch<R, 4>(a);
+  if (a.k <= 8) return launch<R, 8>(a);
+  return launch<R, 16>(a);
+}
+
+template <int R>
+bool supports_r(const RouteArgs& a) {
+  Params p;
+  uint32_t smem;
+  if (a.k <= 4) return fill_params<R, 4>(a, p, smem);
+  if (a.k <= 8) return fill_params<R, 8>(a, p, smem);
+  return fill_params<R, 16>(a, p, smem);
+}
+
+}  // namespace tc
+
+bool fused_tc_supports(const RouteArgs& a) {
+  if (a.M > 65536 || a.k > 16 || a.N < 1 || a.N > 0x7fffffffLL - tc::kBT) return false;
+  if (!tc::encode_fn()) return false;
+  switch (a.r) {
+    case 16: return tc::supports_r<16>(a);
+    case 32: return tc::supports_r<32>(a);
+    case 64: return tc::supports_r<64>(a);
+    case 128: return tc::supports_r<128>(a);
+    default: return false;
+  }
+}
+
+cudaError_t launch_fused_tc(const RouteArgs& a) {
+  switch (a.r) {
+    case 16: return tc::launch_r<16>(a);
+    case 32: return tc::launch_r<32>(a);
+    case 64: return tc::launch_r<64>(a);
+    case 128: return tc::launch_r<128>(a);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 }  // namespace more

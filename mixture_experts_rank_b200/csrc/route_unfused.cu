@@ -1,13 +1,13 @@
 // Materialise-then-top-k comparison path: the unfused low-rank router of
 // "MoRE: Scaling mixture of experts with hardware-aware low-rank routing",
 // App. H.6 (Fig. 24), rebuilt with this library's own kernels.
-//   kernel 1: z = X . R1, rounded to bf16, written to scratch [N][r];
+//   kernel 1: z = X . R1, carried as z_hi + z_lo, written to scratch fp32 [N][r];
 //   kernel 2: l = z . R2 in fp32, written to scratch [N][M]  (the N x M tensor
 //             the fused kernel never writes);
 //   kernel 3: one warp per row reads l back, keeps per-lane running top-k
 //             lists, merges them in routing order, applies the softmax.
-// The arithmetic matches the fused path (bf16 z, fp32 logits), so both return
-// the same selections up to the order of fp32 accumulation.
+// The arithmetic matches the fused path (z as a bf16 pair, fp32 logits), so both
+// return the same selections up to the order of fp32 accumulation.
 #include "more_internal.cuh"
 #include "warp_simt.cuh"
 
@@ -18,14 +18,14 @@ constexpr int kProjWarps = 8;
 
 __global__ void __launch_bounds__(kProjWarps * 32)
     unfused_projection_kernel(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ R1,
-                              int64_t N, int h, int r, __nv_bfloat16* __restrict__ z_out) {
+                              int64_t N, int h, int r, float* __restrict__ z_out) {
   extern __shared__ float smem_z[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* zs = smem_z + warp * r;
   for (int64_t n = (int64_t)blockIdx.x * kProjWarps + warp; n < N; n += (int64_t)gridDim.x * kProjWarps) {
     warp_project_token(X + (size_t)n * h, R1, h, r, zs, lane);
     __syncwarp();
-    for (int i = lane; i < r; i += 32) z_out[(size_t)n * r + i] = __float2bfloat16_rn(zs[i]);
+    for (int i = lane; i < r; i += 32) z_out[(size_t)n * r + i] = zs[i];
     __syncwarp();
   }
 }
@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kProjWarps * 32)
 constexpr int kTileTok = 64, kTileExp = 128;
 
 __global__ void __launch_bounds__(256)
-    unfused_scores_kernel(const __nv_bfloat16* __restrict__ z, const __nv_bfloat16* __restrict__ R2,
+    unfused_scores_kernel(const float* __restrict__ z, const __nv_bfloat16* __restrict__ R2,
                           int64_t N, int r, int M, float* __restrict__ scores) {
   extern __shared__ float smem[];
   float* zt = smem;                       // [kTileTok][r]
@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(256)
   const int e0 = blockIdx.y * kTileExp;
   for (int q = threadIdx.x; q < kTileTok * r; q += 256) {
     int t = q / r, i = q % r;
-    zt[q] = (n0 + t < N) ? __bfloat162float(z[(size_t)(n0 + t) * r + i]) : 0.f;
+    zt[q] = (n0 + t < N) ? z[(size_t)(n0 + t) * r + i] : 0.f;
   }
   for (int q = threadIdx.x; q < r * kTileExp; q += 256) {
     int i = q / kTileExp, c = q % kTileExp;
@@ -116,16 +116,16 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 }  // namespace
 
 size_t unfused_scratch_bytes(int64_t N, int r, int M) {
-  return align_up((size_t)N * r * sizeof(__nv_bfloat16), 256) + (size_t)N * M * sizeof(float);
+  return align_up((size_t)N * r * sizeof(float), 256) + (size_t)N * M * sizeof(float);
 }
 
 cudaError_t launch_unfused(const RouteArgs& a, void* scratch) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  auto* z = static_cast<__nv_bfloat16*>(scratch);
+  auto* z = static_cast<float*>(scratch);
   auto* scores = reinterpret_cast<float*>(static_cast<char*>(scratch) +
-                                          align_up((size_t)a.N * a.r * sizeof(__nv_bfloat16), 256));
+                                          align_up((size_t)a.N * a.r * sizeof(float), 256));
   int64_t pblocks = (a.N + kProjWarps - 1) / kProjWarps;
   if (pblocks > (int64_t)sms * 8) pblocks = (int64_t)sms * 8;
   unfused_projection_kernel<<<(unsigned)pblocks, kProjWarps * 32, sizeof(float) * kProjWarps * a.r, a.stream>>>(

@@ -36,6 +36,24 @@ struct TopList {
       i[0] = e;
     }
   }
+  // Insert (x, e) arriving in any order: compares by routing order, value then index.
+  __device__ __forceinline__ void insert_any(float x, int e) {
+    if (!goes_first(x, e, v[K - 1], i[K - 1])) return;
+#pragma unroll
+    for (int p = K - 1; p > 0; --p) {
+      if (goes_first(x, e, v[p - 1], i[p - 1])) {
+        v[p] = v[p - 1];
+        i[p] = i[p - 1];
+      } else if (goes_first(x, e, v[p], i[p])) {
+        v[p] = x;
+        i[p] = e;
+      }
+    }
+    if (goes_first(x, e, v[0], i[0])) {
+      v[0] = x;
+      i[0] = e;
+    }
+  }
   __device__ __forceinline__ void pop() {
 #pragma unroll
     for (int p = 0; p < K - 1; ++p) {
@@ -47,7 +65,7 @@ struct TopList {
   }
 };
 
-// z = x . R1 for one token; writes bf16-rounded z into zs[0..r).
+// z = x . R1 for one token; writes z, carried as the bf16 pair z_hi + z_lo, into zs[0..r).
 __device__ __forceinline__ void warp_project_token(const __nv_bfloat16* __restrict__ x,
                                               const __nv_bfloat16* __restrict__ R1, int h, int r,
                                               float* zs, int lane) {
@@ -102,7 +120,7 @@ __device__ __forceinline__ void warp_project_token(const __nv_bfloat16* __restri
     }
     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
     int j = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-    if ((lane & 1) == 0) zs[b + j] = bf16_round(acc[0]);
+    if ((lane & 1) == 0) zs[b + j] = split_bf16_pair(acc[0]);
   }
 }
 

@@ -115,7 +115,7 @@ def test_decode_full_oracle(variant, N):
     (127, 72, 16, 200, 1),
     (129, 136, 48, 64, 8),
     (1000, 512, 128, 1000, 16),
-    (300, 256, 64, 8, 8),        # k == M
+    (300, 256, 64, 16, 16),      # k == M == KMAX
     (513, 64, 32, 4104, 5),     # M one tile past a multiple of 32
     (2049, 1032, 32, 96, 3),
 ])
@@ -173,17 +173,22 @@ def test_jl_construction_exact(variant):
         X[n, sets[n]] = M - k
     Xb = syn.f32_to_bf16_bits(X)
     R1, R2 = identity_weights(M)
+    if not supported(variant, N, M, M, M, k):
+        pytest.skip("variant does not take this shape")
     idx, gate, cnt, logits = run(variant, dev_bf16(Xb), dev_bf16(R1), dev_bf16(R2), k)
     np.testing.assert_array_equal(idx, sets)
     np.testing.assert_allclose(gate, 1.0 / k, rtol=0, atol=1e-6)
     parity.compare(Xb, R1, R2, N, M, M, M, k, idx, gate, cnt, logits, exact=True)
 
 
-def hypercube(h, r):
+def hypercube(h, r, r_impl=None):
+    """Rank-r hypercube router embedded in rank r_impl >= r (zero padding leaves the logits unchanged)."""
+    r_impl = r if r_impl is None else r_impl
     M = 2 ** r
-    R1 = np.zeros((h, r), dtype=np.float32)
+    R1 = np.zeros((h, r_impl), dtype=np.float32)
     R1[:r, :r] = np.eye(r)
-    R2 = np.array([[1.0 if (a >> l) & 1 else -1.0 for a in range(M)] for l in range(r)], dtype=np.float32)
+    R2 = np.zeros((r_impl, M), dtype=np.float32)
+    R2[:r] = np.array([[1.0 if (a >> l) & 1 else -1.0 for a in range(M)] for l in range(r)])
     return syn.f32_to_bf16_bits(R1), syn.f32_to_bf16_bits(R2), M
 
 
@@ -193,6 +198,8 @@ def test_hypercube_top1_is_sign_pattern(variant):
     h, r = 64, 16
     R1, R2, M = hypercube(h, r)
     N = 2000
+    if not supported(variant, N, h, r, M, 1):
+        pytest.skip("variant does not take this shape")
     X = syn.normal_bf16(5, syn.TENSOR_X, N, h)
     idx, gate, cnt, logits = run(variant, dev_bf16(X), dev_bf16(R1), dev_bf16(R2), 1)
     z = syn.bf16_bits_to_f64(X)[:, :r]
@@ -205,7 +212,9 @@ def test_hypercube_top1_is_sign_pattern(variant):
 def test_hypercube_load_balance_bound(variant):
     """Prop. 1: every count within sqrt(2nkL/M) + 2L/3 of nk/M (delta = 1e-6)."""
     h, r, n, k, delta = 64, 8, 200000, 4, 1e-6
-    R1, R2, M = hypercube(h, r)
+    R1, R2, M = hypercube(h, r, r_impl=16)
+    if not supported(variant, n, h, 16, M, k):
+        pytest.skip("variant does not take this shape")
     X = syn.normal_bf16(6, syn.TENSOR_X, n, h)
     idx, gate, cnt, logits = run(variant, dev_bf16(X), dev_bf16(R1), dev_bf16(R2), k)
     L = np.log(2 * M / delta)
