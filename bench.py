@@ -201,6 +201,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="override N (profiling a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -219,6 +220,8 @@ def main():
     import synthetic as syn
 
     N, h, r, M, k, unit = WORKLOADS[args.workload]
+    if args.tokens:
+        N = args.tokens
     # rank i routes tokens [i N, (i+1) N) of one synthetic token set (seed 0)
     Xh = syn.normal_bf16(0, syn.TENSOR_X, N * world, h, 1.0, unit, rank * N, N)
     R1h = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
@@ -331,7 +334,8 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": describe(args.workload), "N_per_gpu": N, "h": h, "r": r, "M": M, "k": k,
+                "config": {"workload": describe(args.workload) + (f" (N overridden to {N})" if args.tokens else ""),
+                           "N_per_gpu": N, "h": h, "r": r, "M": M, "k": k,
                            "variant": variant_used, "parallelism": f"token shards x{world}",
                            "l2": f"inputs larger than L2 (X = {x_bytes / 1e9:.2f} GB per GPU)"
                            if x_bytes > L2_BYTES else "inputs fit in L2; no flush (L2-warm)"},
