@@ -52,8 +52,10 @@ using namespace sm100;
 constexpr int kBT = 128;        // tokens per tile (MMA M of Z and pass 1, N of pass 2)
 constexpr int kBE = 128;        // experts per logit tile
 constexpr int kBK = 64;         // hidden elements per X stage (128-byte rows)
-constexpr int kThreads = 384;   // 4 role warps + 8 consumer warps
-constexpr int kConsumerThreads = 256;
+constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
+constexpr int kConsumerThreads = 512;
+constexpr int kConsumerWarps = 16;
+constexpr int kPairBatch = 8;   // TMEM column loads in flight per warp in pass 2
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint32_t kRealKey = 0x00800000u;  // ordered value of -FLT_MAX: keys below are not real chunks
@@ -70,13 +72,14 @@ struct Params {
   int x_stages;
   int r2_stages;
   int r2_resident;   // every expert tile stays in shared memory
-  uint32_t off_x, off_r1, off_r2, off_zs, off_bits, off_lists, off_cand, off_thr, off_cnt, off_flag, off_bar;
+  uint32_t off_x, off_r1, off_r2, off_zs, off_lists, off_cand, off_thr, off_flag, off_nq, off_pc, off_pairs,
+      off_ccount, off_cbase, off_scan, off_bar;
 };
 
 template <int R, int KCAP>
 struct Cfg {
   static constexpr int KL = KCAP + 2;                  // chunk keys kept per token
-  static constexpr int C = 2 * KCAP + 8;               // candidate slots per token
+  static constexpr int S = 2;                          // candidate slots per (token, needed chunk)
   static constexpr int RK = 2 * R;                     // K of the logit MMAs: z_hi | z_lo
   static constexpr uint32_t X_STAGE = kBT * kBK * 2;   // 16 KB
   static constexpr int R1_BOX = R < 64 ? R : 64;       // inner box of R1 (elements)
@@ -108,7 +111,7 @@ struct Bars {
   uint64_t* d_full;      // [2]
   uint64_t* d_empty;     // [2]
   uint64_t* drain;       // [2]
-  uint64_t* cbar;        // consumer-warp barrier (8 arrivals per phase)
+  uint64_t* cbar;        // consumer-warp barrier (16 arrivals per phase)
   uint32_t* tmem_slot;
   int* abort_flag;
 };
@@ -415,32 +418,38 @@ __device__ void fallback_token(const RouteArgs& a, const uint8_t* zs, int t, int
 template <int R, int KCAP>
 __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
+  constexpr int KL = C::KL, S = C::S;
   const RouteArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sp = warp & 3;              // TMEM subpartition: lanes 32 sp .. 32 sp + 31
-  const int g = (warp - 4) >> 2;        // consumer warpgroup 0 / 1
+  const int g = (warp - 4) >> 2;        // consumer warpgroup 0..3
+  const int ctid = threadIdx.x - 128;   // 0..511
   const int t = sp * 32 + lane;         // token of this thread in pass 1 and finalize
   const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
   uint8_t* zs = smem + p.off_zs;
-  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);
+  uint32_t* stage = lists + 3 * KL * kBT;  // (chunk, rank) of each needed pair, after the lists
   uint2* cand = reinterpret_cast<uint2*>(smem + p.off_cand);
   float* thr = reinterpret_cast<float*>(smem + p.off_thr);
-  int* cnt = reinterpret_cast<int*>(smem + p.off_cnt);
   int* flag = reinterpret_cast<int*>(smem + p.off_flag);
+  uint8_t* nq = smem + p.off_nq;
+  uint8_t* pc = smem + p.off_pc;
+  uint32_t* pairs = reinterpret_cast<uint32_t*>(smem + p.off_pairs);
+  int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
+  int* cbase = reinterpret_cast<int*>(smem + p.off_cbase);
+  int* scan = reinterpret_cast<int*>(smem + p.off_scan);
   const uint32_t low = p.low_mask;
   int ds = 0;
-  uint32_t dph = 0;
-  uint32_t cph = 0;
+  uint32_t dph = 0, cph = 0;
   int lt = 0;
 
   for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
     const int64_t n0 = (int64_t)tile * kBT;
     const int buf = lt & 1;
-    // ---------------- Z epilogue: TMEM -> (z_hi, z_lo) -> shared memory -------------
-    if (!wait_bar(&b.zacc_full[buf], (lt >> 1) & 1, b.abort_flag, a.status)) return;
-    tc_fence_after();
-    {
+    // ---------------- Z epilogue (warpgroups 0, 1): TMEM -> (z_hi, z_lo) -> smem ----------
+    if (g < 2) {
+      if (!wait_bar(&b.zacc_full[buf], (lt >> 1) & 1, b.abort_flag, a.status)) return;
+      tc_fence_after();
       constexpr int HALF = R / 2;
       uint32_t zr[HALF];
       const uint32_t taddr = tmem_base + lane_base + 256 + buf * C::ZCOLS + g * HALF;
@@ -482,116 +491,143 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     }
 
     // ---------------- pass 1: chunk maxima -> top (k+2) chunk keys --------------------
-    uint32_t kl[C::KL];
+    // warpgroup g owns columns 32 g .. 32 g + 31 of every 128-expert tile.
+    uint32_t kl[KL];
 #pragma unroll
-    for (int i = 0; i < C::KL; ++i) kl[i] = 0u;
+    for (int i = 0; i < KL; ++i) kl[i] = 0u;
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
       tc_fence_after();
-      uint32_t v[64];
-      const uint32_t taddr = tmem_base + lane_base + ds * 128 + g * 64;
-      tmem_ld_x32(taddr, v);
-      tmem_ld_x32(taddr + 32, v + 32);
+      uint32_t v[32];
+      tmem_ld_x32(tmem_base + lane_base + ds * 128 + g * 32, v);
       tmem_wait_ld();
-      reg_fence<64>(v);
+      reg_fence<32>(v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&b.d_empty[ds]);
       ds ^= 1;
       if (ds == 0) dph ^= 1u;
+      const int c = pt * 4 + g;
+      if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int c = pt * 4 + g * 2 + hh;
-        uint32_t* vc = v + hh * 32;
-        if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (32 * c + j >= a.M) vc[j] = 0xff800000u;
-        }
-        const uint32_t key = (ord_key(max32(vc)) & ~low) | (uint32_t)c;
-        key_insert<C::KL>(kl, key);
+        for (int j = 0; j < 32; ++j)
+          if (32 * c + j >= a.M) v[j] = 0xff800000u;
       }
+      key_insert<KL>(kl, (ord_key(max32(v)) & ~low) | (uint32_t)c);
     }
 
-    // ---------------- select: merge the two warpgroups' lists, mark needed chunks -----
-    if (g == 1) {
+    // ---------------- select: merge the lists, list the needed (chunk, token) pairs -----
+    if (g > 0) {
 #pragma unroll
-      for (int i = 0; i < C::KL; ++i) lists[i * kBT + t] = kl[i];
+      for (int i = 0; i < KL; ++i) lists[((g - 1) * KL + i) * kBT + t] = kl[i];
     }
     if (!consumer_sync(b, cph, a.status)) return;
     if (g == 0) {
 #pragma unroll
-      for (int i = 0; i < C::KL; ++i) key_insert<C::KL>(kl, lists[i * kBT + t]);
+      for (int w = 0; w < 3; ++w)
+#pragma unroll
+        for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(w * KL + i) * kBT + t]);
       const bool active = n0 + t < a.N;
       uint32_t kth = 0;
 #pragma unroll
-      for (int i = 0; i < C::KL; ++i)
+      for (int i = 0; i < KL; ++i)
         if (i == a.k - 1) kth = kl[i];
       const uint32_t T = kth & ~low;
       int f = active ? 0 : 2;
       float threshold = -INFINITY;
       if (T >= kRealKey) {
         threshold = ord_inv(T);
-        if ((kl[C::KL - 1] & ~low) >= T) f |= 1;  // more ties than the list holds
+        if ((kl[KL - 1] & ~low) >= T) f |= 1;  // more ties than the list holds
       }
+      int needed = 0;
       if (f == 0) {
+        // the needed chunks are a prefix of the sorted list: real keys not below T;
+        // each takes the next place in its chunk's pair bucket
 #pragma unroll
-        for (int i = 0; i < C::KL; ++i) {
+        for (int i = 0; i < KL; ++i) {
           const uint32_t vb = kl[i] & ~low;
-          if (vb >= kRealKey && vb >= T) atomicOr(&bits[(kl[i] & low) * 4 + (t >> 5)], 1u << (t & 31));
+          if (vb >= kRealKey && vb >= T) {
+            const uint32_t cid = kl[i] & low;
+            const int rank = atomicAdd(&ccount[cid], 1);
+            stage[t * KL + i] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
+            needed = i + 1;
+          }
         }
       }
       thr[t] = threshold;
-      cnt[t] = 0;
       flag[t] = f;
+      nq[t] = (uint8_t)needed;
+    }
+    if (!consumer_sync(b, cph, a.status)) return;
+    // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty)
+    {
+      int vals[4], run = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = ctid * 4 + j;
+        vals[j] = (i < p.nchunks) ? ccount[i] : 0;
+        run += vals[j];
+      }
+      int incl = run;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      if (lane == 31) scan[ctid >> 5] = incl;
+      if (!consumer_sync(b, cph, a.status)) return;
+      int before = incl - run;
+      for (int w = 0; w < (ctid >> 5); ++w) before += scan[w];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = ctid * 4 + j;
+        if (i <= p.nchunks) cbase[i] = before;
+        if (i < p.nchunks) ccount[i] = 0;
+        before += vals[j];
+      }
+    }
+    if (!consumer_sync(b, cph, a.status)) return;
+    if (g == 0) {
+      const int needed = nq[t];
+      for (int i = 0; i < needed; ++i) {
+        const uint32_t st = stage[t * KL + i];
+        pairs[cbase[st & 0xffffu] + (st >> 16)] = (uint32_t)t | ((uint32_t)i << 8);
+      }
     }
     if (!consumer_sync(b, cph, a.status)) return;
 
     // ---------------- pass 2: candidates of the needed chunks --------------------------
+    // lane group sp of the transposed tile is chunk 4 pt + sp; its pairs are split
+    // among the four warpgroups.
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
       tc_fence_after();
       const int c = pt * 4 + sp;
       const int e = 32 * c + lane;
       const uint32_t col0 = tmem_base + lane_base + ds * 128;
-#pragma unroll 1
-      for (int w = 2 * g; w < 2 * g + 2; ++w) {
-        uint32_t m = (c < p.nchunks) ? bits[c * 4 + w] : 0u;
-        __syncwarp();
-        if (lane == 0 && m) bits[c * 4 + w] = 0u;
-        while (m) {
-          int tok[4];
-          uint32_t val[4];
-          int nb = 0;
+      const int lo = (c < p.nchunks) ? cbase[c] : 0;
+      const int hi = (c < p.nchunks) ? cbase[c + 1] : 0;
+      for (int pi = lo + g; pi < hi; pi += 4 * kPairBatch) {
+        uint32_t ent[kPairBatch], val[kPairBatch];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            tok[q] = -1;
-            if (m) {
-              const int bit = __ffs(m) - 1;
-              m &= m - 1;
-              tok[q] = 32 * w + bit;
-              nb = q + 1;
-            }
-          }
+        for (int q = 0; q < kPairBatch; ++q) {
+          const int pj = pi + 4 * q;
+          ent[q] = (pj < hi) ? pairs[pj] : 0xffffffffu;
+          if (ent[q] != 0xffffffffu) val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
+        }
+        tmem_wait_ld();
+        reg_fence<kPairBatch>(val);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (q < nb) val[q] = tmem_ld_x1(col0 + tok[q]);
-          tmem_wait_ld();
-          reg_fence<4>(val);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (q >= nb) break;
-            const float x = __uint_as_float(val[q]);
-            const bool take = (e < a.M) && (x >= thr[tok[q]]);
-            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            if (bal) {
-              int base = 0;
-              if (lane == 0) base = atomicAdd(&cnt[tok[q]], __popc(bal));
-              base = __shfl_sync(0xffffffffu, base, 0);
-              const int pos = base + __popc(bal & ((1u << lane) - 1u));
-              if (take && pos < C::C) cand[tok[q] * C::C + pos] = make_uint2(val[q], (uint32_t)e);
-            }
-          }
+        for (int q = 0; q < kPairBatch; ++q) {
+          if (ent[q] == 0xffffffffu) break;
+          const int tok = ent[q] & 0xff, slot = ent[q] >> 8;
+          const float x = __uint_as_float(val[q]);
+          const bool take = (e < a.M) && (x >= thr[tok]);
+          const uint32_t bal = __ballot_sync(0xffffffffu, take);
+          const int pos = __popc(bal & ((1u << lane) - 1u));
+          const int base = (tok * KL + slot) * S;
+          if (take && pos < S) cand[base + pos] = make_uint2(val[q], (uint32_t)e);
+          if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
         }
       }
       tc_fence_before();
@@ -606,17 +642,24 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     if (g == 0) {
       const int64_t n = n0 + t;
       const int f = flag[t];
-      const int nc = cnt[t];
       const bool active = (f & 2) == 0;
-      const bool fb = active && ((f & 1) || nc > C::C || nc < a.k);
+      bool fb = active && (f & 1);
       if (active && !fb) {
         TopList<KCAP> sel;
         sel.init();
-        for (int q = 0; q < nc; ++q) {
-          uint2 cv = cand[t * C::C + q];
-          sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
+        const int jn = nq[t];
+        int total = 0;
+        for (int q = 0; q < jn; ++q) {
+          const int nc = pc[t * KL + q];
+          total += nc;
+          if (nc > S) fb = true;
+          for (int s2 = 0; s2 < nc && s2 < S; ++s2) {
+            const uint2 cv = cand[(t * KL + q) * S + s2];
+            sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
+          }
         }
-        write_token<R, KCAP>(a, n, sel);
+        if (total < a.k) fb = true;
+        if (!fb) write_token<R, KCAP>(a, n, sel);
       }
       uint32_t need = __ballot_sync(0xffffffffu, fb);
       while (need) {
@@ -654,12 +697,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&b.zacc_full[i], 1);
       mbar_init(&b.zacc_empty[i], 8);
       mbar_init(&b.d_full[i], 1);
-      mbar_init(&b.d_empty[i], 8);
+      mbar_init(&b.d_empty[i], kConsumerWarps);
       mbar_init(&b.drain[i], 1);
     }
     mbar_init(b.zsm_full, 8);
     mbar_init(b.zsm_empty, 1);
-    mbar_init(b.cbar, 8);
+    mbar_init(b.cbar, kConsumerWarps);
     *b.abort_flag = 0;
     fence_mbar_init();
   }
@@ -672,9 +715,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(b.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= 4) {  // clear the needed-chunk bitmask
-    uint32_t* bits = reinterpret_cast<uint32_t*>(smem + p.off_bits);
-    for (int i = threadIdx.x - 128; i < p.nchunks * 4; i += kConsumerThreads) bits[i] = 0u;
+  if (warp >= 4) {  // clear the per-chunk pair counters
+    int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
+    for (int i = threadIdx.x - 128; i < p.nchunks; i += kConsumerThreads) ccount[i] = 0;
   }
   tc_fence_before();
   __syncthreads();
@@ -754,18 +797,26 @@ uint32_t plan(Params& p) {
         off += r2n * C::R2_STAGE;
         p.off_zs = off = align_up(off, 1024);
         off += C::ZS_BYTES;
-        p.off_bits = off = align_up(off, 16);
-        off += p.nchunks * 16;
-        // candidate slots and the list exchange share memory (disjoint lifetimes)
-        const uint32_t cand_bytes = kBT * C::C * 8, list_bytes = kBT * C::KL * 4;
+        // candidate slots and the list exchange + pair staging share memory (disjoint lifetimes)
+        const uint32_t cand_bytes = kBT * C::KL * C::S * 8, list_bytes = 4 * kBT * C::KL * 4;
         p.off_cand = p.off_lists = off = align_up(off, 16);
         off += cand_bytes > list_bytes ? cand_bytes : list_bytes;
         p.off_thr = off;
         off += kBT * 4;
-        p.off_cnt = off;
-        off += kBT * 4;
         p.off_flag = off;
         off += kBT * 4;
+        p.off_pairs = off;
+        off += kBT * C::KL * 4;
+        p.off_ccount = off;
+        off += p.nchunks * 4;
+        p.off_cbase = off;
+        off += (p.nchunks + 1) * 4;
+        p.off_scan = off = align_up(off, 16);
+        off += kConsumerWarps * 4;
+        p.off_nq = off;
+        off += kBT;
+        p.off_pc = off;
+        off += kBT * C::KL;
         p.off_bar = off = align_up(off, 8);
         off += kBarBytes;
         const uint32_t total = off + 1024;  // alignment slack of the dynamic base
@@ -844,6 +895,7 @@ bool supports_r(const RouteArgs& a) {
 }  // namespace tc
 
 bool fused_tc_supports(const RouteArgs& a) {
+  // 65536 experts = 2048 chunks: the pair-count scan covers 4 chunks per consumer thread
   if (a.M > 65536 || a.k > 16 || a.N < 1 || a.N > 0x7fffffffLL - tc::kBT) return false;
   if (!tc::encode_fn()) return false;
   switch (a.r) {
