@@ -585,6 +585,8 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         if (i < p.nchunks) ccount[i] = 0;
         before += vals[j];
       }
+      // the end of the last bucket (index nchunks lies past the 4 x 512 slots when nchunks == 2048)
+      if (ctid == kConsumerThreads - 1) cbase[p.nchunks] = before;
     }
     if (!consumer_sync(b, cph, a.status)) return;
     if (g == 0) {
@@ -840,8 +842,8 @@ bool fill_params(const RouteArgs& a, Params& p, uint32_t& smem) {
   p.kb_count = (a.h + kBK - 1) / kBK;
   p.p_count = (a.M + kBE - 1) / kBE;
   p.nchunks = (a.M + 31) / 32;
-  int bits = 1;
-  while ((1 << bits) < p.nchunks) ++bits;
+  int bits = 1;  // chunk ids run up to 4 p_count - 1 (the padded last tile)
+  while ((1 << bits) < 4 * p.p_count) ++bits;
   p.low_mask = (1u << bits) - 1u;
   smem = plan<R, KCAP>(p);
   return smem != 0;
