@@ -56,6 +56,7 @@ constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
 constexpr int kConsumerThreads = 512;
 constexpr int kConsumerWarps = 16;
 constexpr int kPairBatch = 8;   // TMEM column loads in flight per warp in pass 2
+constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than S candidates
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint32_t kRealKey = 0x00800000u;  // ordered value of -FLT_MAX: keys below are not real chunks
@@ -73,7 +74,7 @@ struct Params {
   int r2_stages;
   int r2_resident;   // every expert tile stays in shared memory
   uint32_t off_x, off_r1, off_r2, off_zs, off_lists, off_cand, off_thr, off_flag, off_nq, off_pc, off_pairs,
-      off_ccount, off_cbase, off_scan, off_bar;
+      off_ccount, off_cbase, off_scan, off_pool, off_poolcnt, off_bar;
 };
 
 template <int R, int KCAP>
@@ -93,6 +94,8 @@ struct Cfg {
   static constexpr uint32_t ZS_BYTES = kBT * RK * 2;   // z pair of 128 tokens, K-major core matrices
   static constexpr uint32_t ZS_SBO = (RK / 8) * 128;   // byte stride of 8-token groups
   static constexpr int ZCOLS = R < 32 ? 32 : R;        // TMEM columns per Z accumulator
+  static constexpr int ND = (512 - 2 * ZCOLS) / 128 < 3 ? (512 - 2 * ZCOLS) / 128 : 3;  // logit tile buffers
+  static constexpr int ZCOL0 = ND * 128;               // first TMEM column of the Z accumulators
   static constexpr uint32_t IDESC_Z = idesc_bf16_f32(128, R, 0, 1);    // A = X (K-major), B = R1 (MN-major)
   static constexpr uint32_t IDESC_P1 = idesc_bf16_f32(128, 128, 0, 1); // A = z pair, B = R2 tile
   static constexpr uint32_t IDESC_P2 = idesc_bf16_f32(128, 128, 1, 0); // A = R2 tile^T, B = z pair^T
@@ -108,8 +111,8 @@ struct Bars {
   uint64_t* zacc_empty;  // [2]
   uint64_t* zsm_full;
   uint64_t* zsm_empty;
-  uint64_t* d_full;      // [2]
-  uint64_t* d_empty;     // [2]
+  uint64_t* d_full;      // [3]
+  uint64_t* d_empty;     // [3]
   uint64_t* drain;       // [2]
   uint64_t* cbar;        // consumer-warp barrier (16 arrivals per phase)
   uint32_t* tmem_slot;
@@ -128,19 +131,19 @@ __device__ __forceinline__ Bars bars_at(uint8_t* smem, const Params& p) {
   r.zsm_full = r.zacc_empty + 2;
   r.zsm_empty = r.zsm_full + 1;
   r.d_full = r.zsm_empty + 1;
-  r.d_empty = r.d_full + 2;
-  r.drain = r.d_empty + 2;
+  r.d_empty = r.d_full + 3;
+  r.drain = r.d_empty + 3;
   r.cbar = r.drain + 2;
   r.tmem_slot = reinterpret_cast<uint32_t*>(r.cbar + 1);
   r.abort_flag = reinterpret_cast<int*>(r.tmem_slot + 1);
   return r;
 }
-constexpr uint32_t kBarBytes = (16 + 128 + 13) * 8 + 16;
+constexpr uint32_t kBarBytes = (16 + 128 + 15) * 8 + 16;
 
-// Bounded mbarrier wait: false once the limit passes or another thread gave up.
-__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                      unsigned int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of the bounded mbarrier wait: false once the limit passes or another
+// thread gave up.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                           unsigned int* status) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -155,14 +158,20 @@ __device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile i
   }
 }
 
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bar_slow(bar, parity, abort_flag, status);
+}
 
-// Barrier of the 8 consumer warps, on an mbarrier so that the wait is bounded too.
-__device__ __forceinline__ bool consumer_sync(const Bars& b, uint32_t& phase, unsigned int* status) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(b.cbar);
-  const bool ok = wait_bar(b.cbar, phase, b.abort_flag, status);
-  phase ^= 1u;
-  return ok;
+
+// Barrier of the 16 consumer warps (named barrier 1).  It cannot strand a warp:
+// between two of these barriers every consumer warp performs the same bounded
+// mbarrier waits, so when one gives up (and raises the abort flag) all of them
+// leave at a wait before reaching the next barrier.
+__device__ __forceinline__ bool consumer_sync(const Bars&, uint32_t&, unsigned int*) {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+  return true;
 }
 
 // Order-preserving map of fp32 onto uint32 and its inverse.
@@ -286,7 +295,7 @@ __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tm
     const int buf = lt & 1;
     if (!wait_bar(&b.zacc_empty[buf], ((lt >> 1) & 1) ^ 1u, b.abort_flag, p.a.status)) break;
     tc_fence_after();
-    const uint32_t d = tmem_base + 256 + buf * C::ZCOLS;
+    const uint32_t d = tmem_base + C::ZCOL0 + buf * C::ZCOLS;
     for (int kb = 0; kb < p.kb_count; ++kb) {
       if (!wait_bar(&b.x_full[s], ph, b.abort_flag, p.a.status)) goto done;
       tc_fence_after();
@@ -354,8 +363,10 @@ __device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32
             rph ^= 1u;
           }
         }
-        ds ^= 1;
-        if (ds == 0) dph ^= 1u;
+        if (++ds == C::ND) {
+          ds = 0;
+          dph ^= 1u;
+        }
       }
     }
     mma_commit(b.zsm_empty);
@@ -438,6 +449,8 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
   int* cbase = reinterpret_cast<int*>(smem + p.off_cbase);
   int* scan = reinterpret_cast<int*>(smem + p.off_scan);
+  uint2* pool = reinterpret_cast<uint2*>(smem + p.off_pool);
+  int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
   const uint32_t low = p.low_mask;
   int ds = 0;
   uint32_t dph = 0, cph = 0;
@@ -452,7 +465,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       tc_fence_after();
       constexpr int HALF = R / 2;
       uint32_t zr[HALF];
-      const uint32_t taddr = tmem_base + lane_base + 256 + buf * C::ZCOLS + g * HALF;
+      const uint32_t taddr = tmem_base + lane_base + C::ZCOL0 + buf * C::ZCOLS + g * HALF;
       if constexpr (HALF == 8) {
         tmem_ld_x8(taddr, zr);
       } else if constexpr (HALF == 16) {
@@ -505,8 +518,10 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&b.d_empty[ds]);
-      ds ^= 1;
-      if (ds == 0) dph ^= 1u;
+      if (++ds == C::ND) {
+        ds = 0;
+        dph ^= 1u;
+      }
       const int c = pt * 4 + g;
       if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
 #pragma unroll
@@ -557,6 +572,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       thr[t] = threshold;
       flag[t] = f;
       nq[t] = (uint8_t)needed;
+      poolcnt[t] = 0;
     }
     if (!consumer_sync(b, cph, a.status)) return;
     // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty)
@@ -630,13 +646,19 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           const int base = (tok * KL + slot) * S;
           if (take && pos < S) cand[base + pos] = make_uint2(val[q], (uint32_t)e);
           if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
+          if (__popc(bal) > S && take && pos >= S) {  // rare: more candidates than the pair's slots
+            const int ps = atomicAdd(&poolcnt[tok], 1);
+            if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = make_uint2(val[q], (uint32_t)e);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&b.d_empty[ds]);
-      ds ^= 1;
-      if (ds == 0) dph ^= 1u;
+      if (++ds == C::ND) {
+        ds = 0;
+        dph ^= 1u;
+      }
     }
     if (!consumer_sync(b, cph, a.status)) return;
 
@@ -654,11 +676,16 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         for (int q = 0; q < jn; ++q) {
           const int nc = pc[t * KL + q];
           total += nc;
-          if (nc > S) fb = true;
           for (int s2 = 0; s2 < nc && s2 < S; ++s2) {
             const uint2 cv = cand[(t * KL + q) * S + s2];
             sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
           }
+        }
+        const int np = poolcnt[t];
+        if (np > kPoolSlots) fb = true;
+        for (int q = 0; q < np && q < kPoolSlots; ++q) {
+          const uint2 cv = pool[t * kPoolSlots + q];
+          sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
         }
         if (total < a.k) fb = true;
         if (!fb) write_token<R, KCAP>(a, n, sel);
@@ -698,9 +725,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b.zacc_full[i], 1);
       mbar_init(&b.zacc_empty[i], 8);
+      mbar_init(&b.drain[i], 1);
+    }
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&b.d_full[i], 1);
       mbar_init(&b.d_empty[i], kConsumerWarps);
-      mbar_init(&b.drain[i], 1);
     }
     mbar_init(b.zsm_full, 8);
     mbar_init(b.zsm_empty, 1);
@@ -787,7 +816,7 @@ uint32_t plan(Params& p) {
   using C = Cfg<R, KCAP>;
   for (int xs = 4; xs >= 2; --xs) {
     for (int mode = 0; mode < 2; ++mode) {  // 0: R2 resident, 1: streamed
-      const int r2s = mode == 0 ? p.p_count : 4;
+      const int r2s = mode == 0 ? p.p_count : 8;
       if (mode == 0 && p.p_count > 64) continue;
       for (int r2n = r2s; r2n >= 2 || (mode == 0 && r2n == r2s); --r2n) {
         uint32_t off = 0;
@@ -817,6 +846,10 @@ uint32_t plan(Params& p) {
         off += kConsumerWarps * 4;
         p.off_nq = off;
         off += kBT;
+        p.off_poolcnt = off = align_up(off, 4);
+        off += kBT * 4;
+        p.off_pool = off = align_up(off, 8);
+        off += kBT * kPoolSlots * 8;
         p.off_pc = off;
         off += kBT * C::KL;
         p.off_bar = off = align_up(off, 8);
