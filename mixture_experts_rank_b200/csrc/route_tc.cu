@@ -51,7 +51,6 @@ using namespace sm100;
 
 constexpr int kBT = 128;        // tokens per tile (MMA M of Z and pass 1, N of pass 2)
 constexpr int kBE = 128;        // experts per logit tile
-constexpr int kBK = 64;         // hidden elements per X stage (128-byte rows)
 constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
 constexpr int kConsumerThreads = 512;
 constexpr int kConsumerWarps = 16;
@@ -74,18 +73,21 @@ struct Params {
   int r2_stages;
   int r2_resident;   // every expert tile stays in shared memory
   uint32_t off_x, off_r1, off_r2, off_zs, off_lists, off_cand, off_thr, off_flag, off_nq, off_pc, off_pairs,
-      off_ccount, off_cbase, off_scan, off_pool, off_poolcnt, off_bar;
+      off_ccount, off_cbase, off_scan, off_pool, off_poolcnt, off_znorm, off_cnorm, off_bar;
 };
 
 template <int R, int KCAP>
 struct Cfg {
-  static constexpr int KL = KCAP + 2;                  // chunk keys kept per token
-  static constexpr int S = 2;                          // candidate slots per (token, needed chunk)
-  static constexpr int RK = 2 * R;                     // K of the logit MMAs: z_hi | z_lo
-  static constexpr uint32_t X_STAGE = kBT * kBK * 2;   // 16 KB
+  static constexpr int KL = KCAP + 6;                  // chunk keys kept per token
+  static constexpr int S = 1;                          // candidate slots per (token, needed chunk)
+  static constexpr int RK = 2 * R;                     // z_hi | z_lo columns of the z buffer
+  static constexpr int BK = R >= 128 ? 32 : 64;        // hidden elements per X stage
+  static constexpr uint32_t X_STAGE = kBT * BK * 2;    // 16 KB (8 KB at BK = 32)
+  static constexpr uint32_t X_LAYOUT = BK == 64 ? kSwizzle128B : kSwizzle64B;
+  static constexpr uint32_t X_SBO = 8 * BK * 2;        // bytes per 8-row swizzle atom
   static constexpr int R1_BOX = R < 64 ? R : 64;       // inner box of R1 (elements)
   static constexpr int R1_BOXES = R / R1_BOX;
-  static constexpr uint32_t R1_BOX_BYTES = kBK * R1_BOX * 2;
+  static constexpr uint32_t R1_BOX_BYTES = BK * R1_BOX * 2;
   static constexpr uint32_t R1_STAGE = R1_BOX_BYTES * R1_BOXES;
   static constexpr uint32_t R1_ROW = R1_BOX * 2;       // bytes per R1 row inside a box
   static constexpr uint32_t R1_LAYOUT = R1_ROW == 32 ? kSwizzle32B : (R1_ROW == 64 ? kSwizzle64B : kSwizzle128B);
@@ -169,7 +171,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 // between two of these barriers every consumer warp performs the same bounded
 // mbarrier waits, so when one gives up (and raises the abort flag) all of them
 // leave at a wait before reaching the next barrier.
-__device__ __forceinline__ bool consumer_sync(const Bars&, uint32_t&, unsigned int*) {
+__device__ __forceinline__ bool consumer_sync(const Bars&, int, unsigned int*) {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
   return true;
 }
@@ -236,11 +238,11 @@ __device__ void producer_x(const Params& p, const Bars& b, uint8_t* smem, const 
     for (int kb = 0; kb < p.kb_count; ++kb) {
       if (!wait_bar(&b.x_empty[s], ph ^ 1u, b.abort_flag, p.a.status)) return;
       mbar_arrive_expect_tx(&b.x_full[s], C::X_STAGE + C::R1_STAGE);
-      tma_load_2d(smem + p.off_x + s * C::X_STAGE, tmX, &b.x_full[s], kb * kBK, tile * kBT);
+      tma_load_2d(smem + p.off_x + s * C::X_STAGE, tmX, &b.x_full[s], kb * C::BK, tile * kBT);
 #pragma unroll
       for (int q = 0; q < C::R1_BOXES; ++q)
         tma_load_2d(smem + p.off_r1 + s * C::R1_STAGE + q * C::R1_BOX_BYTES, tmR1, &b.x_full[s], q * 64,
-                    kb * kBK);
+                    kb * C::BK);
       if (++s == p.x_stages) {
         s = 0;
         ph ^= 1u;
@@ -300,8 +302,8 @@ __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tm
       if (!wait_bar(&b.x_full[s], ph, b.abort_flag, p.a.status)) goto done;
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk) {
-        uint64_t ad = smem_desc(x0 + s * C::X_STAGE + kk * 32, 16, 1024, kSwizzle128B);
+      for (int kk = 0; kk < C::BK / 16; ++kk) {
+        uint64_t ad = smem_desc(x0 + s * C::X_STAGE + kk * 32, 16, C::X_SBO, C::X_LAYOUT);
         uint64_t bd = smem_desc(r10 + s * C::R1_STAGE + kk * 16 * C::R1_ROW, C::R1_BOX_BYTES, 8 * C::R1_ROW,
                                 C::R1_LAYOUT);
         mma_bf16(d, ad, bd, C::IDESC_Z, (kb | kk) != 0);
@@ -347,9 +349,9 @@ __device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32
         const uint32_t d = tmem_base + ds * 128;
         const uint32_t r2 = r20 + st * C::R2_STAGE;
 #pragma unroll
-        for (int kk = 0; kk < C::RK / 16; ++kk) {
+        for (int kk = 0; kk < R / 16; ++kk) {  // z_hi only; z_lo enters through the CUDA-core correction
           uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
-          uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
+          uint64_t rd = smem_desc(r2 + kk * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
           if (pass == 0)
             mma_bf16(d, zd, rd, C::IDESC_P1, kk != 0);
           else
@@ -426,6 +428,14 @@ __device__ void fallback_token(const RouteArgs& a, const uint8_t* zs, int t, int
   warp_write_selection(a, n, lane, v, e);
 }
 
+// Byte offset of R2 element (row i, expert e_local of a 128-expert stage) in the
+// MN-major 128B-swizzled stage written by TMA (two boxes of 64 experts x R rows).
+template <int R>
+__device__ __forceinline__ uint32_t r2_offset(int i, int e_local) {
+  const int box = e_local >> 6, col = e_local & 63;
+  return (uint32_t)(box * (64 * R * 2) + i * 128 + ((((col >> 3) ^ (i & 7))) << 4) + (col & 7) * 2);
+}
+
 template <int R, int KCAP>
 __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
@@ -434,12 +444,14 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sp = warp & 3;              // TMEM subpartition: lanes 32 sp .. 32 sp + 31
   const int g = (warp - 4) >> 2;        // consumer warpgroup 0..3
+  const int cw = warp - 4;              // consumer warp 0..15
   const int ctid = threadIdx.x - 128;   // 0..511
   const int t = sp * 32 + lane;         // token of this thread in pass 1 and finalize
   const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
   uint8_t* zs = smem + p.off_zs;
+  const uint8_t* r2s = smem + p.off_r2;
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);
-  uint32_t* stage = lists + 3 * KL * kBT;  // (chunk, rank) of each needed pair, after the lists
+  uint32_t* stage = lists + 2 * KL * kBT;  // (chunk, rank) of each needed pair, after the two list slots
   uint2* cand = reinterpret_cast<uint2*>(smem + p.off_cand);
   float* thr = reinterpret_cast<float*>(smem + p.off_thr);
   int* flag = reinterpret_cast<int*>(smem + p.off_flag);
@@ -451,10 +463,33 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   int* scan = reinterpret_cast<int*>(smem + p.off_scan);
   uint2* pool = reinterpret_cast<uint2*>(smem + p.off_pool);
   int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
+  float* znorm = reinterpret_cast<float*>(smem + p.off_znorm);  // [hi g0 | hi g1 | lo g0 | lo g1][token]
+  float* cnorm = reinterpret_cast<float*>(smem + p.off_cnorm);
   const uint32_t low = p.low_mask;
-  int ds = 0;
-  uint32_t dph = 0, cph = 0;
+  int ds = 0, rs = 0;
+  uint32_t dph = 0, rph = 0;
   int lt = 0;
+  float colmax2 = 0.f;  // this warp's largest squared R2 column norm (first tile)
+
+  // R2 stage of the current logit tile: wait until it is in shared memory.
+  auto r2_stage = [&](int pt, int& st) -> bool {
+    if (p.r2_resident) {
+      st = pt;
+      return wait_bar(&b.r2_full[pt], 0, b.abort_flag, a.status);
+    }
+    st = rs;
+    return wait_bar(&b.r2_full[rs], rph, b.abort_flag, a.status);
+  };
+  // This warp is done with the R2 stage of the current logit tile.
+  auto r2_release = [&]() {
+    if (p.r2_resident) return;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b.r2_empty[rs]);
+    if (++rs == p.r2_stages) {
+      rs = 0;
+      rph ^= 1u;
+    }
+  };
 
   for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
     const int64_t n0 = (int64_t)tile * kBT;
@@ -481,6 +516,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       if (lane == 0) mbar_arrive(&b.zacc_empty[buf]);
       // the previous tile's logit MMAs must be done with the z buffer
       if (lt > 0 && !wait_bar(b.zsm_empty, (lt - 1) & 1, b.abort_flag, a.status)) return;
+      float hi2 = 0.f, lo2 = 0.f;
 #pragma unroll
       for (int q = 0; q < HALF / 8; ++q) {
         uint32_t hi[4], lo[4];
@@ -490,6 +526,10 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           __nv_bfloat16 h0 = __float2bfloat16_rn(z0), h1 = __float2bfloat16_rn(z1);
           __nv_bfloat16 l0 = __float2bfloat16_rn(z0 - __bfloat162float(h0));
           __nv_bfloat16 l1 = __float2bfloat16_rn(z1 - __bfloat162float(h1));
+          const float fh0 = __bfloat162float(h0), fh1 = __bfloat162float(h1);
+          const float fl0 = __bfloat162float(l0), fl1 = __bfloat162float(l1);
+          hi2 = fmaf(fh0, fh0, fmaf(fh1, fh1, hi2));
+          lo2 = fmaf(fl0, fl0, fmaf(fl1, fl1, lo2));
           hi[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
           lo[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
         }
@@ -498,12 +538,14 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, (R + i0) >> 3)) =
             make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
+      znorm[g * kBT + t] = hi2;
+      znorm[(2 + g) * kBT + t] = lo2;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(b.zsm_full);
     }
 
-    // ---------------- pass 1: chunk maxima -> top (k+2) chunk keys --------------------
+    // ---------------- pass 1: chunk maxima of z_hi . R2 -> top KL chunk keys -------------
     // warpgroup g owns columns 32 g .. 32 g + 31 of every 128-expert tile.
     uint32_t kl[KL];
 #pragma unroll
@@ -522,6 +564,25 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         ds = 0;
         dph ^= 1u;
       }
+      if (lt == 0) {
+        // first tile of this CTA: squared column norms of R2 (experts 8 cw .. 8 cw + 7 of the stage)
+        int st;
+        if (!r2_stage(pt, st)) return;
+        const uint8_t* base = r2s + st * C::R2_STAGE;
+        const int el = 8 * cw + (lane & 7);
+        float acc = 0.f;
+#pragma unroll 4
+        for (int i = lane >> 3; i < R; i += 4) {
+          const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + r2_offset<R>(i, el)));
+          acc = fmaf(w, w, acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+        colmax2 = fmaxf(colmax2, acc);
+        r2_release();
+      } else {
+        r2_release();
+      }
       const int c = pt * 4 + g;
       if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
 #pragma unroll
@@ -531,37 +592,61 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       key_insert<KL>(kl, (ord_key(max32(v)) & ~low) | (uint32_t)c);
     }
 
-    // ---------------- select: merge the lists, list the needed (chunk, token) pairs -----
-    if (g > 0) {
+    // ---------------- select: merge the lists, certified window, needed pairs --------------
+    // two-round merge of the four partial lists: g2 -> g0 and g3 -> g1, then g1 -> g0
+    if (g >= 2) {
 #pragma unroll
-      for (int i = 0; i < KL; ++i) lists[((g - 1) * KL + i) * kBT + t] = kl[i];
+      for (int i = 0; i < KL; ++i) lists[((g - 2) * KL + i) * kBT + t] = kl[i];
     }
-    if (!consumer_sync(b, cph, a.status)) return;
+    if (lt == 0) {
+      colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 1));
+      colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 2));
+      colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 4));
+      if (lane == 0) cnorm[cw] = colmax2;
+    }
+    if (!consumer_sync(b, 0, a.status)) return;
+    if (lt == 0 && ctid == 0) {
+      float m = 0.f;
+      for (int w = 0; w < kConsumerWarps; ++w) m = fmaxf(m, cnorm[w]);
+      cnorm[kConsumerWarps] = sqrtf(m) * (1.f + 0x1p-20f);  // max column norm of R2, rounded up
+    }
+    if (g < 2) {
+#pragma unroll
+      for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(g * KL + i) * kBT + t]);
+      if (g == 1) {  // each thread rewrites only its own column of slot 1
+#pragma unroll
+        for (int i = 0; i < KL; ++i) lists[(KL + i) * kBT + t] = kl[i];
+      }
+    }
+    if (!consumer_sync(b, 0, a.status)) return;
     if (g == 0) {
 #pragma unroll
-      for (int w = 0; w < 3; ++w)
-#pragma unroll
-        for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(w * KL + i) * kBT + t]);
+      for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(KL + i) * kBT + t]);
       const bool active = n0 + t < a.N;
+      // Certified window: values from z_hi differ from the z_hi + z_lo values by at most
+      // eps = |z_lo| cmax (Cauchy-Schwarz) plus a bound on fp32 accumulation differences.
+      const float cmax = cnorm[kConsumerWarps];
+      const float zh = sqrtf(znorm[t] + znorm[kBT + t]);
+      const float zl = sqrtf(znorm[2 * kBT + t] + znorm[3 * kBT + t]);
+      const float eps = (zl * cmax) * (1.f + 0x1p-8f) + (float)R * 0x1p-20f * zh * cmax + 1e-30f;
       uint32_t kth = 0;
 #pragma unroll
       for (int i = 0; i < KL; ++i)
         if (i == a.k - 1) kth = kl[i];
-      const uint32_t T = kth & ~low;
       int f = active ? 0 : 2;
-      float threshold = -INFINITY;
-      if (T >= kRealKey) {
-        threshold = ord_inv(T);
-        if ((kl[KL - 1] & ~low) >= T) f |= 1;  // more ties than the list holds
+      float wcut = -INFINITY;                  // candidates: approximate logit >= wcut
+      uint32_t cut_key = 0u;                   // chunks whose key range reaches cut_key are needed
+      if ((kth & ~low) >= kRealKey) {
+        const float tlow = ord_inv(kth & ~low);  // <= the k-th largest approximate chunk maximum
+        wcut = __fsub_rd(tlow, __fmul_ru(2.f, eps));
+        cut_key = ord_key(wcut);
+        if ((kl[KL - 1] & ~low) >= kRealKey && (kl[KL - 1] | low) >= cut_key) f |= 1;  // list too short
       }
       int needed = 0;
       if (f == 0) {
-        // the needed chunks are a prefix of the sorted list: real keys not below T;
-        // each takes the next place in its chunk's pair bucket
 #pragma unroll
         for (int i = 0; i < KL; ++i) {
-          const uint32_t vb = kl[i] & ~low;
-          if (vb >= kRealKey && vb >= T) {
+          if ((kl[i] & ~low) >= kRealKey && (kl[i] | low) >= cut_key) {
             const uint32_t cid = kl[i] & low;
             const int rank = atomicAdd(&ccount[cid], 1);
             stage[t * KL + i] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
@@ -569,12 +654,12 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           }
         }
       }
-      thr[t] = threshold;
+      thr[t] = wcut;
       flag[t] = f;
       nq[t] = (uint8_t)needed;
       poolcnt[t] = 0;
     }
-    if (!consumer_sync(b, cph, a.status)) return;
+    if (!consumer_sync(b, 0, a.status)) return;
     // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty)
     {
       int vals[4], run = 0;
@@ -591,7 +676,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         if (lane >= d) incl += o;
       }
       if (lane == 31) scan[ctid >> 5] = incl;
-      if (!consumer_sync(b, cph, a.status)) return;
+      if (!consumer_sync(b, 0, a.status)) return;
       int before = incl - run;
       for (int w = 0; w < (ctid >> 5); ++w) before += scan[w];
 #pragma unroll
@@ -604,7 +689,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       // the end of the last bucket (index nchunks lies past the 4 x 512 slots when nchunks == 2048)
       if (ctid == kConsumerThreads - 1) cbase[p.nchunks] = before;
     }
-    if (!consumer_sync(b, cph, a.status)) return;
+    if (!consumer_sync(b, 0, a.status)) return;
     if (g == 0) {
       const int needed = nq[t];
       for (int i = 0; i < needed; ++i) {
@@ -612,14 +697,18 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         pairs[cbase[st & 0xffffu] + (st >> 16)] = (uint32_t)t | ((uint32_t)i << 8);
       }
     }
-    if (!consumer_sync(b, cph, a.status)) return;
+    if (!consumer_sync(b, 0, a.status)) return;
 
-    // ---------------- pass 2: candidates of the needed chunks --------------------------
-    // lane group sp of the transposed tile is chunk 4 pt + sp; its pairs are split
-    // among the four warpgroups.
+    // ---------------- pass 2: candidates of the needed chunks, corrected by z_lo -----------
+    // lane group sp of the transposed tile is chunk 4 pt + sp; its pairs are split among the
+    // four warpgroups.  A candidate's logit is its z_hi value plus z_lo . R2[:, e], computed
+    // here while the R2 tile is still in shared memory.
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
       tc_fence_after();
+      int st;
+      if (!r2_stage(pt, st)) return;
+      const uint8_t* r2t = r2s + st * C::R2_STAGE;
       const int c = pt * 4 + sp;
       const int e = 32 * c + lane;
       const uint32_t col0 = tmem_base + lane_base + ds * 128;
@@ -641,14 +730,35 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           const int tok = ent[q] & 0xff, slot = ent[q] >> 8;
           const float x = __uint_as_float(val[q]);
           const bool take = (e < a.M) && (x >= thr[tok]);
-          const uint32_t bal = __ballot_sync(0xffffffffu, take);
-          const int pos = __popc(bal & ((1u << lane) - 1u));
-          const int base = (tok * KL + slot) * S;
-          if (take && pos < S) cand[base + pos] = make_uint2(val[q], (uint32_t)e);
+          uint32_t bal = __ballot_sync(0xffffffffu, take);
           if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
-          if (__popc(bal) > S && take && pos >= S) {  // rare: more candidates than the pair's slots
-            const int ps = atomicAdd(&poolcnt[tok], 1);
-            if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = make_uint2(val[q], (uint32_t)e);
+          int pos = 0;
+          while (bal) {
+            const int bl = __ffs(bal) - 1;
+            bal &= bal - 1;
+            // z_lo . R2[:, 32 c + bl], rows split across the lanes
+            const int el = sp * 32 + bl;
+            float part = 0.f;
+#pragma unroll
+            for (int i = lane; i < R; i += 32) {
+              const float zl = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                  zs + zs_offset<R, KCAP>(tok, (R + i) >> 3) + (i & 7) * 2));
+              const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(r2t + r2_offset<R>(i, el)));
+              part = fmaf(zl, w, part);
+            }
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
+            const float xv = __shfl_sync(0xffffffffu, x, bl) + part;
+            if (lane == 0) {
+              const uint2 cv = make_uint2(__float_as_uint(xv), (uint32_t)(32 * c + bl));
+              if (pos < S) {
+                cand[(tok * KL + slot) * S + pos] = cv;
+              } else {  // rare: more candidates than the pair's slots
+                const int ps = atomicAdd(&poolcnt[tok], 1);
+                if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
+              }
+            }
+            ++pos;
           }
         }
       }
@@ -659,8 +769,9 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         ds = 0;
         dph ^= 1u;
       }
+      r2_release();
     }
-    if (!consumer_sync(b, cph, a.status)) return;
+    if (!consumer_sync(b, 0, a.status)) return;
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
     if (g == 0) {
@@ -697,7 +808,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         fallback_token<R, KCAP>(a, zs, sp * 32 + j, n0 + sp * 32 + j, lane);
       }
     }
-    if (!consumer_sync(b, cph, a.status)) return;
+    if (!consumer_sync(b, 0, a.status)) return;
   }
 }
 
@@ -720,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nr2 = p.r2_resident ? p.p_count : p.r2_stages;
     for (int i = 0; i < nr2; ++i) {
       mbar_init(&b.r2_full[i], 1);
-      mbar_init(&b.r2_empty[i], 1);
+      mbar_init(&b.r2_empty[i], 1 + kConsumerWarps);  // the MMA commit and every consumer warp
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b.zacc_full[i], 1);
@@ -829,7 +940,7 @@ uint32_t plan(Params& p) {
         p.off_zs = off = align_up(off, 1024);
         off += C::ZS_BYTES;
         // candidate slots and the list exchange + pair staging share memory (disjoint lifetimes)
-        const uint32_t cand_bytes = kBT * C::KL * C::S * 8, list_bytes = 4 * kBT * C::KL * 4;
+        const uint32_t cand_bytes = kBT * C::KL * C::S * 8, list_bytes = 3 * kBT * C::KL * 4;
         p.off_cand = p.off_lists = off = align_up(off, 16);
         off += cand_bytes > list_bytes ? cand_bytes : list_bytes;
         p.off_thr = off;
@@ -844,6 +955,10 @@ uint32_t plan(Params& p) {
         off += (p.nchunks + 1) * 4;
         p.off_scan = off = align_up(off, 16);
         off += kConsumerWarps * 4;
+        p.off_znorm = off;           // per token: |z_hi|^2 and |z_lo|^2 partial sums of both halves
+        off += 4 * kBT * 4;
+        p.off_cnorm = off;           // per consumer warp: max squared column norm of R2; [16] = result
+        off += (kConsumerWarps + 1) * 4;
         p.off_nq = off;
         off += kBT;
         p.off_poolcnt = off = align_up(off, 4);
@@ -872,7 +987,7 @@ template <int R, int KCAP>
 bool fill_params(const RouteArgs& a, Params& p, uint32_t& smem) {
   p.a = a;
   p.num_tiles = (int)((a.N + kBT - 1) / kBT);
-  p.kb_count = (a.h + kBK - 1) / kBK;
+  p.kb_count = (a.h + Cfg<R, KCAP>::BK - 1) / Cfg<R, KCAP>::BK;
   p.p_count = (a.M + kBE - 1) / kBE;
   p.nchunks = (a.M + 31) / 32;
   int bits = 1;  // chunk ids run up to 4 p_count - 1 (the padded last tile)
@@ -892,8 +1007,9 @@ cudaError_t launch(const RouteArgs& a) {
   const CUtensorMapSwizzle r1sw = C::R1_ROW == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
                                   : C::R1_ROW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                     : CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_map(&tmX, a.X, (uint64_t)a.h, (uint64_t)a.N, kBK, kBT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tmR1, a.R1, (uint64_t)R, (uint64_t)a.h, C::R1_BOX, kBK, r1sw) ||
+  const CUtensorMapSwizzle xsw = C::BK == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map(&tmX, a.X, (uint64_t)a.h, (uint64_t)a.N, C::BK, kBT, xsw) ||
+      !make_map(&tmR1, a.R1, (uint64_t)R, (uint64_t)a.h, C::R1_BOX, C::BK, r1sw) ||
       !make_map(&tmR2, a.R2, (uint64_t)a.M, (uint64_t)R, 64, R, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   static int configured = 0;
