@@ -54,7 +54,7 @@ constexpr int kBE = 128;        // experts per logit tile
 constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
 constexpr int kConsumerThreads = 512;
 constexpr int kConsumerWarps = 16;
-constexpr int kPairBatch = 8;   // TMEM column loads in flight per warp in pass 2
+constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass 2
 constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than S candidates
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -436,6 +436,50 @@ __device__ __forceinline__ uint32_t r2_offset(int i, int e_local) {
   return (uint32_t)(box * (64 * R * 2) + i * 128 + ((((col >> 3) ^ (i & 7))) << 4) + (col & 7) * 2);
 }
 
+// z_lo . R2[:, e] for up to kPairBatch candidates at once (rows split across lanes,
+// independent chains and reductions), then the corrected logits into the candidate slots.
+template <int R, int KCAP>
+__device__ __forceinline__ void correct_and_store(int ncand, const uint32_t* cinfo, const float* cx,
+                                                  const uint8_t* zs, const uint8_t* r2t, int sp, int c,
+                                                  int lane, uint2* cand, uint2* pool, int* poolcnt) {
+  constexpr int KL = Cfg<R, KCAP>::KL, S = Cfg<R, KCAP>::S;
+  float part[kPairBatch];
+#pragma unroll
+  for (int j = 0; j < kPairBatch; ++j) {
+    part[j] = 0.f;
+    if (j < ncand) {
+      const int tok = cinfo[j] & 0xff, el = sp * 32 + ((cinfo[j] >> 16) & 0xff);
+#pragma unroll
+      for (int i = lane; i < R; i += 32) {
+        const float zl = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+            zs + zs_offset<R, KCAP>(tok, (R + i) >> 3) + (i & 7) * 2));
+        const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(r2t + r2_offset<R>(i, el)));
+        part[j] = fmaf(zl, w, part[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1)
+#pragma unroll
+    for (int j = 0; j < kPairBatch; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], d);
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < kPairBatch; ++j) {
+      if (j < ncand) {
+        const int tok = cinfo[j] & 0xff, slot = (cinfo[j] >> 8) & 0xff, bl = (cinfo[j] >> 16) & 0xff;
+        const int rk = cinfo[j] >> 24;
+        const uint2 cv = make_uint2(__float_as_uint(cx[j] + part[j]), (uint32_t)(32 * c + bl));
+        if (rk < S) {
+          cand[(tok * KL + slot) * S + rk] = cv;
+        } else {  // rare: more candidates than the pair's slots
+          const int ps = atomicAdd(&poolcnt[tok], 1);
+          if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
+        }
+      }
+    }
+  }
+}
+
 template <int R, int KCAP>
 __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
@@ -724,6 +768,10 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         }
         tmem_wait_ld();
         reg_fence<kPairBatch>(val);
+        // collect the batch's candidates (warp-uniform), then correct them together
+        int ncand = 0;
+        uint32_t cinfo[kPairBatch];  // token | slot << 8 | lane << 16 | (rank within the pair) << 24
+        float cx[kPairBatch];
 #pragma unroll
         for (int q = 0; q < kPairBatch; ++q) {
           if (ent[q] == 0xffffffffu) break;
@@ -732,35 +780,24 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           const bool take = (e < a.M) && (x >= thr[tok]);
           uint32_t bal = __ballot_sync(0xffffffffu, take);
           if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
-          int pos = 0;
-          while (bal) {
+          for (int rk = 0; bal; ++rk) {
             const int bl = __ffs(bal) - 1;
             bal &= bal - 1;
-            // z_lo . R2[:, 32 c + bl], rows split across the lanes
-            const int el = sp * 32 + bl;
-            float part = 0.f;
-#pragma unroll
-            for (int i = lane; i < R; i += 32) {
-              const float zl = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                  zs + zs_offset<R, KCAP>(tok, (R + i) >> 3) + (i & 7) * 2));
-              const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(r2t + r2_offset<R>(i, el)));
-              part = fmaf(zl, w, part);
+            const float xb = __shfl_sync(0xffffffffu, x, bl);
+            if (ncand == kPairBatch) {  // rare: flush a full list first
+              correct_and_store<R, KCAP>(ncand, cinfo, cx, zs, r2t, sp, c, lane, cand, pool, poolcnt);
+              ncand = 0;
             }
 #pragma unroll
-            for (int d = 16; d > 0; d >>= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
-            const float xv = __shfl_sync(0xffffffffu, x, bl) + part;
-            if (lane == 0) {
-              const uint2 cv = make_uint2(__float_as_uint(xv), (uint32_t)(32 * c + bl));
-              if (pos < S) {
-                cand[(tok * KL + slot) * S + pos] = cv;
-              } else {  // rare: more candidates than the pair's slots
-                const int ps = atomicAdd(&poolcnt[tok], 1);
-                if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
+            for (int j = 0; j < kPairBatch; ++j)
+              if (j == ncand) {
+                cinfo[j] = (uint32_t)tok | ((uint32_t)slot << 8) | ((uint32_t)bl << 16) | ((uint32_t)rk << 24);
+                cx[j] = xb;
               }
-            }
-            ++pos;
+            ++ncand;
           }
         }
+        if (ncand) correct_and_store<R, KCAP>(ncand, cinfo, cx, zs, r2t, sp, c, lane, cand, pool, poolcnt);
       }
       tc_fence_before();
       __syncwarp();
