@@ -54,7 +54,7 @@ constexpr int kBE = 128;        // experts per logit tile
 constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
 constexpr int kConsumerThreads = 512;
 constexpr int kConsumerWarps = 16;
-constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass 2
+constexpr int kPairBatch = 8;   // TMEM column loads in flight per warp in pass 2
 constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than S candidates
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -349,9 +349,11 @@ __device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32
         const uint32_t d = tmem_base + ds * 128;
         const uint32_t r2 = r20 + st * C::R2_STAGE;
 #pragma unroll
-        for (int kk = 0; kk < R / 16; ++kk) {  // z_hi only; z_lo enters through the CUDA-core correction
+        // pass 1 reads z_hi only (K = r); pass 2 reads z_hi | z_lo (K = 2r) for exact logits
+        const int ksteps = pass == 0 ? R / 16 : C::RK / 16;
+        for (int kk = 0; kk < ksteps; ++kk) {
           uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
-          uint64_t rd = smem_desc(r2 + kk * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
+          uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
           if (pass == 0)
             mma_bf16(d, zd, rd, C::IDESC_P1, kk != 0);
           else
@@ -434,50 +436,6 @@ template <int R>
 __device__ __forceinline__ uint32_t r2_offset(int i, int e_local) {
   const int box = e_local >> 6, col = e_local & 63;
   return (uint32_t)(box * (64 * R * 2) + i * 128 + ((((col >> 3) ^ (i & 7))) << 4) + (col & 7) * 2);
-}
-
-// z_lo . R2[:, e] for up to kPairBatch candidates at once (rows split across lanes,
-// independent chains and reductions), then the corrected logits into the candidate slots.
-template <int R, int KCAP>
-__device__ __forceinline__ void correct_and_store(int ncand, const uint32_t* cinfo, const float* cx,
-                                                  const uint8_t* zs, const uint8_t* r2t, int sp, int c,
-                                                  int lane, uint2* cand, uint2* pool, int* poolcnt) {
-  constexpr int KL = Cfg<R, KCAP>::KL, S = Cfg<R, KCAP>::S;
-  float part[kPairBatch];
-#pragma unroll
-  for (int j = 0; j < kPairBatch; ++j) {
-    part[j] = 0.f;
-    if (j < ncand) {
-      const int tok = cinfo[j] & 0xff, el = sp * 32 + ((cinfo[j] >> 16) & 0xff);
-#pragma unroll
-      for (int i = lane; i < R; i += 32) {
-        const float zl = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-            zs + zs_offset<R, KCAP>(tok, (R + i) >> 3) + (i & 7) * 2));
-        const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(r2t + r2_offset<R>(i, el)));
-        part[j] = fmaf(zl, w, part[j]);
-      }
-    }
-  }
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1)
-#pragma unroll
-    for (int j = 0; j < kPairBatch; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], d);
-  if (lane == 0) {
-#pragma unroll
-    for (int j = 0; j < kPairBatch; ++j) {
-      if (j < ncand) {
-        const int tok = cinfo[j] & 0xff, slot = (cinfo[j] >> 8) & 0xff, bl = (cinfo[j] >> 16) & 0xff;
-        const int rk = cinfo[j] >> 24;
-        const uint2 cv = make_uint2(__float_as_uint(cx[j] + part[j]), (uint32_t)(32 * c + bl));
-        if (rk < S) {
-          cand[(tok * KL + slot) * S + rk] = cv;
-        } else {  // rare: more candidates than the pair's slots
-          const int ps = atomicAdd(&poolcnt[tok], 1);
-          if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
-        }
-      }
-    }
-  }
 }
 
 template <int R, int KCAP>
@@ -678,12 +636,15 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       for (int i = 0; i < KL; ++i)
         if (i == a.k - 1) kth = kl[i];
       int f = active ? 0 : 2;
-      float wcut = -INFINITY;                  // candidates: approximate logit >= wcut
+      // The k chunks with the largest z_hi maxima (>= tlow) hold k elements whose exact logit
+      // is >= tlow - eps, so the exact k-th logit is >= tlow - eps (the candidate cut), and an
+      // element reaching it has a z_hi logit >= tlow - 2 eps (the chunk cut).
+      float ccut = -INFINITY;                  // candidates: exact logit >= ccut
       uint32_t cut_key = 0u;                   // chunks whose key range reaches cut_key are needed
       if ((kth & ~low) >= kRealKey) {
-        const float tlow = ord_inv(kth & ~low);  // <= the k-th largest approximate chunk maximum
-        wcut = __fsub_rd(tlow, __fmul_ru(2.f, eps));
-        cut_key = ord_key(wcut);
+        const float tlow = ord_inv(kth & ~low);  // <= the k-th largest z_hi chunk maximum
+        ccut = __fsub_rd(tlow, eps);
+        cut_key = ord_key(__fsub_rd(tlow, __fmul_ru(2.f, eps)));
         if ((kl[KL - 1] & ~low) >= kRealKey && (kl[KL - 1] | low) >= cut_key) f |= 1;  // list too short
       }
       int needed = 0;
@@ -698,7 +659,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           }
         }
       }
-      thr[t] = wcut;
+      thr[t] = ccut;
       flag[t] = f;
       nq[t] = (uint8_t)needed;
       poolcnt[t] = 0;
@@ -743,61 +704,49 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     }
     if (!consumer_sync(b, 0, a.status)) return;
 
-    // ---------------- pass 2: candidates of the needed chunks, corrected by z_lo -----------
-    // lane group sp of the transposed tile is chunk 4 pt + sp; its pairs are split among the
-    // four warpgroups.  A candidate's logit is its z_hi value plus z_lo . R2[:, e], computed
-    // here while the R2 tile is still in shared memory.
+    // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
+    // Lane group sp of the transposed tile is chunk 4 pt + sp.  All pairs of a tile's chunk
+    // go to warpgroup pt % 4, so consecutive tiles are worked by different warps.
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
       tc_fence_after();
-      int st;
-      if (!r2_stage(pt, st)) return;
-      const uint8_t* r2t = r2s + st * C::R2_STAGE;
       const int c = pt * 4 + sp;
-      const int e = 32 * c + lane;
-      const uint32_t col0 = tmem_base + lane_base + ds * 128;
-      const int lo = (c < p.nchunks) ? cbase[c] : 0;
-      const int hi = (c < p.nchunks) ? cbase[c + 1] : 0;
-      for (int pi = lo + g; pi < hi; pi += 4 * kPairBatch) {
-        uint32_t ent[kPairBatch], val[kPairBatch];
+      if ((pt & 3) == g && c < p.nchunks) {
+        const int e = 32 * c + lane;
+        const uint32_t col0 = tmem_base + lane_base + ds * 128;
+        const int lo = cbase[c], hi = cbase[c + 1];
+        for (int pi = lo; pi < hi; pi += kPairBatch) {
+          uint32_t ent[kPairBatch], val[kPairBatch];
+          const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
 #pragma unroll
-        for (int q = 0; q < kPairBatch; ++q) {
-          const int pj = pi + 4 * q;
-          ent[q] = (pj < hi) ? pairs[pj] : 0xffffffffu;
-          if (ent[q] != 0xffffffffu) val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
-        }
-        tmem_wait_ld();
-        reg_fence<kPairBatch>(val);
-        // collect the batch's candidates (warp-uniform), then correct them together
-        int ncand = 0;
-        uint32_t cinfo[kPairBatch];  // token | slot << 8 | lane << 16 | (rank within the pair) << 24
-        float cx[kPairBatch];
-#pragma unroll
-        for (int q = 0; q < kPairBatch; ++q) {
-          if (ent[q] == 0xffffffffu) break;
-          const int tok = ent[q] & 0xff, slot = ent[q] >> 8;
-          const float x = __uint_as_float(val[q]);
-          const bool take = (e < a.M) && (x >= thr[tok]);
-          uint32_t bal = __ballot_sync(0xffffffffu, take);
-          if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
-          for (int rk = 0; bal; ++rk) {
-            const int bl = __ffs(bal) - 1;
-            bal &= bal - 1;
-            const float xb = __shfl_sync(0xffffffffu, x, bl);
-            if (ncand == kPairBatch) {  // rare: flush a full list first
-              correct_and_store<R, KCAP>(ncand, cinfo, cx, zs, r2t, sp, c, lane, cand, pool, poolcnt);
-              ncand = 0;
+          for (int q = 0; q < kPairBatch; ++q) {
+            if (q < nb) {
+              ent[q] = pairs[pi + q];
+              val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
             }
+          }
+          tmem_wait_ld();
+          reg_fence<kPairBatch>(val);
 #pragma unroll
-            for (int j = 0; j < kPairBatch; ++j)
-              if (j == ncand) {
-                cinfo[j] = (uint32_t)tok | ((uint32_t)slot << 8) | ((uint32_t)bl << 16) | ((uint32_t)rk << 24);
-                cx[j] = xb;
+          for (int q = 0; q < kPairBatch; ++q) {
+            if (q >= nb) break;
+            const int tok = ent[q] & 0xff, slot = ent[q] >> 8;
+            const float x = __uint_as_float(val[q]);
+            const bool take = (e < a.M) && (x >= thr[tok]);
+            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+            const int pos = __popc(bal & ((1u << lane) - 1u));
+            if (take) {
+              const uint2 cv = make_uint2(val[q], (uint32_t)e);
+              if (pos < S) {
+                cand[(tok * KL + slot) * S + pos] = cv;
+              } else {  // rare: more candidates than the pair's slots
+                const int ps = atomicAdd(&poolcnt[tok], 1);
+                if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
               }
-            ++ncand;
+            }
+            if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
           }
         }
-        if (ncand) correct_and_store<R, KCAP>(ncand, cinfo, cx, zs, r2t, sp, c, lane, cand, pool, poolcnt);
       }
       tc_fence_before();
       __syncwarp();
