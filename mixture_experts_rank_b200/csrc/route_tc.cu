@@ -715,36 +715,44 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         const int e = 32 * c + lane;
         const uint32_t col0 = tmem_base + lane_base + ds * 128;
         const int lo = cbase[c], hi = cbase[c + 1];
+        const uint32_t lt_mask = (1u << lane) - 1u;
         for (int pi = lo; pi < hi; pi += kPairBatch) {
-          uint32_t ent[kPairBatch], val[kPairBatch];
+          // straight-line batch: all loads first, then the ballots, then predicated stores
           const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
+          uint32_t ent[kPairBatch], val[kPairBatch], bal[kPairBatch];
+          float th[kPairBatch];
 #pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) {
-            if (q < nb) {
-              ent[q] = pairs[pi + q];
-              val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
-            }
-          }
+          for (int q = 0; q < kPairBatch; ++q) ent[q] = (q < nb) ? pairs[pi + q] : 0u;
+#pragma unroll
+          for (int q = 0; q < kPairBatch; ++q)
+            if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
+#pragma unroll
+          for (int q = 0; q < kPairBatch; ++q) th[q] = thr[ent[q] & 0xffu];
           tmem_wait_ld();
           reg_fence<kPairBatch>(val);
+          uint32_t over = 0u;
 #pragma unroll
           for (int q = 0; q < kPairBatch; ++q) {
-            if (q >= nb) break;
+            bal[q] = __ballot_sync(0xffffffffu, q < nb && e < a.M && __uint_as_float(val[q]) >= th[q]);
+            over |= (uint32_t)(__popc(bal[q]) > S) << q;
+          }
+#pragma unroll
+          for (int q = 0; q < kPairBatch; ++q) {
             const int tok = ent[q] & 0xff, slot = ent[q] >> 8;
-            const float x = __uint_as_float(val[q]);
-            const bool take = (e < a.M) && (x >= thr[tok]);
-            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-            const int pos = __popc(bal & ((1u << lane) - 1u));
-            if (take) {
-              const uint2 cv = make_uint2(val[q], (uint32_t)e);
-              if (pos < S) {
-                cand[(tok * KL + slot) * S + pos] = cv;
-              } else {  // rare: more candidates than the pair's slots
+            const int pos = __popc(bal[q] & lt_mask);
+            if (((bal[q] >> lane) & 1u) && pos < S) cand[(tok * KL + slot) * S + pos] = make_uint2(val[q], (uint32_t)e);
+            if (lane == 0 && q < nb) pc[tok * KL + slot] = (uint8_t)__popc(bal[q]);
+          }
+          if (over) {  // rare: more candidates than a pair's slots go to the token's pool
+#pragma unroll
+            for (int q = 0; q < kPairBatch; ++q) {
+              const int tok = ent[q] & 0xff;
+              const int pos = __popc(bal[q] & lt_mask);
+              if (((bal[q] >> lane) & 1u) && pos >= S) {
                 const int ps = atomicAdd(&poolcnt[tok], 1);
-                if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
+                if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = make_uint2(val[q], (uint32_t)e);
               }
             }
-            if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
           }
         }
       }
