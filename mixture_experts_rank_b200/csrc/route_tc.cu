@@ -724,10 +724,13 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
 #pragma unroll
           for (int q = 0; q < kPairBatch; ++q) ent[q] = (q < nb) ? pairs[pi + q] : 0u;
 #pragma unroll
+          for (int q = 0; q < kPairBatch; ++q) th[q] = thr[ent[q] & 0xffu];
+          // the shared-memory loads above are complete before the TMEM loads are issued
+#pragma unroll
+          for (int q = 0; q < kPairBatch; ++q) asm volatile("" : "+r"(ent[q]), "+f"(th[q]));
+#pragma unroll
           for (int q = 0; q < kPairBatch; ++q)
             if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
-#pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) th[q] = thr[ent[q] & 0xffu];
           tmem_wait_ld();
           reg_fence<kPairBatch>(val);
           uint32_t over = 0u;
