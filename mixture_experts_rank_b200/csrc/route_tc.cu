@@ -148,8 +148,8 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, volat
                                            unsigned int* status) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 31u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if ((spin & 3u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kTimeoutNs) {
         atomicOr(status, MORE_DEVERR_WAIT_TIMEOUT);
