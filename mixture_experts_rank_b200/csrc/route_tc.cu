@@ -54,7 +54,7 @@ constexpr int kBE = 128;        // experts per logit tile
 constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
 constexpr int kConsumerThreads = 512;
 constexpr int kConsumerWarps = 16;
-constexpr int kPairBatch = 8;   // TMEM column loads in flight per warp in pass 2
+constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass 2
 constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than S candidates
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -459,7 +459,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   int* flag = reinterpret_cast<int*>(smem + p.off_flag);
   uint8_t* nq = smem + p.off_nq;
   uint8_t* pc = smem + p.off_pc;
-  uint32_t* pairs = reinterpret_cast<uint32_t*>(smem + p.off_pairs);
+  uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs);
   int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
   int* cbase = reinterpret_cast<int*>(smem + p.off_cbase);
   int* scan = reinterpret_cast<int*>(smem + p.off_scan);
@@ -482,11 +482,12 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     st = rs;
     return wait_bar(&b.r2_full[rs], rph, b.abort_flag, a.status);
   };
-  // This warp is done with the R2 stage of the current logit tile.
-  auto r2_release = [&]() {
+  // This warp is done with the R2 stage of the current logit tile; it arrives for
+  // `count` consumer warps (0: only advance the stage counters).
+  auto r2_release = [&](uint32_t count) {
     if (p.r2_resident) return;
     __syncwarp();
-    if (lane == 0) mbar_arrive(&b.r2_empty[rs]);
+    if (lane == 0 && count) mbar_arrive_count(&b.r2_empty[rs], count);
     if (++rs == p.r2_stages) {
       rs = 0;
       rph ^= 1u;
@@ -581,9 +582,9 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         acc += __shfl_xor_sync(0xffffffffu, acc, 8);
         acc += __shfl_xor_sync(0xffffffffu, acc, 16);
         colmax2 = fmaxf(colmax2, acc);
-        r2_release();
+        r2_release(1);
       } else {
-        r2_release();
+        r2_release(cw == 0 ? kConsumerWarps : 0);  // nobody reads R2 here: one warp arrives for all
       }
       const int c = pt * 4 + g;
       if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
@@ -697,76 +698,71 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     if (!consumer_sync(b, 0, a.status)) return;
     if (g == 0) {
       const int needed = nq[t];
+      const float cut = thr[t];
       for (int i = 0; i < needed; ++i) {
         const uint32_t st = stage[t * KL + i];
-        pairs[cbase[st & 0xffffu] + (st >> 16)] = (uint32_t)t | ((uint32_t)i << 8);
+        pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(cut));
       }
     }
     if (!consumer_sync(b, 0, a.status)) return;
 
     // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
-    // Lane group sp of the transposed tile is chunk 4 pt + sp.  All pairs of a tile's chunk
-    // go to warpgroup pt % 4, so consecutive tiles are worked by different warps.
+    // Lane group sp of the transposed tile is chunk 4 pt + sp.  Tile pt belongs to
+    // warpgroup pt % 4: its four warps (one per lane group) take all pairs of their chunk
+    // and release the tile for all sixteen consumer warps; the other warps skip it.
     for (int pt = 0; pt < p.p_count; ++pt) {
-      if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
-      tc_fence_after();
-      const int c = pt * 4 + sp;
-      if ((pt & 3) == g && c < p.nchunks) {
-        const int e = 32 * c + lane;
-        const uint32_t col0 = tmem_base + lane_base + ds * 128;
-        const int lo = cbase[c], hi = cbase[c + 1];
-        const uint32_t lt_mask = (1u << lane) - 1u;
-        for (int pi = lo; pi < hi; pi += kPairBatch) {
-          // straight-line batch: all loads first, then the ballots, then predicated stores
-          const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
-          uint32_t ent[kPairBatch], val[kPairBatch], bal[kPairBatch];
-          float th[kPairBatch];
+      if ((pt & 3) == g) {
+        if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
+        tc_fence_after();
+        const int c = pt * 4 + sp;
+        if (c < p.nchunks) {
+          const int e = 32 * c + lane;
+          const uint32_t col0 = tmem_base + lane_base + ds * 128;
+          const uint32_t lt_mask = (1u << lane) - 1u;
+          const int lo = cbase[c], hi = cbase[c + 1];
+          for (int pi = lo; pi < hi; pi += kPairBatch) {
+            const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
+            uint2 ent[kPairBatch];
+            uint32_t val[kPairBatch];
 #pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) ent[q] = (q < nb) ? pairs[pi + q] : 0u;
+            for (int q = 0; q < kPairBatch; ++q)
+              if (q < nb) ent[q] = pairs[pi + q];  // {token | slot << 8, candidate cut}
 #pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) th[q] = thr[ent[q] & 0xffu];
-          // the shared-memory loads above are complete before the TMEM loads are issued
-#pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) asm volatile("" : "+r"(ent[q]), "+f"(th[q]));
-#pragma unroll
-          for (int q = 0; q < kPairBatch; ++q)
-            if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q] & 0xffu));
-          tmem_wait_ld();
-          reg_fence<kPairBatch>(val);
-          uint32_t over = 0u;
-#pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) {
-            bal[q] = __ballot_sync(0xffffffffu, q < nb && e < a.M && __uint_as_float(val[q]) >= th[q]);
-            over |= (uint32_t)(__popc(bal[q]) > S) << q;
-          }
-#pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) {
-            const int tok = ent[q] & 0xff, slot = ent[q] >> 8;
-            const int pos = __popc(bal[q] & lt_mask);
-            if (((bal[q] >> lane) & 1u) && pos < S) cand[(tok * KL + slot) * S + pos] = make_uint2(val[q], (uint32_t)e);
-            if (lane == 0 && q < nb) pc[tok * KL + slot] = (uint8_t)__popc(bal[q]);
-          }
-          if (over) {  // rare: more candidates than a pair's slots go to the token's pool
+            for (int q = 0; q < kPairBatch; ++q)
+              if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q].x & 0xffu));
+            tmem_wait_ld();
+            reg_fence<kPairBatch>(val);
 #pragma unroll
             for (int q = 0; q < kPairBatch; ++q) {
-              const int tok = ent[q] & 0xff;
-              const int pos = __popc(bal[q] & lt_mask);
-              if (((bal[q] >> lane) & 1u) && pos >= S) {
-                const int ps = atomicAdd(&poolcnt[tok], 1);
-                if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = make_uint2(val[q], (uint32_t)e);
+              if (q >= nb) break;
+              const uint32_t bal =
+                  __ballot_sync(0xffffffffu, e < a.M && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y));
+              const int tok = ent[q].x & 0xff, slot = (ent[q].x >> 8) & 0xff;
+              const int pos = __popc(bal & lt_mask);
+              if ((bal >> lane) & 1u) {
+                const uint2 cv = make_uint2(val[q], (uint32_t)e);
+                if (pos < S) {
+                  cand[(tok * KL + slot) * S + pos] = cv;
+                } else {  // rare: more candidates than the pair's slots
+                  const int ps = atomicAdd(&poolcnt[tok], 1);
+                  if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
+                }
               }
+              if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_count(&b.d_empty[ds], kConsumerWarps / 4);
+        r2_release(kConsumerWarps / 4);
+      } else {
+        r2_release(0);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b.d_empty[ds]);
       if (++ds == C::ND) {
         ds = 0;
         dph ^= 1u;
       }
-      r2_release();
     }
     if (!consumer_sync(b, 0, a.status)) return;
 
@@ -944,8 +940,8 @@ uint32_t plan(Params& p) {
         off += kBT * 4;
         p.off_flag = off;
         off += kBT * 4;
-        p.off_pairs = off;
-        off += kBT * C::KL * 4;
+        p.off_pairs = off = align_up(off, 8);
+        off += kBT * C::KL * 8;
         p.off_ccount = off;
         off += p.nchunks * 4;
         p.off_cbase = off;
