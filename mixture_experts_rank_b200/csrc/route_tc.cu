@@ -709,10 +709,12 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
     // Lane group sp of the transposed tile is chunk 4 pt + sp.  Tile pt belongs to
     // warpgroup pt % 4: its four warps (one per lane group) take all pairs of their chunk
-    // and release the tile for all sixteen consumer warps; the other warps skip it.
+    // and release the tile for all sixteen consumer warps.  Every warp still waits for
+    // every tile: a warp that skipped a wait could reach a buffer's next phase while the
+    // previous one is incomplete, and a parity wait cannot tell those two apart.
     for (int pt = 0; pt < p.p_count; ++pt) {
+      if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
       if ((pt & 3) == g) {
-        if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
         tc_fence_after();
         const int c = pt * 4 + sp;
         if (c < p.nchunks) {
