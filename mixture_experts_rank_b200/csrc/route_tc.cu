@@ -160,9 +160,11 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, volat
   }
 }
 
+// The first attempt suspends in hardware until the phase completes (or ~65 us pass),
+// so a normal wait is one instruction and the bounded loop is a rare call.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                          unsigned int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity, 65536u)) return true;
   return wait_bar_slow(bar, parity, abort_flag, status);
 }
 
@@ -400,7 +402,7 @@ __device__ __forceinline__ void write_token(const RouteArgs& a, int64_t n, const
       a.out_idx[o + j] = sel.i[j];
       a.out_gate[o + j] = ex[j] * inv;
       if (a.out_logits) a.out_logits[o + j] = sel.v[j];
-      atomicAdd(a.out_count + sel.i[j], 1);
+      if ((unsigned)sel.i[j] < (unsigned)a.M) atomicAdd(a.out_count + sel.i[j], 1);
     }
   }
 }

@@ -173,7 +173,7 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t* v) {
 template <int N>
 __device__ __forceinline__ void reg_fence(uint32_t* v) {
 #pragma unroll
-  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(v[i])::"memory");
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(v[i]));
 }
 
 // ---- descriptors ------------------------------------------------------------------

@@ -164,7 +164,7 @@ __device__ __forceinline__ void warp_write_selection(const RouteArgs& a, int64_t
     a.out_idx[o] = e;
     a.out_gate[o] = ex / sum;
     if (a.out_logits) a.out_logits[o] = v;
-    atomicAdd(a.out_count + e, 1);
+    if ((unsigned)e < (unsigned)a.M) atomicAdd(a.out_count + e, 1);
   }
 }
 
