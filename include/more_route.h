@@ -110,6 +110,32 @@ more_status more_route_unfused(const void* X, const void* R1, const void* R2, in
                                size_t scratch_bytes, void* stream);
 
 /*
+ * more_route_unfused with no scratch argument: its scratch is a fixed array of
+ * MORE_STATIC_SCRATCH_BYTES bytes inside the library, so the call allocates
+ * nothing.  This entry point has no counterpart in the MoRE paper; it is for
+ * callers that may not allocate device memory themselves, e.g. code running
+ * under an external allocator or memory budget that forbids raw allocations,
+ * or latency-critical paths where a cudaMalloc (which can synchronise the
+ * device) is not acceptable.
+ *   - Limit: a problem needing more than MORE_STATIC_SCRATCH_BYTES of scratch
+ *     (more_route_unfused_scratch_bytes(N, r, M)) returns MORE_ERR_UNSUPPORTED.
+ *   - The array exists once per device for as long as the library is loaded,
+ *     on every device that loads it, whether or not this call is used.
+ *   - The first call on a device looks up the array's device address (one
+ *     cudaGetSymbolAddress with that device current); make that first call
+ *     before starting any stream capture.
+ *   - All calls share the array and it keeps the last call's contents (every
+ *     call overwrites the part it reads).  Calls that may overlap on the GPU
+ *     (different streams, or different host threads without ordering) race on
+ *     it and give wrong results; serialise them.
+ * Arguments, validation and results are those of more_route_unfused.
+ */
+#define MORE_STATIC_SCRATCH_BYTES (32u << 20)
+more_status more_route_unfused_static(const void* X, const void* R1, const void* R2, int64_t N, int h,
+                                      int r, int M, int k, int32_t* out_idx, float* out_gate,
+                                      int32_t* out_expert_count, float* out_logits, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the library's device error word
  * on the current device: MORE_OK if no kernel recorded an error since the last
  * call, MORE_ERR_DEVICE if one did (e.g. a bounded wait gave up), or

@@ -20,7 +20,7 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "route_unfused", "unfused_scratch_bytes", "device_status", "Router", "MoreError",
+__all__ = ["route", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status", "Router", "MoreError",
            "VARIANTS", "library_path", "abi_version", "KMAX"]
 
 KMAX = 16
@@ -46,6 +46,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_variant.argtypes = route_args + [I, P]
     lib.more_route_unfused.restype = I
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
+    lib.more_route_unfused_static.restype = I
+    lib.more_route_unfused_static.argtypes = route_args + [P]
     lib.more_route_unfused_scratch_bytes.restype = ctypes.c_size_t
     lib.more_route_unfused_scratch_bytes.argtypes = [I64, I, I]
     lib.more_device_status.restype = I
@@ -144,6 +146,25 @@ def route_unfused(X, R1, R2, k: int, *, scratch: torch.Tensor | None = None, out
                                  _ptr(outs[2]), _ptr(outs[3]), _ptr(scratch), scratch.numel(),
                                  _stream_handle(stream))
     _check(st, "more_route_unfused")
+    return outs
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def route_unfused_static(X, R1, R2, k: int, *, out_idx=None, out_gate=None, out_expert_count=None,
+                         out_logits=None, return_logits: bool = True, stream=None):
+    """:func:`route_unfused` without a scratch tensor: the library's fixed scratch
+    (``STATIC_SCRATCH_BYTES``) is used, so nothing is allocated for it.  For callers that
+    may not allocate device memory; calls that overlap on the GPU share the scratch and race.
+    """
+    X, R1, R2 = _as_bf16(X, "X"), _as_bf16(R1, "R1"), _as_bf16(R2, "R2")
+    N, h = X.shape
+    r, M = R2.shape
+    outs = _outputs(N, k, M, X.device, out_idx, out_gate, out_expert_count, out_logits, return_logits)
+    st = _lib.more_route_unfused_static(_ptr(X), _ptr(R1), _ptr(R2), N, h, r, M, k, _ptr(outs[0]),
+                                        _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), _stream_handle(stream))
+    _check(st, "more_route_unfused_static")
     return outs
 
 
