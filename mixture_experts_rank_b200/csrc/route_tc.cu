@@ -56,6 +56,7 @@ constexpr int kConsumerThreads = 512;
 constexpr int kConsumerWarps = 16;
 constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass 2
 constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than S candidates
+constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint32_t kRealKey = 0x00800000u;  // ordered value of -FLT_MAX: keys below are not real chunks
@@ -72,7 +73,7 @@ struct Params {
   int x_stages;
   int r2_stages;
   int r2_resident;   // every expert tile stays in shared memory
-  uint32_t off_x, off_r1, off_r2, off_zs, off_lists, off_cand, off_thr, off_flag, off_nq, off_pc, off_pairs,
+  uint32_t off_x, off_r1, off_r2, off_zs, off_lists, off_cand, off_thr, off_flag, off_nq, off_fb, off_pc, off_pairs,
       off_ccount, off_cbase, off_scan, off_pool, off_poolcnt, off_znorm, off_cnorm, off_bar;
 };
 
@@ -407,24 +408,72 @@ __device__ __forceinline__ void write_token(const RouteArgs& a, int64_t n, const
   }
 }
 
-// Exact warp-wide recomputation of one token's top-k on CUDA cores (ties at the
-// threshold, candidate overflow).  Lanes take expert pairs in increasing order.
+// Exact recomputation on CUDA cores of the logits of one token (ties at the threshold,
+// candidate overflow), for the 256-expert block eb .. eb + 255: lane l takes experts
+// eb + 8 l .. eb + 8 l + 7 (one 16-byte load per R2 row) and inserts them into its list
+// in increasing index order.  zr holds z_i (z_hi + z_lo) in lane i mod 32 of entry i / 32.
 template <int R, int KCAP>
-__device__ void fallback_token(const RouteArgs& a, const uint8_t* zs, int t, int64_t n, int lane) {
+__device__ __forceinline__ void fallback_block(const RouteArgs& a, const float (&zr)[(R + 31) / 32], int eb,
+                                               int lane, TopList<KCAP>& list) {
+  constexpr int L = R < 32 ? R : 32;
+  const int e0 = eb + 8 * lane;
+  const bool ok = e0 < a.M;  // M is a multiple of 8, so the lane's 8 experts are all in range
+  const uint4* src = reinterpret_cast<const uint4*>(a.R2) + (ok ? (e0 >> 3) : 0);
+  const size_t rowv = (size_t)(a.M >> 3);
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+  for (int j = 0; j < (R + 31) / 32; ++j) {
+#pragma unroll 4
+    for (int l = 0; l < L; ++l) {
+      const float zi = __shfl_sync(0xffffffffu, zr[j], l);
+      const uint4 w = ok ? __ldg(src + (size_t)(32 * j + l) * rowv) : make_uint4(0u, 0u, 0u, 0u);
+      const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(wp[q]);
+        acc[2 * q] = fmaf(zi, f.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(zi, f.y, acc[2 * q + 1]);
+      }
+    }
+  }
+  if (ok) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) list.insert(acc[q], e0 + q);
+  }
+}
+
+// The cooperative fallback's first step: this warp's partial top-k (over the 256-expert
+// blocks cw, cw + 16, ...) of each of the nb tokens in tok, written to part.
+template <int R, int KCAP>
+__device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t* zs, const uint8_t* tok, int nb,
+                                           uint2* part, int cw, int lane) {
+  for (int j = 0; j < nb; ++j) {
+    const int tf = tok[j];
+    float zr[(R + 31) / 32];
+#pragma unroll
+    for (int q = 0; q < (R + 31) / 32; ++q)
+      zr[q] = (32 * q + lane < R) ? zs_value<R, KCAP>(zs, tf, 32 * q + lane) : 0.f;
+    TopList<KCAP> list;
+    list.init();
+    for (int eb = 256 * cw; eb < a.M; eb += 256 * kConsumerWarps) fallback_block<R, KCAP>(a, zr, eb, lane, list);
+    float v;
+    int e;
+    warp_merge_topk<KCAP>(list, a.k, lane, v, e);
+    if (lane < KCAP) part[(j * kConsumerWarps + cw) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
+  }
+}
+
+// The second step: merge the sixteen partial lists of one token (part: warp-major, KCAP
+// entries each, the first k valid) and write the token's outputs.
+template <int KCAP>
+__device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* part, int64_t n, int lane) {
   TopList<KCAP> list;
   list.init();
-  const int pitch = a.M >> 1;
-  for (int e = 2 * lane; e < a.M; e += 64) {
-    const __nv_bfloat162* col = reinterpret_cast<const __nv_bfloat162*>(a.R2 + e);
-    float acc0 = 0.f, acc1 = 0.f;
-    for (int i = 0; i < R; ++i) {
-      float zi = zs_value<R, KCAP>(zs, t, i);
-      float2 w = __bfloat1622float2(col[(size_t)i * pitch]);
-      acc0 = fmaf(zi, w.x, acc0);
-      acc1 = fmaf(zi, w.y, acc1);
-    }
-    list.insert(acc0, e);
-    list.insert(acc1, e + 1);
+  for (int q = lane; q < kConsumerWarps * KCAP; q += 32) {
+    const uint2 c = part[q];
+    if ((q % KCAP) < a.k) list.insert_any(__uint_as_float(c.x), (int)c.y);
   }
   float v;
   int e;
@@ -460,6 +509,9 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   float* thr = reinterpret_cast<float*>(smem + p.off_thr);
   int* flag = reinterpret_cast<int*>(smem + p.off_flag);
   uint8_t* nq = smem + p.off_nq;
+  int* fbcount = reinterpret_cast<int*>(smem + p.off_fb);
+  uint8_t* fblist = smem + p.off_fb + 4;
+  uint2* part = reinterpret_cast<uint2*>(smem + p.off_lists);  // fallback partial lists (finalize only)
   uint8_t* pc = smem + p.off_pc;
   uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs);
   int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
@@ -488,8 +540,10 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   // `count` consumer warps (0: only advance the stage counters).
   auto r2_release = [&](uint32_t count) {
     if (p.r2_resident) return;
-    __syncwarp();
-    if (lane == 0 && count) mbar_arrive_count(&b.r2_empty[rs], count);
+    if (count) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive_count(&b.r2_empty[rs], count);
+    }
     if (++rs == p.r2_stages) {
       rs = 0;
       rph ^= 1u;
@@ -666,6 +720,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       flag[t] = f;
       nq[t] = (uint8_t)needed;
       poolcnt[t] = 0;
+      if (t == 0 && g == 0) *fbcount = 0;
     }
     if (!consumer_sync(b, 0, a.status)) return;
     // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty)
@@ -703,7 +758,9 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       const float cut = thr[t];
       for (int i = 0; i < needed; ++i) {
         const uint32_t st = stage[t * KL + i];
-        pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(cut));
+        // {token | candidate slot << 8, candidate cut}; the slot also indexes the pair count
+        pairs[cbase[st & 0xffffu] + (st >> 16)] =
+            make_uint2((uint32_t)t | ((uint32_t)(t * KL + i) << 8), __float_as_uint(cut));
       }
     }
     if (!consumer_sync(b, 0, a.status)) return;
@@ -721,6 +778,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         const int c = pt * 4 + sp;
         if (c < p.nchunks) {
           const int e = 32 * c + lane;
+          const bool e_ok = e < a.M;
           const uint32_t col0 = tmem_base + lane_base + ds * 128;
           const uint32_t lt_mask = (1u << lane) - 1u;
           const int lo = cbase[c], hi = cbase[c + 1];
@@ -736,23 +794,29 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
               if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q].x & 0xffu));
             tmem_wait_ld();
             reg_fence<kPairBatch>(val);
+            // per pair: ballot the experts at or above the cut; the first one takes the
+            // pair's slot, lane 0 records the count, any further ones go to the pool below
+            uint32_t bal[kPairBatch];
+            uint32_t extra = 0u;
 #pragma unroll
             for (int q = 0; q < kPairBatch; ++q) {
-              if (q >= nb) break;
-              const uint32_t bal =
-                  __ballot_sync(0xffffffffu, e < a.M && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y));
-              const int tok = ent[q].x & 0xff, slot = (ent[q].x >> 8) & 0xff;
-              const int pos = __popc(bal & lt_mask);
-              if ((bal >> lane) & 1u) {
-                const uint2 cv = make_uint2(val[q], (uint32_t)e);
-                if (pos < S) {
-                  cand[(tok * KL + slot) * S + pos] = cv;
-                } else {  // rare: more candidates than the pair's slots
+              const bool take = q < nb && e_ok && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y);
+              bal[q] = __ballot_sync(0xffffffffu, take);
+              const uint32_t slot = ent[q].x >> 8;
+              const uint32_t before = bal[q] & lt_mask;
+              if (take && before == 0u) cand[slot] = make_uint2(val[q], (uint32_t)e);
+              if (lane == 0 && q < nb) pc[slot] = (uint8_t)__popc(bal[q]);
+              extra |= bal[q] & (bal[q] - 1u);  // set iff the pair has two or more candidates
+            }
+            if (extra) {  // rare: more candidates than the pair's slot
+#pragma unroll
+              for (int q = 0; q < kPairBatch; ++q) {
+                if (((bal[q] >> lane) & 1u) && (bal[q] & lt_mask)) {
+                  const int tok = ent[q].x & 0xff;
                   const int ps = atomicAdd(&poolcnt[tok], 1);
-                  if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = cv;
+                  if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = make_uint2(val[q], (uint32_t)e);
                 }
               }
-              if (lane == 0) pc[tok * KL + slot] = (uint8_t)__popc(bal);
             }
           }
         }
@@ -771,41 +835,49 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     if (!consumer_sync(b, 0, a.status)) return;
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
-    if (g == 0) {
-      const int64_t n = n0 + t;
-      const int f = flag[t];
-      const bool active = (f & 2) == 0;
+    // warp cw finalizes tokens 8 cw .. 8 cw + 7 (one per lane 0..7)
+    {
+      const int tf = cw * 8 + (lane & 7);
+      const int64_t n = n0 + tf;
+      const int f = flag[tf];
+      const bool mine = lane < 8;
+      const bool active = mine && (f & 2) == 0;
       bool fb = active && (f & 1);
       if (active && !fb) {
         TopList<KCAP> sel;
         sel.init();
-        const int jn = nq[t];
+        const int jn = nq[tf];
         int total = 0;
         for (int q = 0; q < jn; ++q) {
-          const int nc = pc[t * KL + q];
+          const int nc = pc[tf * KL + q];
           total += nc;
-          for (int s2 = 0; s2 < nc && s2 < S; ++s2) {
-            const uint2 cv = cand[(t * KL + q) * S + s2];
+          if (nc > 0) {
+            const uint2 cv = cand[tf * KL + q];
             sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
           }
         }
-        const int np = poolcnt[t];
+        const int np = poolcnt[tf];
         if (np > kPoolSlots) fb = true;
         for (int q = 0; q < np && q < kPoolSlots; ++q) {
-          const uint2 cv = pool[t * kPoolSlots + q];
+          const uint2 cv = pool[tf * kPoolSlots + q];
           sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
         }
         if (total < a.k) fb = true;
         if (!fb) write_token<R, KCAP>(a, n, sel);
       }
-      uint32_t need = __ballot_sync(0xffffffffu, fb);
-      while (need) {
-        const int j = __ffs(need) - 1;
-        need &= need - 1;
-        fallback_token<R, KCAP>(a, zs, sp * 32 + j, n0 + sp * 32 + j, lane);
-      }
+      if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)tf;
     }
     if (!consumer_sync(b, 0, a.status)) return;
+    // fallback tokens, kFbBatch at a time: every consumer warp ranks its 256-expert blocks
+    // (blocks cw, cw + 16, ...) for each token, then warp j merges the 16 partial lists of
+    // the batch's token j and writes it
+    for (int fb0 = 0, nfb = *fbcount; fb0 < nfb; fb0 += kFbBatch) {
+      const int nb = nfb - fb0 < kFbBatch ? nfb - fb0 : kFbBatch;
+      fallback_rank<R, KCAP>(a, zs, fblist + fb0, nb, part, cw, lane);
+      if (!consumer_sync(b, 0, a.status)) return;
+      if (cw < nb) fallback_merge<KCAP>(a, part + cw * kConsumerWarps * KCAP, n0 + fblist[fb0 + cw], lane);
+      if (!consumer_sync(b, 0, a.status)) return;
+    }
   }
 }
 
@@ -937,9 +1009,13 @@ uint32_t plan(Params& p) {
         p.off_zs = off = align_up(off, 1024);
         off += C::ZS_BYTES;
         // candidate slots and the list exchange + pair staging share memory (disjoint lifetimes)
+        // (and, after the finalize, the partial lists of the cooperative fallback)
         const uint32_t cand_bytes = kBT * C::KL * C::S * 8, list_bytes = 3 * kBT * C::KL * 4;
+        const uint32_t part_bytes = kFbBatch * kConsumerWarps * KCAP * 8;
+        uint32_t shared_bytes = cand_bytes > list_bytes ? cand_bytes : list_bytes;
+        if (part_bytes > shared_bytes) shared_bytes = part_bytes;
         p.off_cand = p.off_lists = off = align_up(off, 16);
-        off += cand_bytes > list_bytes ? cand_bytes : list_bytes;
+        off += shared_bytes;
         p.off_thr = off;
         off += kBT * 4;
         p.off_flag = off;
@@ -958,6 +1034,8 @@ uint32_t plan(Params& p) {
         off += (kConsumerWarps + 1) * 4;
         p.off_nq = off;
         off += kBT;
+        p.off_fb = off = align_up(off, 4);  // fallback count, then the tile's fallback tokens
+        off += 4 + kBT;
         p.off_poolcnt = off = align_up(off, 4);
         off += kBT * 4;
         p.off_pool = off = align_up(off, 8);
