@@ -8,34 +8,37 @@
 // the (N, k) selection written), Fig. 12 (gates) and eq. (9) (counts).  The N x M
 // logits exist only in TMEM.
 //
-// How (one persistent CTA per SM, 128-token tiles, 12 warps):
-//   warp 0  TMA producer of X (128 x 64 bf16, 128B swizzle) and R1 (64 x r) stages.
+// How (one persistent CTA per SM, 128-token tiles, 20 warps):
+//   warp 0  TMA producer of X (128 x BK bf16, swizzled) and R1 (BK x r) stages.
 //   warp 1  MMA issuer for Z = X R1: M=128 tokens, N=r, K=16 steps over h, into a
 //           double-buffered TMEM accumulator (the next tile streams while the
 //           current one is routed, so HBM never waits on the top-k).
-//   warp 2  MMA issuer for the logit tiles: pass 1 D[tok, exp] = Z R2 (128 x 128),
-//           pass 2 D^T[exp, tok] = R2^T Z^T.  z enters as the bf16 pair
-//           z_hi + z_lo (K = 2r), which keeps ~16 bits of z.
+//   warp 2  MMA issuer for the logit tiles: pass 1 D[tok, exp] = z_hi R2 (K = r),
+//           pass 2 D^T[exp, tok] = R2^T [z_hi | z_lo]^T (K = 2r, exact to ~16 bits of z).
 //   warp 3  TMA producer of R2 tiles (r x 128 experts); R2 stays resident in
 //           shared memory when it fits, else it is streamed from L2.
-//   warps 4-11  two consumer warpgroups (TMEM lanes = tokens in pass 1, experts
-//           in pass 2):
-//     epilogue  Z from TMEM -> (z_hi, z_lo) bf16 -> shared memory (K-major).
-//     pass 1    every 32-expert chunk of a token is reduced to its maximum and
-//               packed into a 32-bit key (order-preserving value bits above the
-//               chunk id); a branch-free sorted list keeps the best k+2 keys.
-//               The k largest logits lie in the k chunks with the largest
-//               maxima, so the list names every chunk that can hold them.
-//     select    threshold T = the k-th key's value bits (rounded down); the
-//               needed chunks are those whose key is not below T, marked in a
-//               per-chunk token bitmask.
-//     pass 2    each warp owns a 32-expert lane group of the transposed tile;
-//               for every token that needs its chunk it reads that column,
-//               ballots the experts >= T and appends them as candidates.
-//     finalize  one thread per token sorts its few candidates in routing order
+//   warps 4-19  four consumer warpgroups (TMEM lanes = tokens in pass 1, experts
+//           in pass 2; warpgroup g takes lane group warp % 4):
+//     epilogue  Z from TMEM -> (z_hi, z_lo) bf16 pair -> shared memory (K-major),
+//               plus |z_hi|, |z_lo| per token and the largest column norm of R2.
+//     pass 1    every 32-expert chunk of a token is reduced to the maximum of its
+//               z_hi logits, packed into a 32-bit key (order-preserving value bits
+//               above the chunk id); a branch-free sorted list keeps the best
+//               k + 6 keys per warpgroup.
+//     select    the four lists are merged.  z_hi logits differ from the exact ones
+//               by at most eps (|z_lo| times the largest R2 column norm, plus fp32
+//               rounding), so the exact k-th logit is at least tlow - eps (tlow: the
+//               k-th chunk maximum) and only chunks whose maximum reaches
+//               tlow - 2 eps can hold a top-k expert.  (token, chunk) pairs are
+//               bucketed by chunk with a counting sort.
+//     pass 2    the four warps of a tile's owning warpgroup read, for every pair of
+//               their chunk, the token's column and ballot the experts whose exact
+//               logit reaches tlow - eps (the candidates).
+//     finalize  one warp per token ranks its few candidates in routing order
 //               (larger logit, then lower expert), softmax, stores, counts.
-//               Ties at the threshold, candidate overflow or a short list send
-//               the token to an exact warp-wide recomputation on CUDA cores.
+//               A list too short to certify the cut, or more candidates than the
+//               slots hold, sends the token to an exact recomputation on CUDA
+//               cores shared by all sixteen consumer warps.
 // Every barrier wait is bounded (a few seconds); on expiry the kernel records
 // MORE_DEVERR_WAIT_TIMEOUT in the library's device error word and unwinds.
 #include <cudaTypedefs.h>
@@ -80,6 +83,7 @@ struct Params {
 template <int R, int KCAP>
 struct Cfg {
   static constexpr int KL = KCAP + 6;                  // chunk keys kept per token
+  static constexpr int KLP = (KL + 15) & ~15;          // row stride of the candidate slots and counts
   static constexpr int S = 1;                          // candidate slots per (token, needed chunk)
   static constexpr int RK = 2 * R;                     // z_hi | z_lo columns of the z buffer
   static constexpr int BK = R >= 128 ? 32 : 64;        // hidden elements per X stage
@@ -351,9 +355,9 @@ __device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32
         tc_fence_after();
         const uint32_t d = tmem_base + ds * 128;
         const uint32_t r2 = r20 + st * C::R2_STAGE;
-#pragma unroll
         // pass 1 reads z_hi only (K = r); pass 2 reads z_hi | z_lo (K = 2r) for exact logits
         const int ksteps = pass == 0 ? R / 16 : C::RK / 16;
+#pragma unroll
         for (int kk = 0; kk < ksteps; ++kk) {
           uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
           uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
@@ -384,29 +388,6 @@ done:
 }
 
 // ---- consumers ----------------------------------------------------------------------------
-
-template <int R, int KCAP>
-__device__ __forceinline__ void write_token(const RouteArgs& a, int64_t n, const TopList<KCAP>& sel) {
-  const int k = a.k;
-  float top = sel.v[0], sum = 0.f;
-  float ex[KCAP];
-#pragma unroll
-  for (int j = 0; j < KCAP; ++j) {
-    ex[j] = (j < k) ? expf(sel.v[j] - top) : 0.f;
-    sum += ex[j];
-  }
-  const float inv = 1.f / sum;
-  size_t o = (size_t)n * k;
-#pragma unroll
-  for (int j = 0; j < KCAP; ++j) {
-    if (j < k) {
-      a.out_idx[o + j] = sel.i[j];
-      a.out_gate[o + j] = ex[j] * inv;
-      if (a.out_logits) a.out_logits[o + j] = sel.v[j];
-      if ((unsigned)sel.i[j] < (unsigned)a.M) atomicAdd(a.out_count + sel.i[j], 1);
-    }
-  }
-}
 
 // Exact recomputation on CUDA cores of the logits of one token (ties at the threshold,
 // candidate overflow), for the 256-expert block eb .. eb + 255: lane l takes experts
@@ -511,6 +492,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   uint8_t* nq = smem + p.off_nq;
   int* fbcount = reinterpret_cast<int*>(smem + p.off_fb);
   uint8_t* fblist = smem + p.off_fb + 4;
+  uint8_t* fbmark = smem + p.off_fb + 4 + kBT;  // 1: the token's outputs come from the fallback
   uint2* part = reinterpret_cast<uint2*>(smem + p.off_lists);  // fallback partial lists (finalize only)
   uint8_t* pc = smem + p.off_pc;
   uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs);
@@ -711,7 +693,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           if ((kl[i] & ~low) >= kRealKey && (kl[i] | low) >= cut_key) {
             const uint32_t cid = kl[i] & low;
             const int rank = atomicAdd(&ccount[cid], 1);
-            stage[t * KL + i] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
+            stage[i * kBT + t] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
             needed = i + 1;
           }
         }
@@ -757,10 +739,9 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       const int needed = nq[t];
       const float cut = thr[t];
       for (int i = 0; i < needed; ++i) {
-        const uint32_t st = stage[t * KL + i];
-        // {token | candidate slot << 8, candidate cut}; the slot also indexes the pair count
-        pairs[cbase[st & 0xffffu] + (st >> 16)] =
-            make_uint2((uint32_t)t | ((uint32_t)(t * KL + i) << 8), __float_as_uint(cut));
+        const uint32_t st = stage[i * kBT + t];
+        // {token | needed-chunk index << 8, candidate cut}
+        pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(cut));
       }
     }
     if (!consumer_sync(b, 0, a.status)) return;
@@ -802,10 +783,10 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
             for (int q = 0; q < kPairBatch; ++q) {
               const bool take = q < nb && e_ok && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y);
               bal[q] = __ballot_sync(0xffffffffu, take);
-              const uint32_t slot = ent[q].x >> 8;
+              const uint32_t tq = ent[q].x & 0xffu, iq = ent[q].x >> 8;
               const uint32_t before = bal[q] & lt_mask;
-              if (take && before == 0u) cand[slot] = make_uint2(val[q], (uint32_t)e);
-              if (lane == 0 && q < nb) pc[slot] = (uint8_t)__popc(bal[q]);
+              if (take && before == 0u) cand[iq * kBT + tq] = make_uint2(val[q], (uint32_t)e);
+              if (lane == 0 && q < nb) pc[tq * C::KLP + iq] = (uint8_t)__popc(bal[q]);
               extra |= bal[q] & (bal[q] - 1u);  // set iff the pair has two or more candidates
             }
             if (extra) {  // rare: more candidates than the pair's slot
@@ -814,7 +795,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
                 if (((bal[q] >> lane) & 1u) && (bal[q] & lt_mask)) {
                   const int tok = ent[q].x & 0xff;
                   const int ps = atomicAdd(&poolcnt[tok], 1);
-                  if (ps < kPoolSlots) pool[tok * kPoolSlots + ps] = make_uint2(val[q], (uint32_t)e);
+                  if (ps < kPoolSlots) pool[ps * kBT + tok] = make_uint2(val[q], (uint32_t)e);
                 }
               }
             }
@@ -835,39 +816,101 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     if (!consumer_sync(b, 0, a.status)) return;
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
-    // warp cw finalizes tokens 8 cw .. 8 cw + 7 (one per lane 0..7)
+    // Four threads per token (one per warpgroup).  Every thread loads all of the token's
+    // candidates (the slots of its needed chunks, then its pool entries); thread g ranks
+    // candidates g, g + 4, ... in routing order (larger logit, then lower expert) and the
+    // ones of rank < k go to the output staging at their rank, with exp(logit - max).
     {
-      const int tf = cw * 8 + (lane & 7);
-      const int64_t n = n0 + tf;
-      const int f = flag[tf];
-      const bool mine = lane < 8;
-      const bool active = mine && (f & 2) == 0;
-      bool fb = active && (f & 1);
-      if (active && !fb) {
-        TopList<KCAP> sel;
-        sel.init();
-        const int jn = nq[tf];
+      constexpr int NC = KL + kPoolSlots;
+      int32_t* sidx = reinterpret_cast<int32_t*>(pairs);  // staging: [token][k], like the outputs
+      float* sex = reinterpret_cast<float*>(sidx + kBT * a.k);
+      float* slog = sex + kBT * a.k;
+      const int f = flag[t];
+      if ((f & 2) == 0) {
+        const int jn = nq[t], np = poolcnt[t];
+        uint32_t cnt[C::KLP / 4];
+#pragma unroll
+        for (int w = 0; w < C::KLP / 16; ++w) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(pc + t * C::KLP + 16 * w);
+          cnt[4 * w] = q4.x;
+          cnt[4 * w + 1] = q4.y;
+          cnt[4 * w + 2] = q4.z;
+          cnt[4 * w + 3] = q4.w;
+        }
+        // -0 and +0 are equal in routing order: both take the key of +0.  Empty slots take
+        // key 0, below every real value, so they never outrank a candidate.
+        uint32_t o[NC], e[NC];
         int total = 0;
-        for (int q = 0; q < jn; ++q) {
-          const int nc = pc[tf * KL + q];
-          total += nc;
-          if (nc > 0) {
-            const uint2 cv = cand[tf * KL + q];
-            sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
+#pragma unroll
+        for (int q = 0; q < NC; ++q) {
+          bool has;
+          uint2 cv = make_uint2(0u, 0u);
+          if (q < KL) {
+            const int nc = q < jn ? (int)((cnt[q >> 2] >> (8 * (q & 3))) & 0xffu) : 0;
+            total += nc;
+            has = nc > 0;
+            if (has) cv = cand[q * kBT + t];
+          } else {
+            has = q - KL < np;
+            if (has) cv = pool[(q - KL) * kBT + t];
+          }
+          o[q] = has ? ord_key(__uint_as_float(cv.x) + 0.f) : 0u;
+          e[q] = cv.y;
+        }
+        const bool fb = (f & 1) || np > kPoolSlots || total < a.k;
+        if (g == 0) {
+          fbmark[t] = fb ? 1 : 0;
+          if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
+        }
+        if (!fb) {
+          uint32_t top = 0u;
+#pragma unroll
+          for (int q = 0; q < NC; ++q) top = max(top, o[q]);
+          const float vtop = ord_inv(top);
+          for (int q = g; q < NC; q += 4) {
+            uint2 cv = make_uint2(0u, 0u);
+            bool has;
+            if (q < KL) {
+              has = q < jn && pc[t * C::KLP + q] != 0;
+              if (has) cv = cand[q * kBT + t];
+            } else {
+              has = q - KL < np;
+              if (has) cv = pool[(q - KL) * kBT + t];
+            }
+            if (!has) continue;
+            const uint32_t om = ord_key(__uint_as_float(cv.x) + 0.f), em = cv.y;
+            int rank = 0;
+#pragma unroll
+            for (int j = 0; j < NC; ++j) rank += (o[j] > om || (o[j] == om && e[j] < em)) ? 1 : 0;
+            if (rank < a.k) {
+              const float v = ord_inv(om);
+              sidx[t * a.k + rank] = (int)em;
+              sex[t * a.k + rank] = expf(v - vtop);
+              slog[t * a.k + rank] = v;
+              if (em < (uint32_t)a.M) atomicAdd(a.out_count + em, 1);
+            }
           }
         }
-        const int np = poolcnt[tf];
-        if (np > kPoolSlots) fb = true;
-        for (int q = 0; q < np && q < kPoolSlots; ++q) {
-          const uint2 cv = pool[tf * kPoolSlots + q];
-          sel.insert_any(__uint_as_float(cv.x), (int)cv.y);
-        }
-        if (total < a.k) fb = true;
-        if (!fb) write_token<R, KCAP>(a, n, sel);
       }
-      if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)tf;
+      if (!consumer_sync(b, 0, a.status)) return;
+      // gates: each selected exp divided by its token's sum
+      if (g == 0 && (f & 2) == 0 && !fbmark[t]) {
+        float sum = 0.f;
+        for (int j = 0; j < a.k; ++j) sum += sex[t * a.k + j];
+        const float inv = 1.f / sum;
+        for (int j = 0; j < a.k; ++j) sex[t * a.k + j] *= inv;
+      }
+      if (!consumer_sync(b, 0, a.status)) return;
+      // the tile's outputs are contiguous: copy the staging out with coalesced stores
+      const int rows = a.N - n0 < kBT ? (int)(a.N - n0) : kBT;
+      const size_t ob = (size_t)n0 * a.k;
+      for (int x = ctid; x < rows * a.k; x += kConsumerThreads) {
+        if (fbmark[x / a.k]) continue;
+        a.out_idx[ob + x] = sidx[x];
+        a.out_gate[ob + x] = sex[x];
+        if (a.out_logits) a.out_logits[ob + x] = slog[x];
+      }
     }
-    if (!consumer_sync(b, 0, a.status)) return;
     // fallback tokens, kFbBatch at a time: every consumer warp ranks its 256-expert blocks
     // (blocks cw, cw + 16, ...) for each token, then warp j merges the 16 partial lists of
     // the batch's token j and writes it
@@ -1010,7 +1053,7 @@ uint32_t plan(Params& p) {
         off += C::ZS_BYTES;
         // candidate slots and the list exchange + pair staging share memory (disjoint lifetimes)
         // (and, after the finalize, the partial lists of the cooperative fallback)
-        const uint32_t cand_bytes = kBT * C::KL * C::S * 8, list_bytes = 3 * kBT * C::KL * 4;
+        const uint32_t cand_bytes = kBT * C::KLP * C::S * 8, list_bytes = 3 * kBT * C::KL * 4;
         const uint32_t part_bytes = kFbBatch * kConsumerWarps * KCAP * 8;
         uint32_t shared_bytes = cand_bytes > list_bytes ? cand_bytes : list_bytes;
         if (part_bytes > shared_bytes) shared_bytes = part_bytes;
@@ -1020,8 +1063,11 @@ uint32_t plan(Params& p) {
         off += kBT * 4;
         p.off_flag = off;
         off += kBT * 4;
-        p.off_pairs = off = align_up(off, 8);
-        off += kBT * C::KL * 8;
+        p.off_pairs = off = align_up(off, 16);  // pass-2 pairs; in the finalize, the output staging
+        {
+          const uint32_t pair_bytes = kBT * C::KL * 8, staging_bytes = 3 * kBT * KCAP * 4;
+          off += pair_bytes > staging_bytes ? pair_bytes : staging_bytes;
+        }
         p.off_ccount = off;
         off += p.nchunks * 4;
         p.off_cbase = off;
@@ -1034,14 +1080,14 @@ uint32_t plan(Params& p) {
         off += (kConsumerWarps + 1) * 4;
         p.off_nq = off;
         off += kBT;
-        p.off_fb = off = align_up(off, 4);  // fallback count, then the tile's fallback tokens
-        off += 4 + kBT;
+        p.off_fb = off = align_up(off, 4);  // fallback count, the tile's fallback tokens, per-token mark
+        off += 4 + 2 * kBT;
         p.off_poolcnt = off = align_up(off, 4);
         off += kBT * 4;
         p.off_pool = off = align_up(off, 8);
         off += kBT * kPoolSlots * 8;
-        p.off_pc = off;
-        off += kBT * C::KL;
+        p.off_pc = off = align_up(off, 16);
+        off += kBT * C::KLP;
         p.off_bar = off = align_up(off, 8);
         off += kBarBytes;
         const uint32_t total = off + 1024;  // alignment slack of the dynamic base
