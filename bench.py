@@ -217,13 +217,15 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     import mixture_experts_rank_b200 as more
+    from mixture_experts_rank_b200 import shard
     import synthetic as syn
 
     N, h, r, M, k, unit = WORKLOADS[args.workload]
     if args.tokens:
         N = args.tokens
-    # rank i routes tokens [i N, (i+1) N) of one synthetic token set (seed 0)
-    Xh = syn.normal_bf16(0, syn.TENSOR_X, N * world, h, 1.0, unit, rank * N, N)
+    # weak scaling: rank i routes rows [i N, (i+1) N) of one synthetic set of N x world tokens (seed 0)
+    begin, count = shard.shard_range(N * world, world, rank)
+    Xh = syn.normal_bf16(0, syn.TENSOR_X, N * world, h, 1.0, unit, begin, count)
     R1h = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
     R2h = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
 
@@ -284,9 +286,7 @@ def main():
     total_ms = ev[0].elapsed_time(ev[-1])
     per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = shard.max_over_ranks(total_ms, torch.device("cuda", local))
     if more.device_status() != 0:
         raise RuntimeError("a kernel recorded a device error during the timed steps")
     ms = total_ms / args.steps
@@ -311,9 +311,7 @@ def main():
         torch.cuda.synchronize()
         e_ms = t0.elapsed_time(t1) / e_steps
         if dist is not None:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+            e_ms = shard.max_over_ranks(e_ms, torch.device("cuda", local))
         bi, bo = router.bytes_per_call(N)
         e2e = {"value": N * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": e_ms}

@@ -1,0 +1,44 @@
+"""Token sharding of the router across ranks (one process per GPU).
+
+Routing is independent per token ("MoRE: Scaling mixture of experts with
+hardware-aware low-rank routing", App. F: every token's top-k depends only on its
+own row of X and the shared R1, R2), so N tokens split into contiguous row
+ranges, one per rank, with R1 and R2 replicated.  No collective is needed on the
+data path; the helpers below are the host-side bookkeeping around it:
+
+* ``shard_range``: the row range of a rank;
+* ``global_expert_counts``: the sum over ranks of the per-rank expert counts
+  (the per-expert load statistic f of App. F eq. (9) over the whole batch), one
+  all-reduce of M integers, outside the routing call;
+* ``max_over_ranks``: the slowest rank's time, which sets the batch's time.
+"""
+from __future__ import annotations
+
+import torch
+
+
+def shard_range(n_total: int, world: int, rank: int) -> tuple[int, int]:
+    """Rows ``[begin, begin + count)`` of ``rank``: contiguous, sizes differ by at most one."""
+    if world < 1 or not 0 <= rank < world or n_total < 0:
+        raise ValueError(f"bad shard request: n_total={n_total} world={world} rank={rank}")
+    base, extra = divmod(n_total, world)
+    begin = rank * base + min(rank, extra)
+    return begin, base + (1 if rank < extra else 0)
+
+
+def global_expert_counts(local_counts: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum of every rank's ``out_expert_count`` (int32 [M]); returns a new int64 tensor."""
+    import torch.distributed as dist
+
+    total = local_counts.to(torch.int64).clone()
+    dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
+    return total
+
+
+def max_over_ranks(value: float, device, group=None) -> float:
+    """The largest of the ranks' values (used for per-step times)."""
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
