@@ -174,13 +174,16 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 }
 
 
-// Barrier of the 16 consumer warps (named barrier 1).  It cannot strand a warp:
-// between two of these barriers every consumer warp performs the same bounded
-// mbarrier waits, so when one gives up (and raises the abort flag) all of them
-// leave at a wait before reaching the next barrier.
-__device__ __forceinline__ bool consumer_sync(const Bars&, int, unsigned int*) {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
-  return true;
+// Barrier of the 16 consumer warps on an mbarrier, so that it is bounded like every
+// other wait: if any role gives up (and raises the abort flag), a warp waiting here
+// leaves too instead of waiting for a warp that has already returned.  `phase` is
+// the calling thread's parity of the barrier, flipped at every use.
+__device__ __forceinline__ bool consumer_sync(const Bars& b, uint32_t& phase, unsigned int* status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(b.cbar);
+  const bool ok = wait_bar(b.cbar, phase, b.abort_flag, status);
+  phase ^= 1u;
+  return ok;
 }
 
 // Order-preserving map of fp32 onto uint32 and its inverse.
@@ -475,6 +478,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
   using C = Cfg<R, KCAP>;
   constexpr int KL = C::KL, S = C::S;
   const RouteArgs& a = p.a;
+  uint32_t cph = 0;  // parity of the consumer barrier
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sp = warp & 3;              // TMEM subpartition: lanes 32 sp .. 32 sp + 31
   const int g = (warp - 4) >> 2;        // consumer warpgroup 0..3
@@ -645,7 +649,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 4));
       if (lane == 0) cnorm[cw] = colmax2;
     }
-    if (!consumer_sync(b, 0, a.status)) return;
+    if (!consumer_sync(b, cph, a.status)) return;
     if (lt == 0 && ctid == 0) {
       float m = 0.f;
       for (int w = 0; w < kConsumerWarps; ++w) m = fmaxf(m, cnorm[w]);
@@ -659,7 +663,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         for (int i = 0; i < KL; ++i) lists[(KL + i) * kBT + t] = kl[i];
       }
     }
-    if (!consumer_sync(b, 0, a.status)) return;
+    if (!consumer_sync(b, cph, a.status)) return;
     if (g == 0) {
 #pragma unroll
       for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(KL + i) * kBT + t]);
@@ -704,7 +708,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       poolcnt[t] = 0;
       if (t == 0 && g == 0) *fbcount = 0;
     }
-    if (!consumer_sync(b, 0, a.status)) return;
+    if (!consumer_sync(b, cph, a.status)) return;
     // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty)
     {
       int vals[4], run = 0;
@@ -721,7 +725,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         if (lane >= d) incl += o;
       }
       if (lane == 31) scan[ctid >> 5] = incl;
-      if (!consumer_sync(b, 0, a.status)) return;
+      if (!consumer_sync(b, cph, a.status)) return;
       int before = incl - run;
       for (int w = 0; w < (ctid >> 5); ++w) before += scan[w];
 #pragma unroll
@@ -734,7 +738,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
       // the end of the last bucket (index nchunks lies past the 4 x 512 slots when nchunks == 2048)
       if (ctid == kConsumerThreads - 1) cbase[p.nchunks] = before;
     }
-    if (!consumer_sync(b, 0, a.status)) return;
+    if (!consumer_sync(b, cph, a.status)) return;
     if (g == 0) {
       const int needed = nq[t];
       const float cut = thr[t];
@@ -744,7 +748,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(cut));
       }
     }
-    if (!consumer_sync(b, 0, a.status)) return;
+    if (!consumer_sync(b, cph, a.status)) return;
 
     // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
     // Lane group sp of the transposed tile is chunk 4 pt + sp.  Tile pt belongs to
@@ -813,7 +817,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         dph ^= 1u;
       }
     }
-    if (!consumer_sync(b, 0, a.status)) return;
+    if (!consumer_sync(b, cph, a.status)) return;
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
     // Four threads per token (one per warpgroup).  Every thread loads all of the token's
@@ -892,7 +896,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           }
         }
       }
-      if (!consumer_sync(b, 0, a.status)) return;
+      if (!consumer_sync(b, cph, a.status)) return;
       // gates: each selected exp divided by its token's sum
       if (g == 0 && (f & 2) == 0 && !fbmark[t]) {
         float sum = 0.f;
@@ -900,7 +904,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         const float inv = 1.f / sum;
         for (int j = 0; j < a.k; ++j) sex[t * a.k + j] *= inv;
       }
-      if (!consumer_sync(b, 0, a.status)) return;
+      if (!consumer_sync(b, cph, a.status)) return;
       // the tile's outputs are contiguous: copy the staging out with coalesced stores
       const int rows = a.N - n0 < kBT ? (int)(a.N - n0) : kBT;
       const size_t ob = (size_t)n0 * a.k;
@@ -917,9 +921,9 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
     for (int fb0 = 0, nfb = *fbcount; fb0 < nfb; fb0 += kFbBatch) {
       const int nb = nfb - fb0 < kFbBatch ? nfb - fb0 : kFbBatch;
       fallback_rank<R, KCAP>(a, zs, fblist + fb0, nb, part, cw, lane);
-      if (!consumer_sync(b, 0, a.status)) return;
+      if (!consumer_sync(b, cph, a.status)) return;
       if (cw < nb) fallback_merge<KCAP>(a, part + cw * kConsumerWarps * KCAP, n0 + fblist[fb0 + cw], lane);
-      if (!consumer_sync(b, 0, a.status)) return;
+      if (!consumer_sync(b, cph, a.status)) return;
     }
   }
 }
