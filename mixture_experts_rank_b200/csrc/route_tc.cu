@@ -752,10 +752,11 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
 
     // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
     // Lane group sp of the transposed tile is chunk 4 pt + sp.  Tile pt belongs to
-    // warpgroup pt % 4: its four warps (one per lane group) take all pairs of their chunk
-    // and release the tile for all sixteen consumer warps.  Every warp still waits for
-    // every tile: a warp that skipped a wait could reach a buffer's next phase while the
-    // previous one is incomplete, and a parity wait cannot tell those two apart.
+    // warpgroup pt % 4: its four warps (one per lane group) take all pairs of their chunk.
+    // Every warp waits for every tile and arrives once on its empty barrier (the owners
+    // when done, the others at once): a buffer is refilled only after all sixteen warps
+    // have seen its current phase, so no warp can fall two phases behind, which a parity
+    // wait could not tell from the phase it waits for.
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
       if ((pt & 3) == g) {
@@ -807,9 +808,11 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_count(&b.d_empty[ds], kConsumerWarps / 4);
+        if (lane == 0) mbar_arrive(&b.d_empty[ds]);
         r2_release(kConsumerWarps / 4);
       } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.d_empty[ds]);
         r2_release(0);
       }
       if (++ds == C::ND) {
