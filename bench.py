@@ -44,6 +44,10 @@ WORKLOADS = {
     "sweep_M8192": (65536, 512, 32, 8192, 8, False),
     "sweep_M16384": (65536, 512, 32, 16384, 8, False),
     "tiny": (4096, 128, 32, 192, 4, False),
+    "decode_N1": (1, 2048, 32, 4096, 8, False),
+    "decode_N8": (8, 2048, 32, 4096, 8, False),
+    "decode_N64": (64, 2048, 32, 4096, 8, False),
+    "decode_N256": (256, 2048, 32, 4096, 8, False),
 }
 METRIC = "routed tokens/s (fused low-rank router + top-k)"
 L2_BYTES = 126 * 1024 * 1024
