@@ -50,6 +50,10 @@ WORKLOADS = {
     "decode_N256": (256, 2048, 32, 4096, 8, False),
 }
 METRIC = "routed tokens/s (fused low-rank router + top-k)"
+# DRAM bytes (read + write) per token of the fused kernel, from the ncu capture summarised in
+# profiles/fused_route_kernel_prefill_r32_n65536.md (N = 65,536, scaled by tokens).  Only valid
+# while that kernel is unchanged; workloads without a capture report traffic null.
+NCU_TRAFFIC_PER_TOKEN = {"prefill_r32": (269.474048e6 + 11.228928e6) / 65536}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -328,6 +332,8 @@ def main():
         kernel_ms = launch_ms if launch_ms is not None else ms
         achieved = x_bytes / (kernel_ms / 1e3) / 1e9
         traffic = None
+        if variant_used == "fused_tc" and args.workload in NCU_TRAFFIC_PER_TOKEN:
+            traffic = NCU_TRAFFIC_PER_TOKEN[args.workload] * N  # bytes per launch
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
                 else "fallback 6.65 TB/s",
