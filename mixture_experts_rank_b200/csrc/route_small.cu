@@ -1,17 +1,21 @@
-// Small-batch (decode-sized) MoRE routing kernel on CUDA cores: one warp per token.
+// Small-batch (decode-sized) MoRE routing kernel on CUDA cores: one CTA of 8 warps
+// per token, so that one token's reads of R1 and R2 are spread over 256 threads.
 //
 // Per token, following "MoRE: Scaling mixture of experts with hardware-aware
 // low-rank routing", App. F, Algorithm 1 (z accumulated in fp32, one sweep over
 // the experts with a running top-k) and Fig. 12 (softmax over the k selected
 // logits):
-//   1. z = x . R1: lanes stride over h, 16 outputs per pass, reduce-scatter
-//      through shuffles; z is carried as the bf16 pair z_hi + z_lo (finer than
-//      Algorithm 1's single bf16) and kept in shared memory.
-//   2. lanes take expert pairs (2 lane + 64 j, +1); each lane keeps a sorted
-//      running top-k of its experts (strict '>' insertion, so on equal logits
-//      the lower expert index stays ahead).
-//   3. k warp-wide arg-max rounds merge the 32 lists in routing order.
-//   4. softmax over the k logits, outputs, and one atomic count per selection.
+//   1. z = x . R1: warp w sums hidden rows w*32 + lane + 256 j, 16 outputs per pass
+//      with a shuffle reduce-scatter; the eight warps' partial sums are added in
+//      shared memory, and z is carried as the bf16 pair z_hi + z_lo (finer than
+//      Algorithm 1's single bf16), as in every kernel of this library.
+//   2. warp w takes the 256-expert blocks w, w + 8, ...: lane l the experts
+//      8 l .. 8 l + 7 of a block (one 16-byte load per R2 row), into a sorted
+//      running top-k of its own (strict '>' insertion in increasing expert order,
+//      so on equal logits the lower expert index stays ahead).
+//   3. k warp-wide arg-max rounds merge each warp's lanes, then warp 0 merges the
+//      eight warp lists in routing order, applies the softmax and writes the outputs
+//      and one atomic count per selection.
 #include "more_internal.cuh"
 #include "warp_simt.cuh"
 
@@ -19,38 +23,133 @@ namespace more {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
+constexpr int kRMax = 128;
 
+// The 16 sums z[b .. b + 16) over this warp's hidden rows (w*32 + lane + 256 j), reduced
+// across the warp by a reduce-scatter: afterwards every value sits on two neighbouring
+// lanes; `value` is this lane's value and `index` its z index.
+__device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict__ x,
+                                                 const __nv_bfloat16* __restrict__ R1, int h, int r, int b,
+                                                 int warp, int lane, float& value, int& index) {
+  float acc[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+  for (int t = warp * 32 + lane; t < h; t += kWarpsPerBlock * 32) {
+    const float xt = __bfloat162float(x[t]);
+    const uint4* w = reinterpret_cast<const uint4*>(R1 + (size_t)t * r + b);
+    const uint4 w0 = __ldg(w), w1 = __ldg(w + 1);
+    const __nv_bfloat162* p0 = reinterpret_cast<const __nv_bfloat162*>(&w0);
+    const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&w1);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 u = __bfloat1622float2(p0[q]);
+      const float2 v = __bfloat1622float2(p1[q]);
+      acc[2 * q] = fmaf(xt, u.x, acc[2 * q]);
+      acc[2 * q + 1] = fmaf(xt, u.y, acc[2 * q + 1]);
+      acc[8 + 2 * q] = fmaf(xt, v.x, acc[8 + 2 * q]);
+      acc[8 + 2 * q + 1] = fmaf(xt, v.y, acc[8 + 2 * q + 1]);
+    }
+  }
+  // reduce-scatter: after the step with distance d a lane keeps the half selected by its bit d
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const bool hi = lane & 16;
+    const float send = hi ? acc[j] : acc[j + 8];
+    acc[j] = (hi ? acc[j + 8] : acc[j]) + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const bool hi = lane & 8;
+    const float send = hi ? acc[j] : acc[j + 4];
+    acc[j] = (hi ? acc[j + 4] : acc[j]) + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const bool hi = lane & 4;
+    const float send = hi ? acc[j] : acc[j + 2];
+    acc[j] = (hi ? acc[j + 2] : acc[j]) + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  {
+    const bool hi = lane & 2;
+    const float send = hi ? acc[0] : acc[1];
+    acc[0] = (hi ? acc[1] : acc[0]) + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+  value = acc[0];
+  index = b + ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
 
 template <int K>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     small_n_route_kernel(RouteArgs a) {
-  extern __shared__ float smem_z[];
+  __shared__ float zpart[kWarpsPerBlock][kRMax];
+  __shared__ float zs[kRMax];
+  __shared__ float pv[kWarpsPerBlock][K];
+  __shared__ int pe[kWarpsPerBlock][K];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* zs = smem_z + warp * a.r;
-  const int64_t stride = (int64_t)gridDim.x * kWarpsPerBlock;
-  for (int64_t n = (int64_t)blockIdx.x * kWarpsPerBlock + warp; n < a.N; n += stride) {
-    warp_project_token(a.X + (size_t)n * a.h, a.R1, a.h, a.r, zs, lane);
-    __syncwarp();
+  for (int64_t n = blockIdx.x; n < a.N; n += gridDim.x) {
+    // 1. z = x . R1
+    const __nv_bfloat16* x = a.X + (size_t)n * a.h;
+    for (int b = 0; b < a.r; b += 16) {
+      float v;
+      int i;
+      warp_partial_z16(x, a.R1, a.h, a.r, b, warp, lane, v, i);
+      if ((lane & 1) == 0) zpart[warp][i] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < a.r) {
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w) z += zpart[w][threadIdx.x];
+      zs[threadIdx.x] = split_bf16_pair(z);
+    }
+    __syncthreads();
+    // 2. this warp's 256-expert blocks
     TopList<K> list;
     list.init();
-    for (int e = 2 * lane; e < a.M; e += 64) {
-      float acc0 = 0.f, acc1 = 0.f;
-      const __nv_bfloat162* col = reinterpret_cast<const __nv_bfloat162*>(a.R2 + e);
-      const int pitch = a.M >> 1;  // row pitch in bf16 pairs
+    const size_t rowv = (size_t)(a.M >> 3);  // 16-byte groups per R2 row
+    for (int eb = 256 * warp; eb < a.M; eb += 256 * kWarpsPerBlock) {
+      const int e0 = eb + 8 * lane;
+      const bool ok = e0 < a.M;  // M is a multiple of 8: the lane's 8 experts are all in range
+      const uint4* src = reinterpret_cast<const uint4*>(a.R2) + (ok ? (e0 >> 3) : 0);
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll 8
       for (int i = 0; i < a.r; ++i) {
-        float zi = zs[i];
-        float2 w = __bfloat1622float2(col[(size_t)i * pitch]);
-        acc0 = fmaf(zi, w.x, acc0);
-        acc1 = fmaf(zi, w.y, acc1);
+        const float zi = zs[i];
+        const uint4 w = ok ? __ldg(src + (size_t)i * rowv) : make_uint4(0u, 0u, 0u, 0u);
+        const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(wp[q]);
+          acc[2 * q] = fmaf(zi, f.x, acc[2 * q]);
+          acc[2 * q + 1] = fmaf(zi, f.y, acc[2 * q + 1]);
+        }
       }
-      list.insert(acc0, e);
-      list.insert(acc1, e + 1);
+      if (ok) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) list.insert(acc[q], e0 + q);
+      }
     }
-    float my_v;
-    int my_i;
-    warp_merge_topk<K>(list, a.k, lane, my_v, my_i);
-    warp_write_selection(a, n, lane, my_v, my_i);
-    __syncwarp();
+    // 3. merge: lanes, then warps
+    float v;
+    int e;
+    warp_merge_topk<K>(list, a.k, lane, v, e);
+    if (lane < K) {
+      pv[warp][lane] = v;
+      pe[warp][lane] = e;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      TopList<K> all;
+      all.init();
+      for (int q = lane; q < kWarpsPerBlock * K; q += 32)
+        if (q % K < a.k) all.insert_any(pv[q / K][q % K], pe[q / K][q % K]);
+      warp_merge_topk<K>(all, a.k, lane, v, e);
+      warp_write_selection(a, n, lane, v, e);
+    }
+    __syncthreads();
   }
 }
 
@@ -59,11 +158,10 @@ cudaError_t launch_k(const RouteArgs& a) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t blocks = (a.N + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  int64_t cap = (int64_t)sms * 8;
+  int64_t blocks = a.N;  // one CTA per token, up to 8 resident per SM
+  const int64_t cap = (int64_t)sms * 8;
   if (blocks > cap) blocks = cap;
-  size_t smem = sizeof(float) * kWarpsPerBlock * a.r;
-  small_n_route_kernel<K><<<(unsigned)blocks, kWarpsPerBlock * 32, smem, a.stream>>>(a);
+  small_n_route_kernel<K><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, a.stream>>>(a);
   return cudaGetLastError();
 }
 
