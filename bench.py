@@ -210,6 +210,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0, help="override N (profiling a smaller case)")
+    ap.add_argument("--launch", default="auto", choices=["auto", "eager", "graph"],
+                    help="graph: each timed step replays a CUDA graph of one routing call (auto: N <= 65536)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -250,13 +252,14 @@ def main():
     if args.variant == "unfused":
         scratch = torch.empty(more.unfused_scratch_bytes(N, r, M), dtype=torch.uint8, device="cuda")
 
-    def step():
+    def step(st=None):
+        st = stream if st is None else st
         if args.variant == "unfused":
             more.route_unfused(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate, out_expert_count=cnt,
-                               out_logits=logits, stream=stream)
+                               out_logits=logits, stream=st)
         else:
             more.route(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
-                       variant=args.variant, stream=stream)
+                       variant=args.variant, stream=st)
 
     variant_used = args.variant
     if args.variant == "auto":
@@ -278,6 +281,17 @@ def main():
     if more.device_status() != 0:
         raise RuntimeError("a kernel recorded a device error during warm-up")
 
+    # small batches are launch-bound: each step is then the replay of a CUDA graph holding
+    # one routing call (the C-ABI call is asynchronous and allocates nothing, so it captures)
+    use_graph = args.launch == "graph" or (args.launch == "auto" and N <= 65536)
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(torch.cuda.current_stream())
+        graph.replay()
+        torch.cuda.synchronize()
+
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -286,7 +300,10 @@ def main():
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     ev[0].record(stream)
     for i in range(args.steps):
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
         ev[i + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -345,6 +362,7 @@ def main():
                 "config": {"workload": describe(args.workload) + (f" (N overridden to {N})" if args.tokens else ""),
                            "N_per_gpu": N, "h": h, "r": r, "M": M, "k": k,
                            "variant": variant_used, "parallelism": f"token shards x{world}",
+                           "launch": "CUDA graph replay of one call per step" if graph is not None else "eager",
                            "l2": f"inputs larger than L2 (X = {x_bytes / 1e9:.2f} GB per GPU)"
                            if x_bytes > L2_BYTES else "inputs fit in L2; no flush (L2-warm)"},
                 "roofline": roof, "gpu_launches": launches_per_step * args.steps, "clocks": clocks}

@@ -1,20 +1,20 @@
-// Small-batch (decode-sized) MoRE routing kernel on CUDA cores: one CTA of 8 warps
-// per token, so that one token's reads of R1 and R2 are spread over 256 threads.
+// Small-batch (decode-sized) MoRE routing kernel on CUDA cores: one CTA of 16 warps
+// per token, so that one token's reads of R1 and R2 are spread over 512 threads.
 //
 // Per token, following "MoRE: Scaling mixture of experts with hardware-aware
 // low-rank routing", App. F, Algorithm 1 (z accumulated in fp32, one sweep over
 // the experts with a running top-k) and Fig. 12 (softmax over the k selected
 // logits):
-//   1. z = x . R1: warp w sums hidden rows w*32 + lane + 256 j, 16 outputs per pass
-//      with a shuffle reduce-scatter; the eight warps' partial sums are added in
+//   1. z = x . R1: warp w sums hidden rows w*32 + lane + 512 j, 16 outputs per pass
+//      with a shuffle reduce-scatter; the sixteen warps' partial sums are added in
 //      shared memory, and z is carried as the bf16 pair z_hi + z_lo (finer than
 //      Algorithm 1's single bf16), as in every kernel of this library.
-//   2. warp w takes the 256-expert blocks w, w + 8, ...: lane l the experts
+//   2. warp w takes the 256-expert blocks w, w + 16, ...: lane l the experts
 //      8 l .. 8 l + 7 of a block (one 16-byte load per R2 row), into a sorted
 //      running top-k of its own (strict '>' insertion in increasing expert order,
 //      so on equal logits the lower expert index stays ahead).
 //   3. k warp-wide arg-max rounds merge each warp's lanes, then warp 0 merges the
-//      eight warp lists in routing order, applies the softmax and writes the outputs
+//      sixteen warp lists in routing order, applies the softmax and writes the outputs
 //      and one atomic count per selection.
 #include "more_internal.cuh"
 #include "warp_simt.cuh"
@@ -22,10 +22,10 @@
 namespace more {
 namespace {
 
-constexpr int kWarpsPerBlock = 8;
+constexpr int kWarpsPerBlock = 16;
 constexpr int kRMax = 128;
 
-// The 16 sums z[b .. b + 16) over this warp's hidden rows (w*32 + lane + 256 j), reduced
+// The 16 sums z[b .. b + 16) over this warp's hidden rows (w*32 + lane + 512 j), reduced
 // across the warp by a reduce-scatter: afterwards every value sits on two neighbouring
 // lanes; `value` is this lane's value and `index` its z index.
 __device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict__ x,
@@ -34,20 +34,33 @@ __device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict
   float acc[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-  for (int t = warp * 32 + lane; t < h; t += kWarpsPerBlock * 32) {
-    const float xt = __bfloat162float(x[t]);
-    const uint4* w = reinterpret_cast<const uint4*>(R1 + (size_t)t * r + b);
-    const uint4 w0 = __ldg(w), w1 = __ldg(w + 1);
-    const __nv_bfloat162* p0 = reinterpret_cast<const __nv_bfloat162*>(&w0);
-    const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&w1);
+  constexpr int kStride = kWarpsPerBlock * 32;
+  // batches of 4 hidden rows: all loads first, then the arithmetic, so the loads overlap
+  for (int t0 = warp * 32 + lane; t0 < h; t0 += 4 * kStride) {
+    float xt[4];
+    uint4 w0[4], w1[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 u = __bfloat1622float2(p0[q]);
-      const float2 v = __bfloat1622float2(p1[q]);
-      acc[2 * q] = fmaf(xt, u.x, acc[2 * q]);
-      acc[2 * q + 1] = fmaf(xt, u.y, acc[2 * q + 1]);
-      acc[8 + 2 * q] = fmaf(xt, v.x, acc[8 + 2 * q]);
-      acc[8 + 2 * q + 1] = fmaf(xt, v.y, acc[8 + 2 * q + 1]);
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + j * kStride;
+      const bool ok = t < h;
+      xt[j] = ok ? __bfloat162float(x[t]) : 0.f;
+      const uint4* w = reinterpret_cast<const uint4*>(R1 + (size_t)(ok ? t : 0) * r + b);
+      w0[j] = ok ? __ldg(w) : make_uint4(0u, 0u, 0u, 0u);
+      w1[j] = ok ? __ldg(w + 1) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162* p0 = reinterpret_cast<const __nv_bfloat162*>(&w0[j]);
+      const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&w1[j]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 u = __bfloat1622float2(p0[q]);
+        const float2 v = __bfloat1622float2(p1[q]);
+        acc[2 * q] = fmaf(xt[j], u.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(xt[j], u.y, acc[2 * q + 1]);
+        acc[8 + 2 * q] = fmaf(xt[j], v.x, acc[8 + 2 * q]);
+        acc[8 + 2 * q + 1] = fmaf(xt[j], v.y, acc[8 + 2 * q + 1]);
+      }
     }
   }
   // reduce-scatter: after the step with distance d a lane keeps the half selected by its bit d
@@ -115,16 +128,21 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       float acc[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < a.r; ++i) {
-        const float zi = zs[i];
-        const uint4 w = ok ? __ldg(src + (size_t)i * rowv) : make_uint4(0u, 0u, 0u, 0u);
-        const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w);
+      // batches of 8 R2 rows (r is a multiple of 16): loads first, then the arithmetic
+      for (int i0 = 0; i0 < a.r; i0 += 8) {
+        uint4 w[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(wp[q]);
-          acc[2 * q] = fmaf(zi, f.x, acc[2 * q]);
-          acc[2 * q + 1] = fmaf(zi, f.y, acc[2 * q + 1]);
+        for (int j = 0; j < 8; ++j) w[j] = ok ? __ldg(src + (size_t)(i0 + j) * rowv) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float zi = zs[i0 + j];
+          const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(wp[q]);
+            acc[2 * q] = fmaf(zi, f.x, acc[2 * q]);
+            acc[2 * q + 1] = fmaf(zi, f.y, acc[2 * q + 1]);
+          }
         }
       }
       if (ok) {
@@ -158,8 +176,8 @@ cudaError_t launch_k(const RouteArgs& a) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t blocks = a.N;  // one CTA per token, up to 8 resident per SM
-  const int64_t cap = (int64_t)sms * 8;
+  int64_t blocks = a.N;  // one CTA per token, up to 4 resident per SM
+  const int64_t cap = (int64_t)sms * 4;
   if (blocks > cap) blocks = cap;
   small_n_route_kernel<K><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, a.stream>>>(a);
   return cudaGetLastError();
