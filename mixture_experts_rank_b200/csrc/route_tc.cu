@@ -752,14 +752,15 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
 
     // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
     // Lane group sp of the transposed tile is chunk 4 pt + sp.  Tile pt belongs to
-    // warpgroup pt % 4: its four warps (one per lane group) take all pairs of their chunk.
-    // Every warp waits for every tile and arrives once on its empty barrier (the owners
-    // when done, the others at once): a buffer is refilled only after all sixteen warps
-    // have seen its current phase, so no warp can fall two phases behind, which a parity
-    // wait could not tell from the phase it waits for.
+    // warpgroups 0-1 when pt is even, 2-3 when odd: the two warps of a lane group split the
+    // pairs of their chunk (first and second half), so a tile is worked by eight warps and
+    // two tiles at once.  Every warp waits for every tile and arrives once on its empty
+    // barrier (the owners when done, the others at once): a buffer is refilled only after
+    // all sixteen warps have seen its current phase, so no warp can fall two phases
+    // behind, which a parity wait could not tell from the phase it waits for.
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
-      if ((pt & 3) == g) {
+      if ((pt & 1) == (g >> 1)) {
         tc_fence_after();
         const int c = pt * 4 + sp;
         if (c < p.nchunks) {
@@ -767,7 +768,8 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
           const bool e_ok = e < a.M;
           const uint32_t col0 = tmem_base + lane_base + ds * 128;
           const uint32_t lt_mask = (1u << lane) - 1u;
-          const int lo = cbase[c], hi = cbase[c + 1];
+          const int c_lo = cbase[c], c_hi = cbase[c + 1], c_mid = (c_lo + c_hi + 1) >> 1;
+          const int lo = (g & 1) ? c_mid : c_lo, hi = (g & 1) ? c_hi : c_mid;
           for (int pi = lo; pi < hi; pi += kPairBatch) {
             const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
             uint2 ent[kPairBatch];
@@ -809,7 +811,7 @@ __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.d_empty[ds]);
-        r2_release(kConsumerWarps / 4);
+        r2_release(kConsumerWarps / 8);  // the tile's eight warps stand for all sixteen
       } else {
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.d_empty[ds]);
