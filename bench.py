@@ -53,7 +53,7 @@ METRIC = "routed tokens/s (fused low-rank router + top-k)"
 # DRAM bytes (read + write) per token of the fused kernel, from the ncu capture summarised in
 # profiles/fused_route_kernel_prefill_r32_n65536.md (N = 65,536, scaled by tokens).  Only valid
 # while that kernel is unchanged; workloads without a capture report traffic null.
-NCU_TRAFFIC_PER_TOKEN = {"prefill_r32": (269.474048e6 + 11.228928e6) / 65536}
+NCU_TRAFFIC_PER_TOKEN = {"prefill_r32": (269.635072e6 + 8.524544e6) / 65536}
 L2_BYTES = 126 * 1024 * 1024
 
 
