@@ -476,7 +476,7 @@ __device__ __forceinline__ uint32_t r2_offset(int i, int e_local) {
 template <int R, int KCAP>
 __device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  constexpr int KL = C::KL, S = C::S;
+  constexpr int KL = C::KL;
   const RouteArgs& a = p.a;
   uint32_t cph = 0;  // parity of the consumer barrier
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
