@@ -15,6 +15,7 @@ import ctypes
 import os
 import subprocess
 from dataclasses import dataclass
+from typing import NamedTuple
 
 import numpy as np
 
@@ -54,6 +55,9 @@ def _bind(lib):
     lib.oracle_logits_at.restype = ctypes.c_int
     lib.oracle_logits_at.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, ctypes.c_int64, _P, _P, _P]
+    lib.oracle_train_stats.restype = ctypes.c_int
+    lib.oracle_train_stats.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _P, ctypes.c_int64, _P, _P, _P, ctypes.c_int]
     return lib
 
 
@@ -155,3 +159,27 @@ def logits_at(X, R1, R2, N: int, h: int, r: int, M: int, rows, experts) -> np.nd
     if rc != 0:
         raise ValueError("oracle_logits_at: invalid arguments")
     return out
+
+
+class TrainStats(NamedTuple):
+    m: np.ndarray     # (n,) largest logit of each token
+    Z: np.ndarray     # (n,) sum_j exp(l_j - m)
+    psum: np.ndarray  # (M,) sum over the tokens of the full-softmax probabilities
+
+
+def train_stats(X, R1, R2, N: int, h: int, r: int, M: int, rows=None, threads: int | None = None) -> TrainStats:
+    """m, Z and psum of tokens ``rows`` (default: all N): App. F, Algorithm 2, eqs. (6)-(7)."""
+    X = _u16(X, (N, h))
+    R1 = _u16(R1, (h, r))
+    R2 = _u16(R2, (r, M))
+    rows, n = _rows(rows, N)
+    m = np.empty(n)
+    Z = np.empty(n)
+    psum = np.empty(M)
+    rc = _load().oracle_train_stats(X.ctypes.data, R1.ctypes.data, R2.ctypes.data, N, h, r, M,
+                                    None if rows is None else rows.ctypes.data, n, m.ctypes.data,
+                                    Z.ctypes.data, psum.ctypes.data,
+                                    threads or max(1, min(64, os.cpu_count() or 1)))
+    if rc != 0:
+        raise ValueError("oracle_train_stats: invalid arguments")
+    return TrainStats(m, Z, psum)

@@ -14,6 +14,8 @@
  *           the strict comparison of the merge and the first-index argmax]
  *   gates = softmax over the k selected logits          [MoRE §2, App. F Fig. 12]
  *   counts[e] = number of (token, slot) pairs naming e  [MoRE App. F eq. (9), f]
+ *   training statistics m_n, Z_n and psum of App. F, Algorithm 2, eqs. (6)-(7)
+ *           (oracle_train_stats)
  * plus what the parity checks need: the margin l_(k) - l_(k+1) of Def. 1
  * [MoRE §3, Definition 1] (+inf when k = M), the gaps between consecutive
  * selected logits, and the root-mean-square of the token's M logits.
@@ -170,6 +172,84 @@ int oracle_route(const uint16_t* X, const uint16_t* R1, const uint16_t* R2, int6
   for (int t = 0; t < used; ++t) {
     if (!inline_run[t]) pthread_join(th[t], NULL);
     for (int e = 0; e < M; ++e) counts[e] += priv[(size_t)t * M + e];
+  }
+  free(priv);
+  return 0;
+}
+
+/*
+ * Training statistics of App. F, Algorithm 2 and eqs. (6)-(7), for the tokens rows[0 ..
+ * n_rows) (or 0 .. n_rows-1): per token the largest logit m_n = max_j l_nj and the
+ * softmax normalizer relative to it, Z_n = sum_j exp(l_nj - m_n) (Algorithm 2 keeps Z
+ * relative to the running maximum); per expert the column sum of the full softmax over
+ * all M experts, psum_i = sum_n exp(l_ni - m_n) / Z_n.  Plain fp64 loops; psum is summed
+ * per thread in token order and the thread partials are added in thread order.
+ * Returns 0, or 1 on bad arguments.
+ */
+typedef struct {
+  const uint16_t *X, *R1, *R2;
+  int h, r, M;
+  const int64_t* rows;
+  int64_t begin, end;
+  double *m, *Z;
+  double* psum; /* private per job, length M */
+} oracle_stats_job;
+
+static void* oracle_stats_worker(void* arg) {
+  oracle_stats_job* jb = (oracle_stats_job*)arg;
+  double* z = (double*)malloc(sizeof(double) * (size_t)jb->r);
+  double* l = (double*)malloc(sizeof(double) * (size_t)jb->M);
+  for (int64_t q = jb->begin; q < jb->end; ++q) {
+    int64_t n = jb->rows ? jb->rows[q] : q;
+    oracle_token_logits(jb->X + (size_t)n * jb->h, jb->R1, jb->R2, jb->h, jb->r, jb->M, z, l);
+    double mx = l[0];
+    for (int e = 1; e < jb->M; ++e)
+      if (l[e] > mx) mx = l[e];
+    double sum = 0.0;
+    for (int e = 0; e < jb->M; ++e) sum += exp(l[e] - mx);
+    jb->m[q] = mx;
+    jb->Z[q] = sum;
+    for (int e = 0; e < jb->M; ++e) jb->psum[e] += exp(l[e] - mx) / sum;
+  }
+  free(z);
+  free(l);
+  return NULL;
+}
+
+int oracle_train_stats(const uint16_t* X, const uint16_t* R1, const uint16_t* R2, int64_t N, int h,
+                       int r, int M, const int64_t* rows, int64_t n_rows, double* m, double* Z,
+                       double* psum, int nthreads) {
+  if (N < 0 || h < 1 || r < 1 || M < 1 || n_rows < 0) return 1;
+  if (!rows && n_rows > N) return 1;
+  if (rows)
+    for (int64_t q = 0; q < n_rows; ++q)
+      if (rows[q] < 0 || rows[q] >= N) return 1;
+  memset(psum, 0, sizeof(double) * (size_t)M);
+  if (n_rows == 0) return 0;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  if ((int64_t)nthreads > n_rows) nthreads = (int)n_rows;
+  pthread_t th[256];
+  int inline_run[256];
+  oracle_stats_job jobs[256];
+  double* priv = (double*)calloc((size_t)nthreads * (size_t)M, sizeof(double));
+  int64_t per = (n_rows + nthreads - 1) / nthreads;
+  int used = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    int64_t b = (int64_t)t * per, e = b + per;
+    if (e > n_rows) e = n_rows;
+    if (b >= e) break;
+    jobs[t] = (oracle_stats_job){X, R1, R2, h, r, M, rows, b, e, m, Z, priv + (size_t)t * M};
+    inline_run[t] = 0;
+    if (pthread_create(&th[t], NULL, oracle_stats_worker, &jobs[t]) != 0) {
+      oracle_stats_worker(&jobs[t]);
+      inline_run[t] = 1;
+    }
+    used = t + 1;
+  }
+  for (int t = 0; t < used; ++t) {
+    if (!inline_run[t]) pthread_join(th[t], NULL);
+    for (int e = 0; e < M; ++e) psum[e] += priv[(size_t)t * M + e];
   }
   free(priv);
   return 0;

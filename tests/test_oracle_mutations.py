@@ -34,6 +34,13 @@ MUTATIONS = {
                                "sel_logit[k - 1] - logits[scratch[k + 1 < M ? k + 1 : k].e]"),
     "counts_double_first": ("jb->counts[jb->idx[o + j]] += 1;", "jb->counts[jb->idx[o + j]] += (j == 0) ? 2 : 1;"),
     "rms_without_mean": ("*rms = sqrt(ss / (double)M);", "*rms = sqrt(ss);"),
+    "stats_max_skips_expert_0": ("double mx = l[0];\n    for (int e = 1; e < jb->M; ++e)",
+                                 "double mx = l[1];\n    for (int e = 2; e < jb->M; ++e)"),
+    "stats_Z_without_shift": ("for (int e = 0; e < jb->M; ++e) sum += exp(l[e] - mx);",
+                              "for (int e = 0; e < jb->M; ++e) sum += exp(l[e]);"),
+    "stats_psum_unnormalised": ("jb->psum[e] += exp(l[e] - mx) / sum;", "jb->psum[e] += exp(l[e] - mx);"),
+    "stats_psum_dropped_last_expert": ("for (int e = 0; e < jb->M; ++e) jb->psum[e] += exp(l[e] - mx) / sum;",
+                                       "for (int e = 0; e + 1 < jb->M; ++e) jb->psum[e] += exp(l[e] - mx) / sum;"),
 }
 
 PINS = [
@@ -49,6 +56,9 @@ PINS = [
     pins.test_counts_are_the_bincount_of_indices,
     pins.test_golden_jl_construction,
     pins.test_golden_hypercube_top1_is_sign_pattern,
+    pins.test_train_stats_closed_forms,
+    pins.test_train_stats_against_library_softmax,
+    pins.test_train_stats_shift_and_relabelling,
 ]
 
 

@@ -265,3 +265,63 @@ def test_oracle_rejects_invalid_arguments():
         oracle.route(X, R1, R2, 4, 8, 4, 6, 2, rows=[4])  # row out of range
     empty = oracle.route(X, R1, R2, 4, 8, 4, 6, 2, rows=np.zeros(0, np.int64))
     assert empty.idx.shape == (0, 2) and empty.counts.sum() == 0
+
+
+# --- training statistics (App. F, Algorithm 2, eqs. (6)-(7)) ----------------------------------
+
+def test_train_stats_closed_forms():
+    """Equal logits: m is that value, Z = M, every probability 1/M.  One logit 1 above
+    M - 1 zeros: Z = 1 + (M - 1) e^-1 and that expert's probability is 1 / Z."""
+    M, n = 16, 3
+    X, R1, R2 = identity_router(np.full((n, M), 2.0))
+    st = oracle.train_stats(X, R1, R2, n, M, M, M, threads=2)
+    np.testing.assert_array_equal(st.m, np.full(n, 2.0))
+    np.testing.assert_allclose(st.Z, np.full(n, float(M)), rtol=1e-15)
+    np.testing.assert_allclose(st.psum, np.full(M, n / M), rtol=1e-14)
+    vals = np.zeros((n, M))
+    vals[:, 5] = 1.0
+    X, R1, R2 = identity_router(vals)
+    st = oracle.train_stats(X, R1, R2, n, M, M, M, threads=2)
+    Z = 1.0 + (M - 1) * np.exp(-1.0)
+    np.testing.assert_array_equal(st.m, np.ones(n))
+    np.testing.assert_allclose(st.Z, np.full(n, Z), rtol=1e-14)
+    np.testing.assert_allclose(st.psum[5], n / Z, rtol=1e-14)
+    np.testing.assert_allclose(np.delete(st.psum, 5), n * np.exp(-1.0) / Z, rtol=1e-14)
+
+
+def test_train_stats_against_library_softmax():
+    """m, m + log Z and psum equal numpy's max, scipy's logsumexp and the column sum of
+    scipy's softmax, applied to the independently pinned logits."""
+    from scipy.special import logsumexp, softmax
+
+    N, h, r, M = 50, 96, 16, 80
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=11)
+    rows = np.array([0, 3, 17, 18, 49])
+    st = oracle.train_stats(X, R1, R2, N, h, r, M, rows=rows, threads=3)
+    lg = oracle.logits(X, R1, R2, N, h, r, M, rows=rows)
+    np.testing.assert_array_equal(st.m, lg.max(axis=1))
+    np.testing.assert_allclose(st.m + np.log(st.Z), logsumexp(lg, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(st.psum, softmax(lg, axis=1).sum(axis=0), rtol=1e-12, atol=1e-15)
+    assert abs(st.psum.sum() - rows.size) < 1e-12  # every softmax row sums to one
+
+
+def test_train_stats_shift_and_relabelling():
+    """A per-token constant added to all logits (an R2 row of equal entries times that
+    token's z) moves m only; permuting R2's columns permutes psum."""
+    N, h, r, M = 40, 64, 16, 48
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=12)
+    R2a = R2.copy()
+    R2a[0, :] = syn.f32_to_bf16_bits(np.zeros(M, np.float32))
+    R2b = R2.copy()
+    R2b[0, :] = syn.f32_to_bf16_bits(np.full(M, 0.75, np.float32))
+    a = oracle.train_stats(X, R1, R2a, N, h, r, M, threads=2)
+    b = oracle.train_stats(X, R1, R2b, N, h, r, M, threads=2)
+    z0 = oracle.projection(X, R1, N, h, r)[:, 0]
+    np.testing.assert_allclose(b.m - a.m, 0.75 * z0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(b.Z, a.Z, rtol=1e-12)
+    np.testing.assert_allclose(b.psum, a.psum, rtol=1e-11)
+    perm = np.random.default_rng(5).permutation(M)
+    c = oracle.train_stats(X, R1, np.ascontiguousarray(R2[:, perm]), N, h, r, M, threads=2)
+    d = oracle.train_stats(X, R1, R2, N, h, r, M, threads=2)
+    np.testing.assert_allclose(c.psum, d.psum[perm], rtol=1e-12)
+    np.testing.assert_array_equal(c.m, d.m)
