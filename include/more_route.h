@@ -149,6 +149,28 @@ more_status more_device_status(void* stream, uint32_t* detail);
 /* Static description of a status code. */
 const char* more_status_string(more_status status);
 
+/*
+ * Training forward of the router ("MoRE", App. F, Algorithm 2): everything more_route
+ * returns, plus the statistics a load-balancing loss needs, computed over all M experts
+ * (eqs. (6)-(8)):
+ *   out_m[n]    = max_j l_nj                         fp32 [N], the token's largest logit
+ *   out_Z[n]    = sum_j exp(l_nj - out_m[n])         fp32 [N], the softmax normalizer
+ *                                                    relative to out_m (as Algorithm 2 keeps it)
+ *   out_psum[i] = sum_n exp(l_ni - out_m[n]) / out_Z[n]
+ *                                                    fp32 [M], the column sum of the full
+ *                                                    softmax (eq. (7)); the call zeroes it first
+ * The Switch loss of eq. (9) is then M / N * sum_i f_i psum_i with f from out_expert_count.
+ * The logits are those of more_route (z carried as the bf16 pair z_hi + z_lo, fp32
+ * accumulation); the statistics use fp32 exp.  Requirements: as for more_route, plus
+ * out_psum non-NULL, out_m and out_Z non-NULL unless N == 0, all three 16-byte aligned,
+ * and M <= MORE_STATS_MMAX (else MORE_ERR_UNSUPPORTED).  Asynchronous on `stream`; runs
+ * the routing kernel and then one statistics kernel; allocates nothing.
+ */
+#define MORE_STATS_MMAX 32768
+more_status more_route_train(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                             int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
+                             float* out_logits, float* out_m, float* out_Z, float* out_psum, void* stream);
+
 /* MORE_ROUTE_ABI_VERSION of the built library. */
 int more_abi_version(void);
 

@@ -20,10 +20,11 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status", "Router", "MoreError",
-           "VARIANTS", "library_path", "abi_version", "KMAX"]
+__all__ = ["route", "route_train", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status",
+           "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
 KMAX = 16
+STATS_MMAX = 32768
 VARIANTS = {"auto": 0, "fused_tc": 1, "small_n": 2}
 STATUS = {0: "MORE_OK", 1: "MORE_ERR_INVALID_ARG", 2: "MORE_ERR_UNSUPPORTED", 3: "MORE_ERR_CUDA",
           4: "MORE_ERR_DEVICE"}
@@ -48,6 +49,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
     lib.more_route_unfused_static.restype = I
     lib.more_route_unfused_static.argtypes = route_args + [P]
+    lib.more_route_train.restype = I
+    lib.more_route_train.argtypes = route_args + [P, P, P, P]
     lib.more_route_unfused_scratch_bytes.restype = ctypes.c_size_t
     lib.more_route_unfused_scratch_bytes.argtypes = [I64, I, I]
     lib.more_device_status.restype = I
@@ -126,6 +129,35 @@ def route(X: torch.Tensor, R1: torch.Tensor, R2: torch.Tensor, k: int, *, out_id
                                  _ptr(outs[2]), _ptr(outs[3]), VARIANTS[variant], _stream_handle(stream))
     _check(st, "more_route")
     return outs
+
+
+def route_train(X: torch.Tensor, R1: torch.Tensor, R2: torch.Tensor, k: int, *, out_idx=None, out_gate=None,
+                out_expert_count=None, out_logits=None, out_m=None, out_Z=None, out_psum=None,
+                return_logits: bool = True, stream=None):
+    """:func:`route` plus the training statistics of the full softmax over all M experts.
+
+    Returns ``(idx, gate, expert_count, logits, m, Z, psum)``: ``m`` [N] the largest logit of
+    each token, ``Z`` [N] the sum of exp(logit - m) over all M experts, ``psum`` [M] the
+    column sum of the full softmax over the tokens (all fp32).
+    """
+    X, R1, R2 = _as_bf16(X, "X"), _as_bf16(R1, "R1"), _as_bf16(R2, "R2")
+    N, h = X.shape
+    h1, r = R1.shape
+    r1, M = R2.shape
+    if h1 != h or r1 != r:
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, R1 {tuple(R1.shape)}, R2 {tuple(R2.shape)}")
+    outs = _outputs(N, k, M, X.device, out_idx, out_gate, out_expert_count, out_logits, return_logits)
+    if out_m is None:
+        out_m = torch.empty((N,), dtype=torch.float32, device=X.device)
+    if out_Z is None:
+        out_Z = torch.empty((N,), dtype=torch.float32, device=X.device)
+    if out_psum is None:
+        out_psum = torch.empty((M,), dtype=torch.float32, device=X.device)
+    st = _lib.more_route_train(_ptr(X), _ptr(R1), _ptr(R2), N, h, r, M, k, _ptr(outs[0]), _ptr(outs[1]),
+                               _ptr(outs[2]), _ptr(outs[3]), _ptr(out_m), _ptr(out_Z), _ptr(out_psum),
+                               _stream_handle(stream))
+    _check(st, "more_route_train")
+    return (*outs, out_m, out_Z, out_psum)
 
 
 def unfused_scratch_bytes(N: int, r: int, M: int) -> int:

@@ -125,6 +125,24 @@ more_status more_route(const void* X, const void* R1, const void* R2, int64_t N,
                             MORE_VARIANT_AUTO, stream);
 }
 
+more_status more_route_train(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                             int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
+                             float* out_logits, float* out_m, float* out_Z, float* out_psum, void* stream) {
+  more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  if (st != MORE_OK) return st;
+  if (!out_psum || !aligned16(out_psum) || (N > 0 && (!out_m || !out_Z)) || (out_m && !aligned16(out_m)) ||
+      (out_Z && !aligned16(out_Z)))
+    return MORE_ERR_INVALID_ARG;
+  if (M > MORE_STATS_MMAX) return MORE_ERR_UNSUPPORTED;
+  st = more_route_variant(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
+                          MORE_VARIANT_AUTO, stream);
+  if (st != MORE_OK) return st;
+  RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
+                          stream);
+  if (cudaMemsetAsync(out_psum, 0, sizeof(float) * (size_t)M, a.stream) != cudaSuccess) return MORE_ERR_CUDA;
+  return launch_train_stats(a, out_m, out_Z, out_psum) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
 size_t more_route_unfused_scratch_bytes(int64_t N, int r, int M) {
   if (N < 0 || r < 1 || M < 1) return 0;
   return unfused_scratch_bytes(N, r, M);

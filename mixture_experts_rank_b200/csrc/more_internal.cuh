@@ -25,6 +25,7 @@ struct RouteArgs {
 
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_small_n(const RouteArgs& a);
+cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, float* out_psum);
 cudaError_t launch_fused_tc(const RouteArgs& a);
 bool fused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused(const RouteArgs& a, void* scratch);

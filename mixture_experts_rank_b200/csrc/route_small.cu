@@ -92,6 +92,31 @@ __device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict
   index = b + ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
+// Logits of this lane's 8 experts e0 .. e0 + 7 (one 16-byte load per R2 row, batches of
+// 8 rows); zs holds z_i as the bf16 pair sum.  ok is false for a lane past the last expert.
+__device__ __forceinline__ void lane_logits8(const RouteArgs& a, const float* zs, int e0, bool ok, float* acc) {
+  const uint4* src = reinterpret_cast<const uint4*>(a.R2) + (ok ? (e0 >> 3) : 0);
+  const size_t rowv = (size_t)(a.M >> 3);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+  for (int i0 = 0; i0 < a.r; i0 += 8) {
+    uint4 w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = ok ? __ldg(src + (size_t)(i0 + j) * rowv) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float zi = zs[i0 + j];
+      const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(wp[q]);
+        acc[2 * q] = fmaf(zi, f.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(zi, f.y, acc[2 * q + 1]);
+      }
+    }
+  }
+}
+
 template <int K>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     small_n_route_kernel(RouteArgs a) {
@@ -120,31 +145,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     // 2. this warp's 256-expert blocks
     TopList<K> list;
     list.init();
-    const size_t rowv = (size_t)(a.M >> 3);  // 16-byte groups per R2 row
     for (int eb = 256 * warp; eb < a.M; eb += 256 * kWarpsPerBlock) {
       const int e0 = eb + 8 * lane;
       const bool ok = e0 < a.M;  // M is a multiple of 8: the lane's 8 experts are all in range
-      const uint4* src = reinterpret_cast<const uint4*>(a.R2) + (ok ? (e0 >> 3) : 0);
       float acc[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-      // batches of 8 R2 rows (r is a multiple of 16): loads first, then the arithmetic
-      for (int i0 = 0; i0 < a.r; i0 += 8) {
-        uint4 w[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) w[j] = ok ? __ldg(src + (size_t)(i0 + j) * rowv) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float zi = zs[i0 + j];
-          const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __bfloat1622float2(wp[q]);
-            acc[2 * q] = fmaf(zi, f.x, acc[2 * q]);
-            acc[2 * q + 1] = fmaf(zi, f.y, acc[2 * q + 1]);
-          }
-        }
-      }
+      lane_logits8(a, zs, e0, ok, acc);
       if (ok) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) list.insert(acc[q], e0 + q);
@@ -171,6 +176,100 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   }
 }
 
+// Merge of two (running maximum, sum of exp(l - maximum)) pairs, App. F eq. (8).
+__device__ __forceinline__ void merge_max_sum(float& m, float& s, float om, float os) {
+  const float nm = fmaxf(m, om);
+  if (nm == -INFINITY) return;  // both empty
+  s = (m == -INFINITY ? 0.f : s * expf(m - nm)) + (om == -INFINITY ? 0.f : os * expf(om - nm));
+  m = nm;
+}
+
+// Training statistics of App. F, Algorithm 2 (eqs. (6)-(8)): one CTA of 16 warps per
+// token (grid-stride over tokens).  z as in small_n_route_kernel; sweep 1 keeps, per
+// lane, the running maximum m and the rescaled sum Z over its experts (eq. (8)) and
+// merges lanes, then warps; sweep 2 recomputes the same logits and adds
+// exp(l - m) / Z into the CTA's column sums in shared memory.  Each expert belongs to one
+// lane of one warp, so the shared sums need no atomics; at the end each CTA adds its sums
+// to psum with one global atomic per expert.
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    train_stats_kernel(RouteArgs a, float* __restrict__ out_m, float* __restrict__ out_Z,
+                       float* __restrict__ out_psum) {
+  extern __shared__ float psum_s[];  // M column sums of this CTA
+  __shared__ float zpart[kWarpsPerBlock][kRMax];
+  __shared__ float zs[kRMax];
+  __shared__ float wm[kWarpsPerBlock], wz[kWarpsPerBlock];
+  __shared__ float tok_m, tok_z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < a.M; e += blockDim.x) psum_s[e] = 0.f;
+  for (int64_t n = blockIdx.x; n < a.N; n += gridDim.x) {
+    const __nv_bfloat16* x = a.X + (size_t)n * a.h;
+    for (int b = 0; b < a.r; b += 16) {
+      float v;
+      int i;
+      warp_partial_z16(x, a.R1, a.h, a.r, b, warp, lane, v, i);
+      if ((lane & 1) == 0) zpart[warp][i] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < a.r) {
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w) z += zpart[w][threadIdx.x];
+      zs[threadIdx.x] = split_bf16_pair(z);
+    }
+    __syncthreads();
+    // sweep 1: running maximum and rescaled sum
+    float lm = -INFINITY, ls = 0.f;
+    for (int eb = 256 * warp; eb < a.M; eb += 256 * kWarpsPerBlock) {
+      const int e0 = eb + 8 * lane;
+      const bool ok = e0 < a.M;  // M is a multiple of 8: the lane's 8 experts are all in range
+      float acc[8];
+      lane_logits8(a, zs, e0, ok, acc);
+      if (ok) {
+        float bm = acc[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) bm = fmaxf(bm, acc[q]);
+        float bs = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) bs += expf(acc[q] - bm);
+        merge_max_sum(lm, ls, bm, bs);
+      }
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, lm, d), os = __shfl_xor_sync(0xffffffffu, ls, d);
+      merge_max_sum(lm, ls, om, os);
+    }
+    if (lane == 0) {
+      wm[warp] = lm;
+      wz[warp] = ls;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m = -INFINITY, s = 0.f;
+      for (int w = 0; w < kWarpsPerBlock; ++w) merge_max_sum(m, s, wm[w], wz[w]);
+      tok_m = m;
+      tok_z = s;
+      out_m[n] = m;
+      out_Z[n] = s;
+    }
+    __syncthreads();
+    // sweep 2: this token's softmax probabilities into the column sums
+    const float m = tok_m, inv_z = 1.f / tok_z;
+    for (int eb = 256 * warp; eb < a.M; eb += 256 * kWarpsPerBlock) {
+      const int e0 = eb + 8 * lane;
+      const bool ok = e0 < a.M;
+      float acc[8];
+      lane_logits8(a, zs, e0, ok, acc);
+      if (ok) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) psum_s[e0 + q] += expf(acc[q] - m) * inv_z;
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.M; e += blockDim.x) atomicAdd(out_psum + e, psum_s[e]);
+}
+
 template <int K>
 cudaError_t launch_k(const RouteArgs& a) {
   int dev = 0, sms = 148;
@@ -184,6 +283,26 @@ cudaError_t launch_k(const RouteArgs& a) {
 }
 
 }  // namespace
+
+cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, float* out_psum) {
+  if (a.N == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t smem = sizeof(float) * (size_t)a.M;
+  static int configured[64] = {};
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(train_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(float) * MORE_STATS_MMAX));
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  int64_t blocks = a.N;  // tokens are independent; a CTA keeps its column sums over its tokens
+  const int64_t cap = (int64_t)sms * 2;
+  if (blocks > cap) blocks = cap;
+  train_stats_kernel<<<(unsigned)blocks, kWarpsPerBlock * 32, smem, a.stream>>>(a, out_m, out_Z, out_psum);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_small_n(const RouteArgs& a) {
   if (a.N == 0) return cudaSuccess;

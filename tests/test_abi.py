@@ -28,7 +28,7 @@ def lib():
 
 def test_header_declares_the_route_entry_points():
     names = declared_functions()
-    for required in ("more_route", "more_route_variant", "more_route_unfused",
+    for required in ("more_route", "more_route_variant", "more_route_train", "more_route_unfused",
                      "more_route_unfused_scratch_bytes", "more_device_status", "more_status_string",
                      "more_abi_version"):
         assert required in names
@@ -74,6 +74,20 @@ def test_unfused_scratch_size_and_checks(lib):
     st = lib.more_route_unfused(P(16), P(16), P(16), 1000, 64, 32, 256, 4, P(16), P(16), P(16), None, P(16),
                                 n - 1, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("kwargs,expected", [
+    (dict(psum=0), 1), (dict(m=0), 1), (dict(Z=0), 1), (dict(psum=8), 1), (dict(m=40), 1),
+    (dict(k=0), 1), (dict(M=32776), 2),
+])
+def test_train_entry_rejects_invalid_arguments(lib, kwargs, expected):
+    P = ctypes.c_void_p
+    args = dict(N=16, h=64, r=32, M=64, k=4, m=16, Z=16, psum=16)
+    args.update(kwargs)
+    opt = lambda v: P(v) if v else None
+    st = lib.more_route_train(P(16), P(16), P(16), args["N"], args["h"], args["r"], args["M"], args["k"], P(16),
+                              P(16), P(16), None, opt(args["m"]), opt(args["Z"]), opt(args["psum"]), None)
+    assert st == expected
 
 
 def test_package_refuses_to_run_without_the_library(monkeypatch, tmp_path):
