@@ -25,18 +25,18 @@ namespace {
 constexpr int kWarpsPerBlock = 16;
 constexpr int kRMax = 128;
 
-// The 16 sums z[b .. b + 16) over this warp's hidden rows (w*32 + lane + 512 j), reduced
-// across the warp by a reduce-scatter: afterwards every value sits on two neighbouring
-// lanes; `value` is this lane's value and `index` its z index.
-__device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict__ x,
-                                                 const __nv_bfloat16* __restrict__ R1, int h, int r, int b,
-                                                 int warp, int lane, float& value, int& index) {
+// The 16 sums z[b .. b + 16) over this warp's hidden rows tstart + kStride j (tstart holds
+// the lane), reduced across the warp by a reduce-scatter: afterwards every value sits on
+// two neighbouring lanes; `value` is this lane's value and `index` its z index.
+__device__ __forceinline__ void warp_partial_z16_strided(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ R1, int h, int r,
+                                                         int b, int tstart, int kStride, int lane, float& value,
+                                                         int& index) {
   float acc[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-  constexpr int kStride = kWarpsPerBlock * 32;
   // batches of 4 hidden rows: all loads first, then the arithmetic, so the loads overlap
-  for (int t0 = warp * 32 + lane; t0 < h; t0 += 4 * kStride) {
+  for (int t0 = tstart; t0 < h; t0 += 4 * kStride) {
     float xt[4];
     uint4 w0[4], w1[4];
 #pragma unroll
@@ -90,6 +90,13 @@ __device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict
   acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
   value = acc[0];
   index = b + ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
+
+// The same with warp w taking hidden rows w*32 + lane + 512 j (all 16 warps on one token).
+__device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict__ x,
+                                                 const __nv_bfloat16* __restrict__ R1, int h, int r, int b,
+                                                 int warp, int lane, float& value, int& index) {
+  warp_partial_z16_strided(x, R1, h, r, b, warp * 32 + lane, kWarpsPerBlock * 32, lane, value, index);
 }
 
 // Logits of this lane's 8 experts e0 .. e0 + 7 (one 16-byte load per R2 row, batches of
@@ -184,87 +191,154 @@ __device__ __forceinline__ void merge_max_sum(float& m, float& s, float om, floa
   m = nm;
 }
 
-// Training statistics of App. F, Algorithm 2 (eqs. (6)-(8)): one CTA of 16 warps per
-// token (grid-stride over tokens).  z as in small_n_route_kernel; sweep 1 keeps, per
-// lane, the running maximum m and the rescaled sum Z over its experts (eq. (8)) and
-// merges lanes, then warps; sweep 2 recomputes the same logits and adds
-// exp(l - m) / Z into the CTA's column sums in shared memory.  Each expert belongs to one
-// lane of one warp, so the shared sums need no atomics; at the end each CTA adds its sums
-// to psum with one global atomic per expert.
+constexpr int kStatTokens = 4;  // tokens per iteration of the statistics kernel
+
+// Logits of this lane's 8 experts e0 .. e0 + 7 for kStatTokens tokens at once (one
+// 16-byte load per R2 row, shared by the tokens); zs[j][i] holds token j's z_i.
+__device__ __forceinline__ void lane_logits8_tokens(const RouteArgs& a, const float (*zs)[kRMax], int e0, bool ok,
+                                                    float (&acc)[kStatTokens][8]) {
+  const uint4* src = reinterpret_cast<const uint4*>(a.R2) + (ok ? (e0 >> 3) : 0);
+  const size_t rowv = (size_t)(a.M >> 3);
+#pragma unroll
+  for (int j = 0; j < kStatTokens; ++j)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[j][q] = 0.f;
+  for (int i0 = 0; i0 < a.r; i0 += 8) {
+    uint4 w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) w[u] = ok ? __ldg(src + (size_t)(i0 + u) * rowv) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w[u]);
+      float f[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 t = __bfloat1622float2(wp[q]);
+        f[2 * q] = t.x;
+        f[2 * q + 1] = t.y;
+      }
+#pragma unroll
+      for (int j = 0; j < kStatTokens; ++j) {
+        const float zi = zs[j][i0 + u];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[j][q] = fmaf(zi, f[q], acc[j][q]);
+      }
+    }
+  }
+}
+
+// Training statistics of App. F, Algorithm 2 (eqs. (6)-(8)).  A CTA of 16 warps takes
+// kStatTokens tokens per iteration (grid-stride): warps 4 j .. 4 j + 3 project token j
+// (each a quarter of the hidden rows); then every warp takes its 256-expert blocks for all
+// the tokens at once, so each R2 row load serves every token.  Sweep 1 keeps, per lane and
+// token, the running maximum m and the rescaled sum Z (eq. (8)) and merges lanes, then
+// warps; sweep 2 recomputes the same logits and adds exp(l - m) / Z into the CTA's column
+// sums in shared memory.  Each expert belongs to one lane of one warp, so the shared sums
+// need no atomics; at the end each CTA adds its sums to psum, one atomic per expert.
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     train_stats_kernel(RouteArgs a, float* __restrict__ out_m, float* __restrict__ out_Z,
                        float* __restrict__ out_psum) {
+  static_assert(kWarpsPerBlock == 4 * kStatTokens, "four warps project each token");
   extern __shared__ float psum_s[];  // M column sums of this CTA
   __shared__ float zpart[kWarpsPerBlock][kRMax];
-  __shared__ float zs[kRMax];
-  __shared__ float wm[kWarpsPerBlock], wz[kWarpsPerBlock];
-  __shared__ float tok_m, tok_z;
+  __shared__ float zs[kStatTokens][kRMax];
+  __shared__ float wm[kWarpsPerBlock][kStatTokens], wz[kWarpsPerBlock][kStatTokens];
+  __shared__ float tok_m[kStatTokens], tok_z[kStatTokens];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < a.M; e += blockDim.x) psum_s[e] = 0.f;
-  for (int64_t n = blockIdx.x; n < a.N; n += gridDim.x) {
-    const __nv_bfloat16* x = a.X + (size_t)n * a.h;
-    for (int b = 0; b < a.r; b += 16) {
-      float v;
-      int i;
-      warp_partial_z16(x, a.R1, a.h, a.r, b, warp, lane, v, i);
-      if ((lane & 1) == 0) zpart[warp][i] = v;
+  for (int64_t n0 = (int64_t)blockIdx.x * kStatTokens; n0 < a.N; n0 += (int64_t)gridDim.x * kStatTokens) {
+    const int nt = a.N - n0 < kStatTokens ? (int)(a.N - n0) : kStatTokens;
+    // z of token j = warp / 4 (a token past the batch end projects token n0 instead; it is not used)
+    {
+      const int j = warp >> 2;
+      const __nv_bfloat16* x = a.X + (size_t)(n0 + (j < nt ? j : 0)) * a.h;
+      for (int b = 0; b < a.r; b += 16) {
+        float v;
+        int i;
+        warp_partial_z16_strided(x, a.R1, a.h, a.r, b, (warp & 3) * 32 + lane, 128, lane, v, i);
+        if ((lane & 1) == 0) zpart[warp][i] = v;
+      }
     }
     __syncthreads();
-    if (threadIdx.x < a.r) {
-      float z = 0.f;
+    for (int q = threadIdx.x; q < kStatTokens * a.r; q += blockDim.x) {
+      const int j = q / a.r, i = q - j * a.r;
+      zs[j][i] = split_bf16_pair(zpart[4 * j][i] + zpart[4 * j + 1][i] + zpart[4 * j + 2][i] + zpart[4 * j + 3][i]);
+    }
+    __syncthreads();
+    // sweep 1: running maximum and rescaled sum per token
+    float lm[kStatTokens], ls[kStatTokens];
 #pragma unroll
-      for (int w = 0; w < kWarpsPerBlock; ++w) z += zpart[w][threadIdx.x];
-      zs[threadIdx.x] = split_bf16_pair(z);
+    for (int j = 0; j < kStatTokens; ++j) {
+      lm[j] = -INFINITY;
+      ls[j] = 0.f;
     }
-    __syncthreads();
-    // sweep 1: running maximum and rescaled sum
-    float lm = -INFINITY, ls = 0.f;
     for (int eb = 256 * warp; eb < a.M; eb += 256 * kWarpsPerBlock) {
       const int e0 = eb + 8 * lane;
       const bool ok = e0 < a.M;  // M is a multiple of 8: the lane's 8 experts are all in range
-      float acc[8];
-      lane_logits8(a, zs, e0, ok, acc);
+      float acc[kStatTokens][8];
+      lane_logits8_tokens(a, zs, e0, ok, acc);
       if (ok) {
-        float bm = acc[0];
 #pragma unroll
-        for (int q = 1; q < 8; ++q) bm = fmaxf(bm, acc[q]);
-        float bs = 0.f;
+        for (int j = 0; j < kStatTokens; ++j) {
+          float bm = acc[j][0];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) bs += expf(acc[q] - bm);
-        merge_max_sum(lm, ls, bm, bs);
+          for (int q = 1; q < 8; ++q) bm = fmaxf(bm, acc[j][q]);
+          float bs = 0.f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) bs += expf(acc[j][q] - bm);
+          merge_max_sum(lm[j], ls[j], bm, bs);
+        }
       }
     }
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) {
-      const float om = __shfl_xor_sync(0xffffffffu, lm, d), os = __shfl_xor_sync(0xffffffffu, ls, d);
-      merge_max_sum(lm, ls, om, os);
-    }
-    if (lane == 0) {
-      wm[warp] = lm;
-      wz[warp] = ls;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float m = -INFINITY, s = 0.f;
-      for (int w = 0; w < kWarpsPerBlock; ++w) merge_max_sum(m, s, wm[w], wz[w]);
-      tok_m = m;
-      tok_z = s;
-      out_m[n] = m;
-      out_Z[n] = s;
+    for (int j = 0; j < kStatTokens; ++j) {
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) {
+        const float om = __shfl_xor_sync(0xffffffffu, lm[j], d), os = __shfl_xor_sync(0xffffffffu, ls[j], d);
+        merge_max_sum(lm[j], ls[j], om, os);
+      }
+      if (lane == 0) {
+        wm[warp][j] = lm[j];
+        wz[warp][j] = ls[j];
+      }
     }
     __syncthreads();
-    // sweep 2: this token's softmax probabilities into the column sums
-    const float m = tok_m, inv_z = 1.f / tok_z;
+    if (threadIdx.x < kStatTokens) {
+      const int j = threadIdx.x;
+      float m = -INFINITY, sz = 0.f;
+      for (int w = 0; w < kWarpsPerBlock; ++w) merge_max_sum(m, sz, wm[w][j], wz[w][j]);
+      tok_m[j] = m;
+      tok_z[j] = sz;
+      if (j < nt) {
+        out_m[n0 + j] = m;
+        out_Z[n0 + j] = sz;
+      }
+    }
+    __syncthreads();
+    // sweep 2: the tokens' softmax probabilities into the column sums
+    float m[kStatTokens], inv_z[kStatTokens];
+#pragma unroll
+    for (int j = 0; j < kStatTokens; ++j) {
+      m[j] = tok_m[j];
+      inv_z[j] = 1.f / tok_z[j];
+    }
     for (int eb = 256 * warp; eb < a.M; eb += 256 * kWarpsPerBlock) {
       const int e0 = eb + 8 * lane;
       const bool ok = e0 < a.M;
-      float acc[8];
-      lane_logits8(a, zs, e0, ok, acc);
+      float acc[kStatTokens][8];
+      lane_logits8_tokens(a, zs, e0, ok, acc);
       if (ok) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) psum_s[e0 + q] += expf(acc[q] - m) * inv_z;
+        for (int q = 0; q < 8; ++q) {
+          float add = 0.f;
+#pragma unroll
+          for (int j = 0; j < kStatTokens; ++j)
+            if (j < nt) add += expf(acc[j][q] - m[j]) * inv_z[j];
+          psum_s[e0 + q] += add;
+        }
       }
     }
+    __syncthreads();  // zs and tok_m/tok_z are rewritten by the next iteration
   }
   __syncthreads();
   for (int e = threadIdx.x; e < a.M; e += blockDim.x) atomicAdd(out_psum + e, psum_s[e]);
@@ -297,8 +371,9 @@ cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, f
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  int64_t blocks = a.N;  // tokens are independent; a CTA keeps its column sums over its tokens
-  const int64_t cap = (int64_t)sms * 2;
+  // tokens are independent; a CTA keeps its column sums over its tokens (one CTA per SM fits)
+  int64_t blocks = (a.N + kStatTokens - 1) / kStatTokens;
+  const int64_t cap = (int64_t)sms;
   if (blocks > cap) blocks = cap;
   train_stats_kernel<<<(unsigned)blocks, kWarpsPerBlock * 32, smem, a.stream>>>(a, out_m, out_Z, out_psum);
   return cudaGetLastError();
