@@ -183,3 +183,22 @@ def train_stats(X, R1, R2, N: int, h: int, r: int, M: int, rows=None, threads: i
     if rc != 0:
         raise ValueError("oracle_train_stats: invalid arguments")
     return TrainStats(m, Z, psum)
+
+
+class Dispatch(NamedTuple):
+    offsets: np.ndarray  # (M + 1,) int64: expert e owns sorted[offsets[e]:offsets[e + 1]]
+    sorted: np.ndarray   # (N k,) int64: flat slot ids n k + j, grouped by expert, in slot order
+
+
+def dispatch(idx, M: int) -> Dispatch:
+    """Dispatch bookkeeping after routing ("MoRE", App. E, Fig. 9, "Sort + Count"): the
+    (N, k) expert indices flattened to N k slots, stably sorted by expert, and the
+    per-expert offsets (exclusive prefix sum of the counts, M + 1 entries).  A library
+    stable sort and cumulative sum are the steps; nothing else is done to them."""
+    flat = np.ascontiguousarray(idx, dtype=np.int64).ravel()
+    if flat.size and (flat.min() < 0 or flat.max() >= M):
+        raise ValueError("expert index outside [0, M)")
+    order = np.argsort(flat, kind="stable")
+    counts = np.bincount(flat, minlength=M)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    return Dispatch(offsets, order.astype(np.int64))

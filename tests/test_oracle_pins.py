@@ -325,3 +325,43 @@ def test_train_stats_shift_and_relabelling():
     d = oracle.train_stats(X, R1, R2, N, h, r, M, threads=2)
     np.testing.assert_allclose(c.psum, d.psum[perm], rtol=1e-12)
     np.testing.assert_array_equal(c.m, d.m)
+
+
+# --- dispatch bookkeeping (App. E, Fig. 9 "Sort + Count") -------------------------------------
+
+def brute_force_dispatch(idx, M):
+    """Expert by expert, the slots naming it in increasing slot order."""
+    flat = [int(v) for v in np.asarray(idx).ravel()]
+    sorted_slots, offsets = [], [0]
+    for e in range(M):
+        sorted_slots += [s for s, v in enumerate(flat) if v == e]
+        offsets.append(len(sorted_slots))
+    return np.array(offsets), np.array(sorted_slots, dtype=np.int64)
+
+
+@pytest.mark.parametrize("N,k,M", [(1, 1, 8), (7, 3, 8), (50, 4, 16), (33, 8, 64)])
+def test_dispatch_matches_brute_force(N, k, M):
+    rng = np.random.default_rng(N * 100 + k)
+    idx = rng.integers(0, M, size=(N, k))
+    d = oracle.dispatch(idx, M)
+    off, srt = brute_force_dispatch(idx, M)
+    np.testing.assert_array_equal(d.offsets, off)
+    np.testing.assert_array_equal(d.sorted, srt)
+
+
+def test_dispatch_invariants_on_routing_output():
+    """On real routing output: a permutation of the slots, grouped by expert, increasing
+    within each expert, with offsets equal to the cumulative routing counts."""
+    N, h, r, M, k = 200, 64, 16, 48, 6
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=21)
+    o = oracle.route(X, R1, R2, N, h, r, M, k, threads=2)
+    d = oracle.dispatch(o.idx, M)
+    assert np.array_equal(np.sort(d.sorted), np.arange(N * k))
+    flat = o.idx.ravel()
+    np.testing.assert_array_equal(np.diff(d.offsets), o.counts)
+    for e in range(M):
+        seg = d.sorted[d.offsets[e]:d.offsets[e + 1]]
+        assert np.all(flat[seg] == e)
+        assert np.all(np.diff(seg) > 0)
+    with pytest.raises(ValueError):
+        oracle.dispatch(np.array([[0, M]]), M)
