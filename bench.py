@@ -203,8 +203,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="auto", choices=["auto", "fused_tc", "small_n", "unfused", "train"],
-                    help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum)")
+    ap.add_argument("--variant", default="auto", choices=["auto", "fused_tc", "small_n", "unfused", "train", "dispatch"],
+                    help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum); "
+                         "dispatch: routing followed by more_dispatch of its indices")
     ap.add_argument("--workload", default="prefill_r32", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample size, in CPU seconds")
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
@@ -254,6 +255,10 @@ def main():
         m_buf = torch.empty((N,), dtype=torch.float32, device="cuda")
         z_buf = torch.empty((N,), dtype=torch.float32, device="cuda")
         psum_buf = torch.empty((M,), dtype=torch.float32, device="cuda")
+    if args.variant == "dispatch":
+        d_scratch = torch.empty(max(more.dispatch_scratch_bytes(N, k, M), 16), dtype=torch.uint8, device="cuda")
+        d_off = torch.empty((M + 1,), dtype=torch.int32, device="cuda")
+        d_sorted = torch.empty((N * k,), dtype=torch.int32, device="cuda")
     if args.variant == "unfused":
         scratch = torch.empty(more.unfused_scratch_bytes(N, r, M), dtype=torch.uint8, device="cuda")
 
@@ -262,6 +267,9 @@ def main():
         if args.variant == "train":
             more.route_train(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
                              out_m=m_buf, out_Z=z_buf, out_psum=psum_buf, stream=st)
+        elif args.variant == "dispatch":
+            more.route(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits, stream=st)
+            more.dispatch(idx, M, scratch=d_scratch, out_offsets=d_off, out_sorted=d_sorted, stream=st)
         elif args.variant == "unfused":
             more.route_unfused(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate, out_expert_count=cnt,
                                out_logits=logits, stream=st)
@@ -277,7 +285,7 @@ def main():
         except more.MoreError:
             variant_used = "small_n"
         variant_used = variant_used if N >= 512 else "small_n"
-    launches_per_step = 3 if args.variant == "unfused" else (2 if args.variant == "train" else 1)
+    launches_per_step = {"unfused": 3, "train": 2, "dispatch": 5}.get(args.variant, 1)
 
     def barrier():
         if dist is not None:

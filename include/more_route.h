@@ -144,6 +144,7 @@ more_status more_route_unfused_static(const void* X, const void* R1, const void*
  */
 #define MORE_DEVERR_WAIT_TIMEOUT 0x1u  /* a bounded barrier wait ran out            */
 #define MORE_DEVERR_BAD_CONFIG 0x2u    /* a kernel saw a configuration it rejects  */
+#define MORE_DEVERR_BAD_INPUT 0x4u     /* an input value outside its range (skipped) */
 more_status more_device_status(void* stream, uint32_t* detail);
 
 /* Static description of a status code. */
@@ -170,6 +171,26 @@ const char* more_status_string(more_status status);
 more_status more_route_train(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
                              int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
                              float* out_logits, float* out_m, float* out_Z, float* out_psum, void* stream);
+
+/*
+ * Dispatch bookkeeping after routing ("MoRE", App. E, Fig. 9, "Sort + Count"): the
+ * (N, k) expert indices flattened to N*k slots s = n*k + j, stably sorted by expert, and
+ * the per-expert offsets:
+ *   out_offsets[e] = number of slots naming an expert below e     int32 [M + 1]
+ *                    (out_offsets[M] = N*k)
+ *   out_sorted[out_offsets[e] .. out_offsets[e + 1])               int32 [N*k]
+ *                  = the slots naming expert e, in increasing order
+ * idx: int32 [N][k] device, values in [0, M) (as more_route writes them; a value outside
+ * is skipped and sets MORE_DEVERR_BAD_INPUT, and the offsets then count only valid slots).
+ * scratch: device, 16-byte aligned, at least more_dispatch_scratch_bytes(N, k, M) bytes
+ * (per-chunk histograms).  Requirements: N >= 0, 1 <= k <= MORE_KMAX, 1 <= M <= MORE_MMAX,
+ * N*k < 2^31, out_offsets non-NULL, idx / out_sorted / scratch non-NULL unless N == 0, all
+ * 16-byte aligned.  Asynchronous on `stream` (four kernels and a memset); allocates nothing.
+ * The result does not depend on the launch configuration (a deterministic counting sort).
+ */
+size_t more_dispatch_scratch_bytes(int64_t N, int k, int M);
+more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
+                          int32_t* out_sorted, void* scratch, size_t scratch_bytes, void* stream);
 
 /* MORE_ROUTE_ABI_VERSION of the built library. */
 int more_abi_version(void);

@@ -20,7 +20,7 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "route_train", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status",
+__all__ = ["route", "route_train", "dispatch", "dispatch_scratch_bytes", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status",
            "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
 KMAX = 16
@@ -49,6 +49,10 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
     lib.more_route_unfused_static.restype = I
     lib.more_route_unfused_static.argtypes = route_args + [P]
+    lib.more_dispatch_scratch_bytes.restype = ctypes.c_size_t
+    lib.more_dispatch_scratch_bytes.argtypes = [I64, I, I]
+    lib.more_dispatch.restype = I
+    lib.more_dispatch.argtypes = [P, I64, I, I, P, P, P, ctypes.c_size_t, P]
     lib.more_route_train.restype = I
     lib.more_route_train.argtypes = route_args + [P, P, P, P]
     lib.more_route_unfused_scratch_bytes.restype = ctypes.c_size_t
@@ -158,6 +162,30 @@ def route_train(X: torch.Tensor, R1: torch.Tensor, R2: torch.Tensor, k: int, *, 
                                _stream_handle(stream))
     _check(st, "more_route_train")
     return (*outs, out_m, out_Z, out_psum)
+
+
+def dispatch_scratch_bytes(N: int, k: int, M: int) -> int:
+    return int(_lib.more_dispatch_scratch_bytes(N, k, M))
+
+
+def dispatch(idx: torch.Tensor, M: int, *, scratch: torch.Tensor | None = None, out_offsets=None,
+             out_sorted=None, stream=None):
+    """Dispatch bookkeeping for routing indices ``idx`` (int32 [N, k], CUDA): returns
+    ``(offsets int32 [M + 1], sorted int32 [N k])``; expert e owns ``sorted[offsets[e]:offsets[e+1]]``,
+    the flat slots n k + j naming it, in increasing order."""
+    if idx.dtype != torch.int32 or not idx.is_cuda or not idx.is_contiguous() or idx.dim() != 2:
+        raise ValueError("idx must be a contiguous int32 CUDA tensor of shape [N, k]")
+    N, k = idx.shape
+    if scratch is None:
+        scratch = torch.empty(max(dispatch_scratch_bytes(N, k, M), 16), dtype=torch.uint8, device=idx.device)
+    if out_offsets is None:
+        out_offsets = torch.empty((M + 1,), dtype=torch.int32, device=idx.device)
+    if out_sorted is None:
+        out_sorted = torch.empty((N * k,), dtype=torch.int32, device=idx.device)
+    st = _lib.more_dispatch(_ptr(idx), N, k, M, _ptr(out_offsets), _ptr(out_sorted), _ptr(scratch),
+                            scratch.numel(), _stream_handle(stream))
+    _check(st, "more_dispatch")
+    return out_offsets, out_sorted
 
 
 def unfused_scratch_bytes(N: int, r: int, M: int) -> int:

@@ -143,6 +143,27 @@ more_status more_route_train(const void* X, const void* R1, const void* R2, int6
   return launch_train_stats(a, out_m, out_Z, out_psum) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
 }
 
+size_t more_dispatch_scratch_bytes(int64_t N, int k, int M) {
+  if (N < 0 || k < 1 || M < 1 || M > MORE_MMAX || N * (int64_t)k > 0x7fffffffLL) return 0;
+  return (size_t)dispatch_scratch_bytes(N * (int64_t)k, M);
+}
+
+more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
+                          int32_t* out_sorted, void* scratch, size_t scratch_bytes, void* stream) {
+  if (N < 0 || k < 1 || M < 1 || !out_offsets || !aligned16(out_offsets)) return MORE_ERR_INVALID_ARG;
+  if (k > MORE_KMAX || M > MORE_MMAX || N * (int64_t)k > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
+  const int64_t S = N * (int64_t)k;
+  if (S > 0 && (!idx || !out_sorted || !scratch || !aligned16(idx) || !aligned16(out_sorted) ||
+                !aligned16(scratch) || scratch_bytes < (size_t)dispatch_scratch_bytes(S, M)))
+    return MORE_ERR_INVALID_ARG;
+  unsigned int* status = status_word();
+  if (!status) return MORE_ERR_CUDA;
+  return launch_dispatch(idx, S, M, out_offsets, out_sorted, scratch, status,
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MORE_OK
+             : MORE_ERR_CUDA;
+}
+
 size_t more_route_unfused_scratch_bytes(int64_t N, int r, int M) {
   if (N < 0 || r < 1 || M < 1) return 0;
   return unfused_scratch_bytes(N, r, M);

@@ -25,6 +25,9 @@ struct RouteArgs {
 
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_small_n(const RouteArgs& a);
+int64_t dispatch_scratch_bytes(int64_t S, int M);
+cudaError_t launch_dispatch(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted,
+                            void* scratch, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, float* out_psum);
 cudaError_t launch_fused_tc(const RouteArgs& a);
 bool fused_tc_supports(const RouteArgs& a);

@@ -90,6 +90,30 @@ def test_train_entry_rejects_invalid_arguments(lib, kwargs, expected):
     assert st == expected
 
 
+@pytest.mark.parametrize("kwargs,expected", [
+    (dict(k=0), 1), (dict(M=0), 1), (dict(N=-1), 1), (dict(offsets=0), 1), (dict(offsets=8), 1),
+    (dict(idx=0), 1), (dict(sorted_=0), 1), (dict(scratch=0), 1), (dict(scratch_bytes=-1), 1),
+    (dict(k=17), 2), (dict(M=262152), 2),
+])
+def test_dispatch_rejects_invalid_arguments(lib, kwargs, expected):
+    P = ctypes.c_void_p
+    a = dict(N=100, k=4, M=64, idx=16, offsets=16, sorted_=16, scratch=16, scratch_bytes=0)
+    a.update(kwargs)
+    need = lib.more_dispatch_scratch_bytes(max(a["N"], 0), max(a["k"], 1), max(a["M"], 1))
+    nbytes = need + a["scratch_bytes"] if kwargs.get("scratch_bytes") is not None else need
+    opt = lambda v: P(v) if v else None
+    st = lib.more_dispatch(opt(a["idx"]), a["N"], a["k"], a["M"], opt(a["offsets"]), opt(a["sorted_"]),
+                           opt(a["scratch"]), nbytes, None)
+    assert st == expected
+
+
+def test_dispatch_scratch_size():
+    import mixture_experts_rank_b200 as m
+    assert m.dispatch_scratch_bytes(262144, 8, 4096) >= (262144 * 8 // 2048) * 4096 * 4
+    assert m.dispatch_scratch_bytes(-1, 8, 64) == 0
+    assert m.dispatch_scratch_bytes(1 << 28, 16, 64) == 0  # N k beyond 2^31 slots
+
+
 def test_package_refuses_to_run_without_the_library(monkeypatch, tmp_path):
     """The binding has no fallback: a missing nvcc and library means import fails."""
     import importlib
