@@ -10,6 +10,8 @@ data path; the helpers below are the host-side bookkeeping around it:
 * ``global_expert_counts``: the sum over ranks of the per-rank expert counts
   (the per-expert load statistic f of App. F eq. (9) over the whole batch), one
   all-reduce of M integers, outside the routing call;
+* ``global_psum``: the same for the softmax column sums psum of the training call
+  (App. F eq. (7)), so the balancing loss of eq. (9) covers the whole batch;
 * ``max_over_ranks``: the slowest rank's time, which sets the batch's time.
 """
 from __future__ import annotations
@@ -31,6 +33,16 @@ def global_expert_counts(local_counts: torch.Tensor, group=None) -> torch.Tensor
     import torch.distributed as dist
 
     total = local_counts.to(torch.int64).clone()
+    dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
+    return total
+
+
+def global_psum(local_psum: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum of every rank's ``out_psum`` (fp32 [M], from ``route_train``) in fp64: the column
+    sum of the full softmax over the whole batch (App. F eq. (7)), for the balancing loss."""
+    import torch.distributed as dist
+
+    total = local_psum.to(torch.float64).clone()
     dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
     return total
 

@@ -43,9 +43,11 @@ def _rank_main(rank, world, port, n_total, shape, out_dir):
         res = oracle.route(X, R1, R2, count, h, r, M, k, threads=2)
         local = torch.from_numpy(res.counts.astype(np.int32))
         total = shard.global_expert_counts(local)
+        st = oracle.train_stats(X, R1, R2, count, h, r, M, threads=2)
+        psum = shard.global_psum(torch.from_numpy(st.psum.astype(np.float32)))
         slowest = shard.max_over_ranks(1.5 + rank, torch.device("cpu"))
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), begin=begin, count=count, idx=res.idx,
-                 total=total.numpy(), slowest=slowest)
+                 total=total.numpy(), slowest=slowest, psum=psum.numpy())
     finally:
         dist.destroy_process_group()
 
@@ -80,7 +82,10 @@ def test_two_gloo_ranks_match_single_batch(tmp_path):
     whole = oracle.route(X, R1, R2, n_total, h, r, M, k, threads=2)
     idx = np.concatenate([p["idx"] for p in parts])
     np.testing.assert_array_equal(idx, whole.idx)                  # shards cover the batch in order
+    whole_stats = oracle.train_stats(X, R1, R2, n_total, h, r, M, threads=2)
     for p in parts:
         np.testing.assert_array_equal(p["total"], whole.counts)    # all-reduced counts = whole batch
         assert float(p["slowest"]) == 2.5                          # max over ranks
+        # all-reduced softmax column sums = the whole batch's (fp32 per rank, then summed)
+        np.testing.assert_allclose(p["psum"], whole_stats.psum, rtol=1e-6)
     assert int(parts[0]["total"].sum()) == n_total * k
