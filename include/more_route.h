@@ -70,7 +70,7 @@ typedef enum more_status {
 typedef enum more_variant {
   MORE_VARIANT_AUTO = 0,     /* the fused tensor-core kernel for large N, the small-N kernel otherwise */
   MORE_VARIANT_FUSED_TC = 1, /* persistent kernel: TMA-staged X, tcgen05 MMAs into TMEM             */
-  MORE_VARIANT_SMALL_N = 2   /* CUDA-core kernel, one warp per token (decode-sized batches)         */
+  MORE_VARIANT_SMALL_N = 2   /* CUDA-core kernel, one CTA of 16 warps per token (decode batches)    */
 } more_variant;
 
 /*
@@ -160,7 +160,7 @@ const char* more_status_string(more_status status);
  *   out_psum[i] = sum_n exp(l_ni - out_m[n]) / out_Z[n]
  *                                                    fp32 [M], the column sum of the full
  *                                                    softmax (eq. (7)); the call zeroes it first
- * The Switch loss of eq. (9) is then M / N * sum_i f_i psum_i with f from out_expert_count.
+ * The Switch loss of eq. (9) is then (M / N) sum_i f_i psum_i, with f_i = out_expert_count[i] / (N k).
  * The logits are those of more_route (z carried as the bf16 pair z_hi + z_lo, fp32
  * accumulation); the statistics use fp32 exp.  Requirements: as for more_route, plus
  * out_psum non-NULL, out_m and out_Z non-NULL unless N == 0, all three 16-byte aligned,
