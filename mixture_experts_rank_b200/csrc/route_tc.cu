@@ -31,16 +31,21 @@
 //               k-th chunk maximum) and only chunks whose maximum reaches
 //               tlow - 2 eps can hold a top-k expert.  (token, chunk) pairs are
 //               bucketed by chunk with a counting sort.
-//     pass 2    the four warps of a tile's owning warpgroup read, for every pair of
-//               their chunk, the token's column and ballot the experts whose exact
-//               logit reaches tlow - eps (the candidates).
-//     finalize  one warp per token ranks its few candidates in routing order
-//               (larger logit, then lower expert), softmax, stores, counts.
+//     pass 2    a tile is worked by two warpgroups (0-1 for even tiles, 2-3 for odd):
+//               the two warps of a lane group split the pairs of their chunk, read
+//               each pair's token column and ballot the experts whose exact logit
+//               reaches tlow - eps (the candidates).
+//     finalize  four threads per token rank its few candidates in routing order
+//               (larger logit, then lower expert) into a shared-memory staging of the
+//               outputs, which the tile writes with coalesced stores; softmax, counts.
 //               A list too short to certify the cut, or more candidates than the
 //               slots hold, sends the token to an exact recomputation on CUDA
 //               cores shared by all sixteen consumer warps.
-// Every barrier wait is bounded (a few seconds); on expiry the kernel records
-// MORE_DEVERR_WAIT_TIMEOUT in the library's device error word and unwinds.
+// Every consumer warp waits for every logit tile and arrives once on its empty
+// barrier, so no warp can fall two phases behind a buffer (a parity wait cannot tell
+// those apart).  Every barrier wait, the consumers' own barrier included, is bounded
+// (a few seconds); on expiry the kernel records MORE_DEVERR_WAIT_TIMEOUT in the
+// library's device error word and every role unwinds.
 #include <cudaTypedefs.h>
 
 #include "more_internal.cuh"
