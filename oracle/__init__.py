@@ -202,3 +202,47 @@ def dispatch(idx, M: int) -> Dispatch:
     counts = np.bincount(flat, minlength=M)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
     return Dispatch(offsets, order.astype(np.int64))
+
+
+class RouterGrads(NamedTuple):
+    X: np.ndarray   # (N, h) gradient of the loss with respect to X
+    R1: np.ndarray  # (h, r) ... to R1
+    R2: np.ndarray  # (r, M) ... to R2
+    g: np.ndarray   # (N,) g_n = sum_i pbar_i P_ni of eq. (12)
+
+
+def router_backward_f64(X, R1, R2, top_idx, top_vals_bar, pbar) -> RouterGrads:
+    """Backward of the low-rank router ("MoRE", App. F, F.2.2, Algorithm 3 and eqs. (10)-(12)),
+    fp64 throughout, for float inputs (the bf16 entry point widens and calls this).
+
+    Two gradients arrive: ``top_vals_bar`` (N x k), the gradient of the loss with respect to
+    the selected logits l[n, top_idx[n, j]], and ``pbar`` (M), the gradient with respect to
+    psum (eq. (7)).  In the steps of Algorithm 3: z = X R1; the logits l = z R2 and the full
+    softmax P over all M experts; g_n = sum_i pbar_i P_ni; the logit gradient
+    ybar = P (pbar - g) (eq. (12)) plus top_vals_bar scattered into the selected columns;
+    zbar = ybar R2^T and the R2 gradient z^T ybar; the X gradient zbar R1^T and the R1
+    gradient X^T zbar.  Matrix products are library matmuls.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    R1 = np.asarray(R1, dtype=np.float64)
+    R2 = np.asarray(R2, dtype=np.float64)
+    top_idx = np.asarray(top_idx, dtype=np.int64)
+    top_vals_bar = np.asarray(top_vals_bar, dtype=np.float64)
+    pbar = np.asarray(pbar, dtype=np.float64)
+    N = X.shape[0]
+    z = X @ R1
+    logits = z @ R2
+    m = logits.max(axis=1, keepdims=True)
+    E = np.exp(logits - m)
+    P = E / E.sum(axis=1, keepdims=True)
+    g = P @ pbar
+    ybar = P * (pbar[None, :] - g[:, None])
+    np.add.at(ybar, (np.repeat(np.arange(N), top_idx.shape[1]), top_idx.ravel()), top_vals_bar.ravel())
+    zbar = ybar @ R2.T
+    return RouterGrads(zbar @ R1.T, X.T @ zbar, z.T @ ybar, g)
+
+
+def router_backward(X, R1, R2, N: int, h: int, r: int, M: int, top_idx, top_vals_bar, pbar) -> RouterGrads:
+    """:func:`router_backward_f64` on bf16 inputs (raw bit patterns, widened exactly)."""
+    wide = lambda a, shape: ((_u16(a, shape).astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return router_backward_f64(wide(X, (N, h)), wide(R1, (h, r)), wide(R2, (r, M)), top_idx, top_vals_bar, pbar)

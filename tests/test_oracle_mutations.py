@@ -80,3 +80,33 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
         except AssertionError:
             caught.append(getattr(pin, "__name__", "pin"))
     assert caught, f"no pin caught the planted mistake {name}"
+
+
+PY_MUTATIONS = {
+    "backward_g_sign": ("ybar = P * (pbar[None, :] - g[:, None])", "ybar = P * (pbar[None, :] + g[:, None])"),
+    "backward_no_topk_scatter": ("np.add.at(ybar,", "(lambda *a: None)(ybar,"),
+    "backward_R1_grad_from_z": ("X.T @ zbar, z.T @ ybar, g)", "X.T @ (z * 0 + zbar.mean()), z.T @ ybar, g)"),
+}
+PY_PINS = [pins.test_backward_matches_finite_differences, pins.test_backward_matches_torch_autograd,
+           pins.test_backward_constant_pbar_and_bf16_entry]
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_planted_backward_mistake_is_caught(name, monkeypatch):
+    """The same for the numpy backward: a mutated copy of the oracle module's source."""
+    import types
+
+    old, new = PY_MUTATIONS[name]
+    src = open(oracle.__file__).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    mutant = types.ModuleType("oracle_mutant")
+    mutant.__file__ = oracle.__file__
+    exec(compile(src.replace(old, new), oracle.__file__, "exec"), mutant.__dict__)
+    monkeypatch.setattr(oracle, "router_backward_f64", mutant.router_backward_f64)
+    caught = []
+    for pin in PY_PINS:
+        try:
+            pin()
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"

@@ -365,3 +365,69 @@ def test_dispatch_invariants_on_routing_output():
         assert np.all(np.diff(seg) > 0)
     with pytest.raises(ValueError):
         oracle.dispatch(np.array([[0, M]]), M)
+
+
+# --- backward (App. F, F.2.2, Algorithm 3) -------------------------------------------------------
+
+def _backward_case(seed, N=3, h=7, r=4, M=9, k=2):
+    rng = np.random.default_rng(seed)
+    X, R1, R2 = rng.standard_normal((N, h)), rng.standard_normal((h, r)) / 2, rng.standard_normal((r, M)) / 2
+    top_idx = np.argsort(-(X @ R1 @ R2), axis=1, kind="stable")[:, :k]
+    return X, R1, R2, top_idx, rng.standard_normal((N, k)), rng.standard_normal(M)
+
+
+def _loss(X, R1, R2, top_idx, tvb, pbar):
+    """sum tvb * selected logits + pbar . psum: the loss whose gradients Algorithm 3 returns."""
+    logits = X @ R1 @ R2
+    E = np.exp(logits - logits.max(axis=1, keepdims=True))
+    P = E / E.sum(axis=1, keepdims=True)
+    return float((tvb * np.take_along_axis(logits, top_idx, axis=1)).sum() + P.sum(axis=0) @ pbar)
+
+
+def test_backward_matches_finite_differences():
+    X, R1, R2, ti, tvb, pbar = _backward_case(1)
+    gr = oracle.router_backward_f64(X, R1, R2, ti, tvb, pbar)
+    for name, A, G in (("X", X, gr.X), ("R1", R1, gr.R1), ("R2", R2, gr.R2)):
+        fd = np.zeros_like(A)
+        for idx in np.ndindex(A.shape):
+            d = 1e-6
+            A[idx] += d
+            up = _loss(X, R1, R2, ti, tvb, pbar)
+            A[idx] -= 2 * d
+            dn = _loss(X, R1, R2, ti, tvb, pbar)
+            A[idx] += d
+            fd[idx] = (up - dn) / (2 * d)
+        np.testing.assert_allclose(G, fd, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_backward_matches_torch_autograd():
+    import torch
+
+    X, R1, R2, ti, tvb, pbar = _backward_case(2, N=5, h=12, r=6, M=20, k=3)
+    gr = oracle.router_backward_f64(X, R1, R2, ti, tvb, pbar)
+    tX, tR1, tR2 = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (X, R1, R2))
+    logits = tX @ tR1 @ tR2
+    loss = (torch.tensor(tvb) * torch.gather(logits, 1, torch.tensor(ti))).sum() + \
+        torch.softmax(logits, dim=1).sum(dim=0) @ torch.tensor(pbar)
+    loss.backward()
+    np.testing.assert_allclose(gr.X, tX.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(gr.R1, tR1.grad.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(gr.R2, tR2.grad.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_backward_constant_pbar_and_bf16_entry():
+    """A constant pbar adds the same to every psum_i's weight, and sum_i psum_i = N does not
+    depend on the logits: the balancing term's gradient vanishes, and g_n equals that constant."""
+    X, R1, R2, ti, tvb, _ = _backward_case(3)
+    with_c = oracle.router_backward_f64(X, R1, R2, ti, tvb, np.full(R2.shape[1], 0.37))
+    without = oracle.router_backward_f64(X, R1, R2, ti, tvb, np.zeros(R2.shape[1]))
+    np.testing.assert_allclose(with_c.g, 0.37, rtol=1e-14)
+    np.testing.assert_allclose(with_c.X, without.X, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(with_c.R2, without.R2, rtol=1e-12, atol=1e-14)
+    N, h, r, M = 4, 16, 8, 24
+    Xb, R1b, R2b = syn.router_inputs(N, h, r, M, seed=4)
+    ti = oracle.route(Xb, R1b, R2b, N, h, r, M, 2, threads=1).idx
+    gb = oracle.router_backward(Xb, R1b, R2b, N, h, r, M, ti, np.ones((N, 2)), np.zeros(M))
+    gf = oracle.router_backward_f64(syn.bf16_bits_to_f64(Xb), syn.bf16_bits_to_f64(R1b), syn.bf16_bits_to_f64(R2b), ti,
+                                    np.ones((N, 2)), np.zeros(M))
+    np.testing.assert_array_equal(gb.R1, gf.R1)
