@@ -192,6 +192,43 @@ size_t more_dispatch_scratch_bytes(int64_t N, int k, int M);
 more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
                           int32_t* out_sorted, void* scratch, size_t scratch_bytes, void* stream);
 
+/*
+ * Backward of the router ("MoRE", App. F, F.2.2, Algorithm 3 and eqs. (10)-(12)), with z
+ * recomputed from X (activation recompute), in fp32 on the CUDA cores.  With z = X R1,
+ * l = z R2 (fp32) and P_ni = exp(l_ni - saved_m[n]) / saved_Z[n]:
+ *   g_n      = sum_i pbar_i P_ni                                  (eq. (12))
+ *   ybar_ni  = P_ni (pbar_i - g_n) + sum_j [top_idx[n][j] = i] top_vals_bar[n][j]
+ *   out_Xbar  = ybar R2^T R1^T        fp32 [N][h]   (gradient with respect to X)
+ *   out_R1bar = X^T (ybar R2^T)       fp32 [h][r]
+ *   out_R2bar = z^T ybar              fp32 [r][M]
+ *   out_g     = g                     fp32 [N]      (may be NULL)
+ * Inputs (device):
+ *   X, R1, R2       bf16 as for more_route;
+ *   top_idx         int32 [N][k], the forward's selections (constants of the backward); a
+ *                   value outside [0, M) is skipped and sets MORE_DEVERR_BAD_INPUT; a
+ *                   repeated index receives each of its gradients;
+ *   top_vals_bar    fp32 [N][k], the gradient on the selected logits; NULL for none (then
+ *                   top_idx may be NULL);
+ *   pbar            fp32 [M], the gradient on psum (the load-balancing term); NULL for none
+ *                   (then g = 0 and saved_m / saved_Z are not read);
+ *   saved_m, saved_Z  fp32 [N], as more_route_train returns them (Algorithm 2), required
+ *                   when pbar is given and N > 0;
+ *   scratch         at least more_route_backward_scratch_bytes(N, h, r, M) bytes (z, zbar, g
+ *                   and per-split partial sums); its contents need no initialisation.
+ * Every output is overwritten (not accumulated into).  Requirements: as for more_route
+ * (h, M multiples of 8, r a multiple of 16 in [16, 128], 1 <= k <= MORE_KMAX, k <= M,
+ * M <= MORE_MMAX, N < 2^31), out_R1bar and out_R2bar non-NULL, X / out_Xbar / scratch
+ * non-NULL unless N == 0, every non-NULL pointer 16-byte aligned.  N == 0 zeroes out_R1bar
+ * and out_R2bar.  Asynchronous on `stream` (four kernels); allocates nothing; the result
+ * does not depend on the launch (fixed summation order, no atomics on the gradients).
+ */
+size_t more_route_backward_scratch_bytes(int64_t N, int h, int r, int M);
+more_status more_route_backward(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                                int k, const int32_t* top_idx, const float* top_vals_bar, const float* pbar,
+                                const float* saved_m, const float* saved_Z, float* out_Xbar, float* out_R1bar,
+                                float* out_R2bar, float* out_g, void* scratch, size_t scratch_bytes,
+                                void* stream);
+
 /* MORE_ROUTE_ABI_VERSION of the built library. */
 int more_abi_version(void);
 

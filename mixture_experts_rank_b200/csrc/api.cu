@@ -164,6 +164,52 @@ more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* 
              : MORE_ERR_CUDA;
 }
 
+size_t more_route_backward_scratch_bytes(int64_t N, int h, int r, int M) {
+  if (N < 0 || N > 0x7fffffffLL || h < 1 || r < 1 || r > 128 || M < 1) return 0;
+  return (size_t)backward_scratch_bytes(N, h, r, M);
+}
+
+more_status more_route_backward(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                                int k, const int32_t* top_idx, const float* top_vals_bar, const float* pbar,
+                                const float* saved_m, const float* saved_Z, float* out_Xbar, float* out_R1bar,
+                                float* out_R2bar, float* out_g, void* scratch, size_t scratch_bytes,
+                                void* stream) {
+  if (N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1) return MORE_ERR_INVALID_ARG;
+  if (!R1 || !R2 || !out_R1bar || !out_R2bar) return MORE_ERR_INVALID_ARG;
+  if (N > 0 && (!X || !out_Xbar || !scratch || (top_vals_bar && !top_idx) || (pbar && (!saved_m || !saved_Z))))
+    return MORE_ERR_INVALID_ARG;
+  const void* ptrs[] = {X,       R1,      R2,       top_idx,   top_vals_bar, pbar, saved_m,
+                        saved_Z, out_Xbar, out_R1bar, out_R2bar, out_g,        scratch};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MORE_ERR_INVALID_ARG;
+  if (N > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
+  if (k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX) return MORE_ERR_UNSUPPORTED;
+  if (N > 0 && scratch_bytes < (size_t)backward_scratch_bytes(N, h, r, M)) return MORE_ERR_INVALID_ARG;
+  BackwardArgs b;
+  b.X = static_cast<const __nv_bfloat16*>(X);
+  b.R1 = static_cast<const __nv_bfloat16*>(R1);
+  b.R2 = static_cast<const __nv_bfloat16*>(R2);
+  b.N = N;
+  b.h = h;
+  b.r = r;
+  b.M = M;
+  b.k = k;
+  b.top_idx = top_idx;
+  b.top_vals_bar = top_vals_bar;
+  b.pbar = pbar;
+  b.m = saved_m;
+  b.Z = saved_Z;
+  b.Xbar = out_Xbar;
+  b.R1bar = out_R1bar;
+  b.R2bar = out_R2bar;
+  b.g = out_g;
+  b.scratch = scratch;
+  b.status = status_word();
+  b.stream = static_cast<cudaStream_t>(stream);
+  if (!b.status) return MORE_ERR_CUDA;
+  return launch_backward(b) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
 size_t more_route_unfused_scratch_bytes(int64_t N, int r, int M) {
   if (N < 0 || r < 1 || M < 1) return 0;
   return unfused_scratch_bytes(N, r, M);

@@ -29,6 +29,29 @@ int64_t dispatch_scratch_bytes(int64_t S, int M);
 cudaError_t launch_dispatch(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted,
                             void* scratch, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, float* out_psum);
+
+// Arguments of one backward call after validation (pointers as in more_route_backward).
+struct BackwardArgs {
+  const __nv_bfloat16* X;
+  const __nv_bfloat16* R1;
+  const __nv_bfloat16* R2;
+  int64_t N;
+  int h, r, M, k;
+  const int32_t* top_idx;     // may be null (with top_vals_bar)
+  const float* top_vals_bar;  // may be null
+  const float* pbar;          // may be null (then m and Z are not read)
+  const float* m;
+  const float* Z;
+  float* Xbar;
+  float* R1bar;
+  float* R2bar;
+  float* g;  // may be null
+  void* scratch;
+  unsigned int* status;
+  cudaStream_t stream;
+};
+int64_t backward_scratch_bytes(int64_t N, int h, int r, int M);
+cudaError_t launch_backward(const BackwardArgs& b);
 cudaError_t launch_fused_tc(const RouteArgs& a);
 bool fused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused(const RouteArgs& a, void* scratch);
