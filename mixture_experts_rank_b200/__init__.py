@@ -20,7 +20,8 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "route_train", "dispatch", "dispatch_scratch_bytes", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status",
+__all__ = ["route", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
+           "dispatch_scratch_bytes", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status",
            "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
 KMAX = 16
@@ -55,6 +56,10 @@ def _load_library() -> ctypes.CDLL:
     lib.more_dispatch.argtypes = [P, I64, I, I, P, P, P, ctypes.c_size_t, P]
     lib.more_route_train.restype = I
     lib.more_route_train.argtypes = route_args + [P, P, P, P]
+    lib.more_route_backward_scratch_bytes.restype = ctypes.c_size_t
+    lib.more_route_backward_scratch_bytes.argtypes = [I64, I, I, I]
+    lib.more_route_backward.restype = I
+    lib.more_route_backward.argtypes = [P, P, P, I64, I, I, I, I] + [P] * 10 + [ctypes.c_size_t, P]
     lib.more_route_unfused_scratch_bytes.restype = ctypes.c_size_t
     lib.more_route_unfused_scratch_bytes.argtypes = [I64, I, I]
     lib.more_device_status.restype = I
@@ -162,6 +167,63 @@ def route_train(X: torch.Tensor, R1: torch.Tensor, R2: torch.Tensor, k: int, *, 
                                _stream_handle(stream))
     _check(st, "more_route_train")
     return (*outs, out_m, out_Z, out_psum)
+
+
+def route_backward_scratch_bytes(N: int, h: int, r: int, M: int) -> int:
+    return int(_lib.more_route_backward_scratch_bytes(N, h, r, M))
+
+
+def _as_f32(t, name, shape):
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape {shape}")
+    return t
+
+
+def route_backward(X: torch.Tensor, R1: torch.Tensor, R2: torch.Tensor, k: int, *, top_idx=None,
+                   top_vals_bar=None, pbar=None, m=None, Z=None, scratch: torch.Tensor | None = None,
+                   out_Xbar=None, out_R1bar=None, out_R2bar=None, out_g=None, stream=None):
+    """Backward of the router (App. F, Algorithm 3) with z recomputed from X.
+
+    ``top_idx`` (int32 [N, k]) and ``top_vals_bar`` (fp32 [N, k]): the forward's selections and
+    the gradient on the selected logits; ``pbar`` (fp32 [M]): the gradient on psum, with ``m``
+    and ``Z`` (fp32 [N]) as :func:`route_train` returns them.  Either gradient may be None.
+    Returns ``(Xbar fp32 [N, h], R1bar fp32 [h, r], R2bar fp32 [r, M], g fp32 [N])``.
+    """
+    X, R1, R2 = _as_bf16(X, "X"), _as_bf16(R1, "R1"), _as_bf16(R2, "R2")
+    N, h = X.shape
+    h1, r = R1.shape
+    r1, M = R2.shape
+    if h1 != h or r1 != r:
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, R1 {tuple(R1.shape)}, R2 {tuple(R2.shape)}")
+    if top_vals_bar is not None:
+        if top_idx is None or top_idx.dtype != torch.int32 or not top_idx.is_cuda or \
+                not top_idx.is_contiguous() or tuple(top_idx.shape) != (N, k):
+            raise ValueError("top_idx must be a contiguous int32 CUDA tensor of shape [N, k]")
+        _as_f32(top_vals_bar, "top_vals_bar", (N, k))
+    else:
+        top_idx = None
+    if pbar is not None:
+        _as_f32(pbar, "pbar", (M,))
+        if m is None or Z is None:
+            raise ValueError("pbar needs the forward's m and Z")
+        _as_f32(m, "m", (N,))
+        _as_f32(Z, "Z", (N,))
+    else:
+        m = Z = None
+    dev = X.device
+    if scratch is None:
+        scratch = torch.empty(max(route_backward_scratch_bytes(N, h, r, M), 16), dtype=torch.uint8, device=dev)
+    out_Xbar = torch.empty((N, h), dtype=torch.float32, device=dev) if out_Xbar is None else out_Xbar
+    out_R1bar = torch.empty((h, r), dtype=torch.float32, device=dev) if out_R1bar is None else out_R1bar
+    out_R2bar = torch.empty((r, M), dtype=torch.float32, device=dev) if out_R2bar is None else out_R2bar
+    out_g = torch.empty((N,), dtype=torch.float32, device=dev) if out_g is None else out_g
+    st = _lib.more_route_backward(_ptr(X), _ptr(R1), _ptr(R2), N, h, r, M, k, _ptr(top_idx), _ptr(top_vals_bar),
+                                  _ptr(pbar), _ptr(m), _ptr(Z), _ptr(out_Xbar), _ptr(out_R1bar), _ptr(out_R2bar),
+                                  _ptr(out_g), _ptr(scratch), scratch.numel(), _stream_handle(stream))
+    _check(st, "more_route_backward")
+    return out_Xbar, out_R1bar, out_R2bar, out_g
 
 
 def dispatch_scratch_bytes(N: int, k: int, M: int) -> int:

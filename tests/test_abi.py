@@ -28,7 +28,8 @@ def lib():
 
 def test_header_declares_the_route_entry_points():
     names = declared_functions()
-    for required in ("more_route", "more_route_variant", "more_route_train", "more_route_unfused",
+    for required in ("more_route", "more_route_variant", "more_route_train", "more_route_backward",
+                     "more_route_backward_scratch_bytes", "more_route_unfused",
                      "more_route_unfused_scratch_bytes", "more_device_status", "more_status_string",
                      "more_abi_version"):
         assert required in names
@@ -129,3 +130,33 @@ def test_package_refuses_to_run_without_the_library(monkeypatch, tmp_path):
             importlib.import_module("mixture_experts_rank_b200")
     finally:
         sys.modules["mixture_experts_rank_b200"] = saved
+
+
+@pytest.mark.parametrize("kwargs,expected", [
+    (dict(k=0), 1), (dict(N=-1), 1), (dict(h=4), 1), (dict(M=70), 1), (dict(X=0), 1), (dict(R1=0), 1),
+    (dict(R1bar=0), 1), (dict(R2bar=0), 1), (dict(Xbar=0), 1), (dict(scratch=0), 1), (dict(idx=0), 1),
+    (dict(m=0), 1), (dict(Z=0), 1), (dict(pbar=8), 1), (dict(g=40), 1), (dict(short=1), 1),
+    (dict(r=24), 2), (dict(r=144), 2), (dict(k=17, M=64), 2), (dict(M=262152), 2),
+])
+def test_backward_rejects_invalid_arguments(lib, kwargs, expected):
+    P = ctypes.c_void_p
+    a = dict(N=100, h=64, r=32, M=64, k=4, X=16, R1=16, R2=16, idx=16, tvb=16, pbar=16, m=16, Z=16, Xbar=16,
+             R1bar=16, R2bar=16, g=None, scratch=16, short=0)
+    a.update(kwargs)
+    need = lib.more_route_backward_scratch_bytes(max(a["N"], 0), a["h"], a["r"], a["M"])
+    opt = lambda v: P(v) if v else None
+    st = lib.more_route_backward(opt(a["X"]), opt(a["R1"]), opt(a["R2"]), a["N"], a["h"], a["r"], a["M"], a["k"],
+                                 opt(a["idx"]), opt(a["tvb"]), opt(a["pbar"]), opt(a["m"]), opt(a["Z"]),
+                                 opt(a["Xbar"]), opt(a["R1bar"]), opt(a["R2bar"]), opt(a["g"]), opt(a["scratch"]),
+                                 need - a["short"], None)
+    assert st == expected
+
+
+def test_backward_scratch_size():
+    import mixture_experts_rank_b200 as m
+    # z and zbar ([N][r padded to a power of two >= 16], fp32), g, and the per-split partial sums
+    assert m.route_backward_scratch_bytes(262144, 2048, 32, 4096) >= 2 * 262144 * 32 * 4 + 262144 * 4
+    assert m.route_backward_scratch_bytes(1000, 64, 48, 64) >= 2 * 1000 * 64 * 4
+    assert m.route_backward_scratch_bytes(0, 64, 32, 64) >= 0
+    assert m.route_backward_scratch_bytes(-1, 64, 32, 64) == 0
+    assert m.route_backward_scratch_bytes(10, 64, 144, 64) == 0
