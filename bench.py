@@ -8,7 +8,7 @@ workload: prefill, N = 262,144 tokens (256 sequences x 1024), h = 2048, M = 4096
 r = 32, k = 8, X rows at unit RMS, R1 ~ N(0, 1/h), R2 ~ N(0, 1/r), seed 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--variant auto|fused_tc|small_n|unfused] [--workload NAME]
+                  [--variant auto|fused_tc|small_n|unfused|train|dispatch|backward] [--workload NAME]
 
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank routes its own
 N-token shard of a larger synthetic token set (weak scaling, no collective on the
@@ -50,6 +50,7 @@ WORKLOADS = {
     "decode_N256": (256, 2048, 32, 4096, 8, False),
 }
 METRIC = "routed tokens/s (fused low-rank router + top-k)"
+BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X, R1, R2)"
 # DRAM bytes (read + write) per token of the fused kernel, from the ncu capture summarised in
 # profiles/fused_route_kernel_prefill_r32_n65536.md (N = 65,536, scaled by tokens).  Only valid
 # while that kernel is unchanged; workloads without a capture report traffic null.
@@ -146,25 +147,37 @@ def run_reference(args, world, rank):
     cores = os.cpu_count() or 1
     R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
     R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+    backward = args.variant == "backward"
+    rng = np.random.default_rng(1)
+
+    def one_step(X, S):
+        if backward:  # the oracle's Algorithm 3 on the sample, seeded selections and gradients
+            oracle.router_backward(X, R1, R2, S, h, r, M, rng.integers(0, M, (S, k)),
+                                   rng.standard_normal((S, k)), rng.standard_normal(M))
+        else:
+            oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+
     # size the per-step sample from a short probe: about args.ref_step_seconds of CPU work
     probe = max(cores, 16)
     Xp = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, probe)
     t = time.perf_counter()
-    oracle.route(Xp, R1, R2, probe, h, r, M, k, threads=cores)
+    one_step(Xp, probe)
     per_tok = (time.perf_counter() - t) / probe
-    S = int(max(cores, min(N, args.ref_step_seconds / max(per_tok, 1e-9))))
+    S = int(max(cores, min(N, args.ref_step_seconds / max(per_tok, 1e-9), 32768 if backward else N)))
     X = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, S)
     for _ in range(args.warmup):
-        oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+        one_step(X, S)
     times = []
     for _ in range(args.steps):
         t = time.perf_counter()
-        oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+        one_step(X, S)
         times.append(time.perf_counter() - t)
+    if backward:
+        cores = blas_threads()
     step = sum(times) / len(times)
     value = S / step
     sample = f"first {S} tokens of the workload per step ({S / N:.4%} of N), all M experts"
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    line = {"impl": "reference", "metric": BACKWARD_METRIC if backward else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": describe(args.workload), "N": N, "h": h, "r": r,
@@ -197,15 +210,52 @@ def cpu_baseline(workload, seconds):
             "sample": f"first {S} of the {N} tokens, all M experts, {el:.1f} s on {cores} threads"}
 
 
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        counts = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(counts) if counts else 1
+    except Exception:  # pragma: no cover
+        return 1
+
+
+def backward_cpu_baseline(workload, seconds):
+    """The oracle's backward (numpy fp64) on a bounded sample of tokens: a sample's X, R1 and
+    R2 gradients; the selections and gradients are seeded draws."""
+    import oracle
+    import synthetic as syn
+    N, h, r, M, k, unit = WORKLOADS[workload]
+    R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
+    R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+    rng = np.random.default_rng(1)
+
+    def run(S):
+        X = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, S)
+        idx = rng.integers(0, M, (S, k))
+        t = time.perf_counter()
+        oracle.router_backward(X, R1, R2, S, h, r, M, idx, rng.standard_normal((S, k)), rng.standard_normal(M))
+        return time.perf_counter() - t
+
+    probe = 256
+    per_tok = run(probe) / probe
+    S = int(max(probe, min(N, seconds / max(per_tok, 1e-9), 32768)))
+    el = run(S)
+    threads = blas_threads()
+    return {"value": S / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {S} of the {N} tokens, all M experts, {el:.1f} s (numpy, {threads} BLAS threads)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="auto", choices=["auto", "fused_tc", "small_n", "unfused", "train", "dispatch"],
+    ap.add_argument("--variant", default="auto",
+                    choices=["auto", "fused_tc", "small_n", "unfused", "train", "dispatch", "backward"],
                     help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum); "
-                         "dispatch: routing followed by more_dispatch of its indices")
+                         "dispatch: routing followed by more_dispatch of its indices; "
+                         "backward: more_route_backward (Algorithm 3) given the forward's selections, m and Z")
     ap.add_argument("--workload", default="prefill_r32", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample size, in CPU seconds")
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
@@ -261,6 +311,21 @@ def main():
         d_sorted = torch.empty((N * k,), dtype=torch.int32, device="cuda")
     if args.variant == "unfused":
         scratch = torch.empty(more.unfused_scratch_bytes(N, r, M), dtype=torch.uint8, device="cuda")
+    if args.variant == "backward":
+        # the forward's selections and statistics (untimed), seeded incoming gradients
+        b_m = torch.empty((N,), dtype=torch.float32, device="cuda")
+        b_Z = torch.empty((N,), dtype=torch.float32, device="cuda")
+        more.route_train(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
+                         out_m=b_m, out_Z=b_Z, out_psum=torch.empty((M,), dtype=torch.float32, device="cuda"))
+        grng = np.random.default_rng(2)
+        b_tvb = torch.from_numpy(grng.standard_normal((N, k)).astype(np.float32)).cuda()
+        b_pbar = torch.from_numpy(grng.standard_normal(M).astype(np.float32)).cuda()
+        b_scratch = torch.empty(max(more.route_backward_scratch_bytes(N, h, r, M), 16), dtype=torch.uint8,
+                                device="cuda")
+        b_out = (torch.empty((N, h), dtype=torch.float32, device="cuda"),
+                 torch.empty((h, r), dtype=torch.float32, device="cuda"),
+                 torch.empty((r, M), dtype=torch.float32, device="cuda"),
+                 torch.empty((N,), dtype=torch.float32, device="cuda"))
 
     def step(st=None):
         st = stream if st is None else st
@@ -270,6 +335,10 @@ def main():
         elif args.variant == "dispatch":
             more.route(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits, stream=st)
             more.dispatch(idx, M, scratch=d_scratch, out_offsets=d_off, out_sorted=d_sorted, stream=st)
+        elif args.variant == "backward":
+            more.route_backward(X, R1, R2, k, top_idx=idx, top_vals_bar=b_tvb, pbar=b_pbar, m=b_m, Z=b_Z,
+                                scratch=b_scratch, out_Xbar=b_out[0], out_R1bar=b_out[1], out_R2bar=b_out[2],
+                                out_g=b_out[3], stream=st)
         elif args.variant == "unfused":
             more.route_unfused(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate, out_expert_count=cnt,
                                out_logits=logits, stream=st)
@@ -285,7 +354,7 @@ def main():
         except more.MoreError:
             variant_used = "small_n"
         variant_used = variant_used if N >= 512 else "small_n"
-    launches_per_step = {"unfused": 3, "train": 2, "dispatch": 5}.get(args.variant, 1)
+    launches_per_step = {"unfused": 3, "train": 2, "dispatch": 5, "backward": 5}.get(args.variant, 1)
 
     def barrier():
         if dist is not None:
@@ -335,7 +404,7 @@ def main():
 
     # end to end: pinned host X in, route through the public API, results out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.variant != "backward":
         router = more.Router(R1, R2, k, N)
         Xpin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
         for _ in range(2):
@@ -372,9 +441,18 @@ def main():
                 else "fallback 6.65 TB/s",
                 "tensor": {"achieved_tflops": flops / (kernel_ms / 1e3) / 1e12, "peak_tflops": tc,
                            "frac": flops / (kernel_ms / 1e3) / 1e12 / tc}}
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        if args.variant == "backward":
+            # fp32 FMA work without recompute: z, logits, zbar, Xbar, R1bar, R2bar (6 r (h + M) per
+            # token) plus g (2 M); timed over the whole step (five launches)
+            bflops = N * (6.0 * r * (h + M) + 2.0 * M)
+            fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+            achieved_t = bflops / (ms / 1e3) / 1e12
+            roof = {"bound": "alu", "achieved": achieved_t, "peak": fp32_peak, "unit": "TFLOP/s",
+                    "frac": achieved_t / fp32_peak, "traffic": None, "timed": "whole backward step",
+                    "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz clocks.max.sm"}
+        line = {"metric": METRIC if args.variant != "backward" else BACKWARD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "vs_baseline": None, "dtype": "f32" if args.variant == "backward" else "bf16", "data": "synthetic",
                 "config": {"workload": describe(args.workload) + (f" (N overridden to {N})" if args.tokens else ""),
                            "N_per_gpu": N, "h": h, "r": r, "M": M, "k": k,
                            "variant": variant_used, "parallelism": f"token shards x{world}",
@@ -385,7 +463,8 @@ def main():
         if e2e is not None:
             line["e2e"] = e2e
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+            line["cpu_baseline"] = (backward_cpu_baseline if args.variant == "backward" else cpu_baseline)(
+                args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

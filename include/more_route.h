@@ -219,7 +219,7 @@ more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* 
  * (h, M multiples of 8, r a multiple of 16 in [16, 128], 1 <= k <= MORE_KMAX, k <= M,
  * M <= MORE_MMAX, N < 2^31), out_R1bar and out_R2bar non-NULL, X / out_Xbar / scratch
  * non-NULL unless N == 0, every non-NULL pointer 16-byte aligned.  N == 0 zeroes out_R1bar
- * and out_R2bar.  Asynchronous on `stream` (four kernels); allocates nothing; the result
+ * and out_R2bar.  Asynchronous on `stream` (five kernel launches); allocates nothing; the result
  * does not depend on the launch (fixed summation order, no atomics on the gradients).
  */
 size_t more_route_backward_scratch_bytes(int64_t N, int h, int r, int M);
