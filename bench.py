@@ -8,7 +8,8 @@ workload: prefill, N = 262,144 tokens (256 sequences x 1024), h = 2048, M = 4096
 r = 32, k = 8, X rows at unit RMS, R1 ~ N(0, 1/h), R2 ~ N(0, 1/r), seed 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--variant auto|fused_tc|small_n|unfused|train|dispatch|backward] [--workload NAME]
+                  [--variant auto|fused_tc|small_n|cluster|unfused|train|dispatch|backward]
+                  [--workload NAME]
 
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank routes its own
 N-token shard of a larger synthetic token set (weak scaling, no collective on the
@@ -252,7 +253,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto",
-                    choices=["auto", "fused_tc", "small_n", "unfused", "train", "dispatch", "backward"],
+                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "train", "dispatch", "backward"],
                     help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum); "
                          "dispatch: routing followed by more_dispatch of its indices; "
                          "backward: more_route_backward (Algorithm 3) given the forward's selections, m and Z")

@@ -70,7 +70,9 @@ typedef enum more_status {
 typedef enum more_variant {
   MORE_VARIANT_AUTO = 0,     /* the fused tensor-core kernel for large N, the small-N kernel otherwise */
   MORE_VARIANT_FUSED_TC = 1, /* persistent kernel: TMA-staged X, tcgen05 MMAs into TMEM             */
-  MORE_VARIANT_SMALL_N = 2   /* CUDA-core kernel, one CTA of 16 warps per token (decode batches)    */
+  MORE_VARIANT_SMALL_N = 2,  /* CUDA-core kernel, one CTA of 16 warps per token (decode batches)    */
+  MORE_VARIANT_CLUSTER = 3   /* CUDA-core kernel, 8 tokens per cluster of 8 CTAs: experts split over
+                                the cluster, partial top-k merged through distributed shared memory */
 } more_variant;
 
 /*

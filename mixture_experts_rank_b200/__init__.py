@@ -26,7 +26,7 @@ __all__ = ["route", "route_train", "route_backward", "route_backward_scratch_byt
 
 KMAX = 16
 STATS_MMAX = 32768
-VARIANTS = {"auto": 0, "fused_tc": 1, "small_n": 2}
+VARIANTS = {"auto": 0, "fused_tc": 1, "small_n": 2, "cluster": 3}
 STATUS = {0: "MORE_OK", 1: "MORE_ERR_INVALID_ARG", 2: "MORE_ERR_UNSUPPORTED", 3: "MORE_ERR_CUDA",
           4: "MORE_ERR_DEVICE"}
 

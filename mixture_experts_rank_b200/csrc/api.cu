@@ -97,7 +97,7 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
                                void* stream) {
   more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
   if (st != MORE_OK) return st;
-  if (variant < MORE_VARIANT_AUTO || variant > MORE_VARIANT_SMALL_N) return MORE_ERR_INVALID_ARG;
+  if (variant < MORE_VARIANT_AUTO || variant > MORE_VARIANT_CLUSTER) return MORE_ERR_INVALID_ARG;
   RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
                           stream);
   a.status = status_word();
@@ -112,6 +112,8 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
   if (variant == MORE_VARIANT_FUSED_TC) {
     if (!fused_tc_supports(a)) return MORE_ERR_UNSUPPORTED;
     err = launch_fused_tc(a);
+  } else if (variant == MORE_VARIANT_CLUSTER) {
+    err = launch_cluster(a);
   } else {
     err = launch_small_n(a);
   }

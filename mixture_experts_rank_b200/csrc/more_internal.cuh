@@ -25,6 +25,7 @@ struct RouteArgs {
 
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_small_n(const RouteArgs& a);
+cudaError_t launch_cluster(const RouteArgs& a);
 int64_t dispatch_scratch_bytes(int64_t S, int M);
 cudaError_t launch_dispatch(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted,
                             void* scratch, unsigned int* status, cudaStream_t stream);

@@ -25,73 +25,6 @@ namespace {
 constexpr int kWarpsPerBlock = 16;
 constexpr int kRMax = 128;
 
-// The 16 sums z[b .. b + 16) over this warp's hidden rows tstart + kStride j (tstart holds
-// the lane), reduced across the warp by a reduce-scatter: afterwards every value sits on
-// two neighbouring lanes; `value` is this lane's value and `index` its z index.
-__device__ __forceinline__ void warp_partial_z16_strided(const __nv_bfloat16* __restrict__ x,
-                                                         const __nv_bfloat16* __restrict__ R1, int h, int r,
-                                                         int b, int tstart, int kStride, int lane, float& value,
-                                                         int& index) {
-  float acc[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-  // batches of 4 hidden rows: all loads first, then the arithmetic, so the loads overlap
-  for (int t0 = tstart; t0 < h; t0 += 4 * kStride) {
-    float xt[4];
-    uint4 w0[4], w1[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int t = t0 + j * kStride;
-      const bool ok = t < h;
-      xt[j] = ok ? __bfloat162float(x[t]) : 0.f;
-      const uint4* w = reinterpret_cast<const uint4*>(R1 + (size_t)(ok ? t : 0) * r + b);
-      w0[j] = ok ? __ldg(w) : make_uint4(0u, 0u, 0u, 0u);
-      w1[j] = ok ? __ldg(w + 1) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat162* p0 = reinterpret_cast<const __nv_bfloat162*>(&w0[j]);
-      const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&w1[j]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 u = __bfloat1622float2(p0[q]);
-        const float2 v = __bfloat1622float2(p1[q]);
-        acc[2 * q] = fmaf(xt[j], u.x, acc[2 * q]);
-        acc[2 * q + 1] = fmaf(xt[j], u.y, acc[2 * q + 1]);
-        acc[8 + 2 * q] = fmaf(xt[j], v.x, acc[8 + 2 * q]);
-        acc[8 + 2 * q + 1] = fmaf(xt[j], v.y, acc[8 + 2 * q + 1]);
-      }
-    }
-  }
-  // reduce-scatter: after the step with distance d a lane keeps the half selected by its bit d
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const bool hi = lane & 16;
-    const float send = hi ? acc[j] : acc[j + 8];
-    acc[j] = (hi ? acc[j + 8] : acc[j]) + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const bool hi = lane & 8;
-    const float send = hi ? acc[j] : acc[j + 4];
-    acc[j] = (hi ? acc[j + 4] : acc[j]) + __shfl_xor_sync(0xffffffffu, send, 8);
-  }
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const bool hi = lane & 4;
-    const float send = hi ? acc[j] : acc[j + 2];
-    acc[j] = (hi ? acc[j + 2] : acc[j]) + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-  {
-    const bool hi = lane & 2;
-    const float send = hi ? acc[0] : acc[1];
-    acc[0] = (hi ? acc[1] : acc[0]) + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-  acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
-  value = acc[0];
-  index = b + ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-}
-
 // The same with warp w taking hidden rows w*32 + lane + 512 j (all 16 warps on one token).
 __device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict__ x,
                                                  const __nv_bfloat16* __restrict__ R1, int h, int r, int b,
