@@ -83,30 +83,44 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
 
 
 PY_MUTATIONS = {
-    "backward_g_sign": ("ybar = P * (pbar[None, :] - g[:, None])", "ybar = P * (pbar[None, :] + g[:, None])"),
-    "backward_no_topk_scatter": ("np.add.at(ybar,", "(lambda *a: None)(ybar,"),
-    "backward_R1_grad_from_z": ("X.T @ zbar, z.T @ ybar, g)", "X.T @ (z * 0 + zbar.mean()), z.T @ ybar, g)"),
+    # name: (oracle function, source anchor, replacement)
+    "backward_g_sign": ("router_backward_f64", "ybar = P * (pbar[None, :] - g[:, None])",
+                        "ybar = P * (pbar[None, :] + g[:, None])"),
+    "backward_no_topk_scatter": ("router_backward_f64", "np.add.at(ybar,", "(lambda *a: None)(ybar,"),
+    "backward_R1_grad_from_z": ("router_backward_f64", "X.T @ zbar, z.T @ ybar, g)",
+                                "X.T @ (z * 0 + zbar.mean()), z.T @ ybar, g)"),
+    "dispatch_within_expert_reversed": ("dispatch", 'order = np.argsort(flat, kind="stable")',
+                                        'order = flat.size - 1 - np.argsort(flat[::-1], kind="stable")'),
+    "dispatch_offsets_inclusive": ("dispatch", "offsets = np.concatenate([[0], np.cumsum(counts)])",
+                                   "offsets = np.concatenate([np.cumsum(counts), [flat.size]])"),
+    "dispatch_counts_drop_last_slot": ("dispatch", "counts = np.bincount(flat, minlength=M)",
+                                       "counts = np.bincount(flat[:-1], minlength=M)"),
 }
-PY_PINS = [pins.test_backward_matches_finite_differences, pins.test_backward_matches_torch_autograd,
-           pins.test_backward_constant_pbar_and_bf16_entry]
+PY_PINS = {
+    "router_backward_f64": [pins.test_backward_matches_finite_differences, pins.test_backward_matches_torch_autograd,
+                            pins.test_backward_constant_pbar_and_bf16_entry],
+    "dispatch": [lambda: pins.test_dispatch_matches_brute_force(50, 4, 16),
+                 pins.test_dispatch_invariants_on_routing_output],
+}
 
 
 @pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
-def test_planted_backward_mistake_is_caught(name, monkeypatch):
-    """The same for the numpy backward: a mutated copy of the oracle module's source."""
+def test_planted_python_mistake_is_caught(name, monkeypatch):
+    """The same for the numpy parts of the oracle (backward, dispatch): a mutated copy of the
+    module's source, with the mutated function put in place of the original."""
     import types
 
-    old, new = PY_MUTATIONS[name]
+    func, old, new = PY_MUTATIONS[name]
     src = open(oracle.__file__).read()
     assert src.count(old) == 1, f"mutation anchor for {name} not found"
     mutant = types.ModuleType("oracle_mutant")
     mutant.__file__ = oracle.__file__
     exec(compile(src.replace(old, new), oracle.__file__, "exec"), mutant.__dict__)
-    monkeypatch.setattr(oracle, "router_backward_f64", mutant.router_backward_f64)
+    monkeypatch.setattr(oracle, func, getattr(mutant, func))
     caught = []
-    for pin in PY_PINS:
+    for pin in PY_PINS[func]:
         try:
             pin()
         except AssertionError:
-            caught.append(pin.__name__)
+            caught.append(getattr(pin, "__name__", "pin"))
     assert caught, f"no pin caught the planted mistake {name}"
