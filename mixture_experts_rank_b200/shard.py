@@ -12,6 +12,9 @@ data path; the helpers below are the host-side bookkeeping around it:
   all-reduce of M integers, outside the routing call;
 * ``global_psum``: the same for the softmax column sums psum of the training call
   (App. F eq. (7)), so the balancing loss of eq. (9) covers the whole batch;
+* ``global_router_grads``: the sum over ranks of the R1 and R2 gradients of the backward
+  (App. F, Algorithm 3), each rank's a sum over its own tokens: one all-reduce of
+  h r + r M values; the X gradient stays with the rank whose rows it is;
 * ``max_over_ranks``: the slowest rank's time, which sets the batch's time.
 """
 from __future__ import annotations
@@ -45,6 +48,18 @@ def global_psum(local_psum: torch.Tensor, group=None) -> torch.Tensor:
     total = local_psum.to(torch.float64).clone()
     dist.all_reduce(total, op=dist.ReduceOp.SUM, group=group)
     return total
+
+
+def global_router_grads(R1bar: torch.Tensor, R2bar: torch.Tensor, group=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Sum over ranks of ``out_R1bar`` [h, r] and ``out_R2bar`` [r, M] (fp32, from
+    ``route_backward`` on each rank's token shard, with the same pbar on every rank), summed
+    in fp64 in one all-reduce; returns new fp64 tensors of the same shapes."""
+    import torch.distributed as dist
+
+    n1 = R1bar.numel()
+    flat = torch.cat([R1bar.reshape(-1), R2bar.reshape(-1)]).to(torch.float64)
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    return flat[:n1].view(R1bar.shape), flat[n1:].view(R2bar.shape)
 
 
 def max_over_ranks(value: float, device, group=None) -> float:

@@ -1,10 +1,11 @@
 """The multi-rank host path on CPU: two gloo ranks split a token batch by rows.
 
 Routing is independent per token ("MoRE: Scaling mixture of experts with
-hardware-aware low-rank routing", App. F), so each rank routes its own rows and
-only the per-expert counts (App. F eq. (9)) are summed across ranks.  On CPU the
-fp64 oracle stands in for each rank's routing call; what is tested is the
-sharding, the count all-reduce and the max-over-ranks timing reduction.
+hardware-aware low-rank routing", App. F), so each rank routes its own rows.  Only
+batch-wide sums cross ranks: the per-expert counts (App. F eq. (9)), the softmax
+column sums psum (eq. (7)), and the R1 and R2 gradients of the backward
+(Algorithm 3).  On CPU the fp64 oracle stands in for each rank's calls; what is
+tested is the sharding, those all-reduces, and the max-over-ranks timing reduction.
 """
 import os
 import socket
@@ -46,8 +47,15 @@ def _rank_main(rank, world, port, n_total, shape, out_dir):
         st = oracle.train_stats(X, R1, R2, count, h, r, M, threads=2)
         psum = shard.global_psum(torch.from_numpy(st.psum.astype(np.float32)))
         slowest = shard.max_over_ranks(1.5 + rank, torch.device("cpu"))
+        # backward of this rank's rows (the same pbar everywhere), R1 and R2 gradients summed
+        rng = np.random.default_rng(5)
+        tvb_all, pbar = rng.standard_normal((n_total, k)), rng.standard_normal(M)
+        g = oracle.router_backward(X, R1, R2, count, h, r, M, res.idx, tvb_all[begin:begin + count], pbar)
+        r1bar, r2bar = shard.global_router_grads(torch.from_numpy(g.R1.astype(np.float32)),
+                                                 torch.from_numpy(g.R2.astype(np.float32)))
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), begin=begin, count=count, idx=res.idx,
-                 total=total.numpy(), slowest=slowest, psum=psum.numpy())
+                 total=total.numpy(), slowest=slowest, psum=psum.numpy(), xbar=g.X, r1bar=r1bar.numpy(),
+                 r2bar=r2bar.numpy())
     finally:
         dist.destroy_process_group()
 
@@ -89,3 +97,11 @@ def test_two_gloo_ranks_match_single_batch(tmp_path):
         # all-reduced softmax column sums = the whole batch's (fp32 per rank, then summed)
         np.testing.assert_allclose(p["psum"], whole_stats.psum, rtol=1e-6)
     assert int(parts[0]["total"].sum()) == n_total * k
+    # backward: per-rank X gradients are the whole batch's rows; R1 and R2 gradients all-reduced
+    rng = np.random.default_rng(5)
+    tvb_all, pbar = rng.standard_normal((n_total, k)), rng.standard_normal(M)
+    gw = oracle.router_backward(X, R1, R2, n_total, h, r, M, whole.idx, tvb_all, pbar)
+    np.testing.assert_allclose(np.concatenate([p["xbar"] for p in parts]), gw.X, rtol=1e-12, atol=1e-15)
+    for p in parts:  # fp32 per rank, then summed: relative 1e-6 of the largest entry
+        np.testing.assert_allclose(p["r1bar"], gw.R1, rtol=0, atol=1e-6 * np.abs(gw.R1).max())
+        np.testing.assert_allclose(p["r2bar"], gw.R2, rtol=0, atol=1e-6 * np.abs(gw.R2).max())
