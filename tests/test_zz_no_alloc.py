@@ -4,8 +4,8 @@ more_route_unfused_static is for callers that may not allocate device memory (an
 external allocator or memory budget that forbids raw allocations, or a latency-critical
 path where an allocation is not acceptable): it runs the materialise-then-top-k kernels
 on a fixed scratch array inside the library.  Two calls in a row, on different inputs,
-must match more_route_unfused within the parity tolerances.  This file runs last so
-that a failure here cannot hide the results of the other tests.
+must match more_route_unfused within the parity tolerances.  tests/conftest.py runs
+this file right after the routing parity tests, ahead of the rows built on routing.
 """
 import ctypes
 
