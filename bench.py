@@ -404,9 +404,9 @@ def main():
     value = N * world / (ms / 1e3)
 
     # end to end: pinned host X in, route through the public API, results out
-    e2e = None
-    if not args.no_e2e and args.variant != "backward":
-        router = more.Router(R1, R2, k, N)
+    e2e = None  # through the public routing API; the other variants' steps are not routing calls
+    if not args.no_e2e and args.variant in more.VARIANTS:
+        router = more.Router(R1, R2, k, N, variant=args.variant)
         Xpin = torch.from_numpy(Xh.view(np.int16)).view(torch.bfloat16).pin_memory()
         for _ in range(2):
             router.route_host(Xpin)

@@ -304,11 +304,15 @@ class Router:
 
     Device buffers are allocated once for ``max_tokens`` tokens, so repeated calls
     allocate nothing.  ``route_host`` takes a (preferably pinned) CPU bf16 tensor
-    and returns CPU tensors (idx, gate, counts, logits).
+    and returns CPU tensors (idx, gate, counts, logits).  ``variant`` is the routing
+    kernel, as for :func:`route`.
     """
 
     def __init__(self, R1: torch.Tensor, R2: torch.Tensor, k: int, max_tokens: int, device="cuda",
-                 return_logits: bool = True):
+                 return_logits: bool = True, variant: str = "auto"):
+        if variant not in VARIANTS:
+            raise ValueError(f"unknown variant {variant!r}")
+        self.variant = variant
         self.R1 = R1.to(device=device, dtype=torch.bfloat16).contiguous()
         self.R2 = R2.to(device=device, dtype=torch.bfloat16).contiguous()
         self.h, self.r = self.R1.shape
@@ -335,7 +339,7 @@ class Router:
             self.X[:N].copy_(X_host, non_blocking=True)
             logits = None if self.logits is None else self.logits[:N]
             route(self.X[:N], self.R1, self.R2, self.k, out_idx=self.idx[:N], out_gate=self.gate[:N],
-                  out_expert_count=self.count, out_logits=logits, stream=s)
+                  out_expert_count=self.count, out_logits=logits, variant=self.variant, stream=s)
             self.h_idx[:N].copy_(self.idx[:N], non_blocking=True)
             self.h_gate[:N].copy_(self.gate[:N], non_blocking=True)
             self.h_count.copy_(self.count, non_blocking=True)
