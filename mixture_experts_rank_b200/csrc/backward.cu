@@ -473,16 +473,23 @@ cudaError_t launch_rp(BwdArgs a, cudaStream_t stream) {
   const size_t tok_bytes = sizeof(float) * T::kTokenBlockFloats;
   const size_t r2_bytes = sizeof(float) * T::kR2Floats;
   const size_t r1_bytes = sizeof(float) * T::kR1Floats;
-  cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_token_block_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)tok_bytes)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(bwd_r2_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r2_bytes)) !=
-      cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(bwd_r1_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r1_bytes)) !=
-      cudaSuccess)
-    return e;
+  // shared-memory limits, set once per device (a call captured into a CUDA graph then only launches)
+  static int configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
+    if ((e = cudaFuncSetAttribute(bwd_token_block_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)tok_bytes)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(bwd_r2_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)r2_bytes)) != cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(bwd_r1_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)r1_bytes)) != cudaSuccess)
+      return e;
+    if (dev >= 0 && dev < 64) configured[dev] = 1;
+  }
   const unsigned blocks = (unsigned)ceil_div(a.N, kBN);
   bwd_token_block_kernel<RP><<<blocks, kThreads, tok_bytes, stream>>>(a);
   bwd_r2_kernel<RP><<<dim3((unsigned)ceil_div(a.M, kBM), (unsigned)a.S2), kThreads, r2_bytes, stream>>>(a);
