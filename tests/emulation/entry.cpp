@@ -1,0 +1,59 @@
+// C entry points of the emulated library: the backward and the cluster routing call, with the
+// arguments the C ABI takes (host pointers here).
+#include "prelude.h"
+#include "more_internal.cuh"
+
+extern "C" long emu_backward_scratch_bytes(int64_t N, int h, int r, int M) {
+  return (long)more::backward_scratch_bytes(N, h, r, M);
+}
+
+extern "C" int emu_backward(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                            const int32_t* idx, const float* tvb, const float* pbar, const float* m, const float* Z,
+                            float* Xbar, float* R1bar, float* R2bar, float* g, void* scratch, unsigned* status) {
+  more::BackwardArgs b;
+  b.X = (const __nv_bfloat16*)X;
+  b.R1 = (const __nv_bfloat16*)R1;
+  b.R2 = (const __nv_bfloat16*)R2;
+  b.N = N;
+  b.h = h;
+  b.r = r;
+  b.M = M;
+  b.k = k;
+  b.top_idx = idx;
+  b.top_vals_bar = tvb;
+  b.pbar = pbar;
+  b.m = m;
+  b.Z = Z;
+  b.Xbar = Xbar;
+  b.R1bar = R1bar;
+  b.R2bar = R2bar;
+  b.g = g;
+  b.scratch = scratch;
+  b.status = status;
+  b.stream = nullptr;
+  return (int)more::launch_backward(b);
+}
+
+extern "C" int emu_route_cluster(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                                 int32_t* idx, float* gate, int32_t* cnt, float* logits, unsigned* status) {
+  more::RouteArgs a;
+  a.X = (const __nv_bfloat16*)X;
+  a.R1 = (const __nv_bfloat16*)R1;
+  a.R2 = (const __nv_bfloat16*)R2;
+  a.N = N;
+  a.h = h;
+  a.r = r;
+  a.M = M;
+  a.k = k;
+  a.out_idx = idx;
+  a.out_gate = gate;
+  a.out_count = cnt;
+  a.out_logits = logits;
+  a.status = status;
+  a.stream = nullptr;
+  memset(cnt, 0, sizeof(int32_t) * M);  // the C entry point zeroes the counts before launching
+  emu::cluster_size = 8;                 // cluster_route_kernel's __cluster_dims__
+  const int rc = (int)more::launch_cluster(a);
+  emu::cluster_size = 1;
+  return rc;
+}
