@@ -3,7 +3,7 @@
 The kernel sources in ``mixture_experts_rank_b200/csrc`` are compiled unchanged with g++ after a
 textual rewrite of the few CUDA-only constructs:
 - ``kernel<<<grid, block, smem, stream>>>(args)`` becomes a call of the fiber runtime;
-- dynamic shared memory comes from the runtime;
+- shared memory, dynamic and static, comes from the runtime, one copy per CTA;
 - the cooperative-groups header is replaced by the runtime's cluster calls.
 
 The runtime (``fibers.cpp``) runs each CTA's threads, or each cluster's, as fibers: barriers, warp
@@ -26,7 +26,7 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
 CSRC = os.path.join(ROOT, "mixture_experts_rank_b200", "csrc")
-KERNELS = ("backward.cu", "route_cluster.cu")
+KERNELS = ("backward.cu", "route_cluster.cu", "route_small.cu", "dispatch.cu", "route_unfused.cu")
 
 
 def _split_top(s: str) -> list[str]:
@@ -52,12 +52,32 @@ def _balanced(s: str, i: int) -> int:
     raise ValueError("unbalanced parentheses")
 
 
+def _shared_decls(src: str) -> str:
+    """Block-scope shared-memory declarations become per-CTA storage of the runtime:
+    ``extern __shared__ T name[];`` the CTA's dynamic shared memory, and each declarator of
+    ``__shared__ T a[..], b[..];`` a buffer of its own (one id per declarator)."""
+    src = re.sub(r"extern\s+__shared__\s+(?:__align__\(\d+\)\s+)?([\w:]+)\s+(\w+)\[\];",
+                 r"\1* \2 = reinterpret_cast<\1*>(::emu::smem());", src)
+    counter = [0]
+
+    def one(m):
+        indent, typ, decls = m.group(1), m.group(2), m.group(3)
+        out = []
+        for d in _split_top(decls):
+            name, dims = re.match(r"(\w+)((?:\[[^\]]+\])*)$", d.strip()).groups()
+            counter[0] += 1
+            out.append(f"{indent}auto& {name} = ::emu::shared_static<{typ}{dims}>({counter[0]});")
+        return "\n".join(out)
+
+    return re.sub(r"^([ \t]*)__shared__\s+(?:__align__\(\d+\)\s+)?([\w:]+)\s+([^;]+);", one, src, flags=re.M)
+
+
 def transform(src: str) -> str:
     """The emulated form of one kernel source."""
     src = src.replace('#include "more_internal.cuh"',
                       '#include "prelude.h"\n#include "more_internal.cuh"\n#include "postlude.h"')
     src = src.replace("#include <cooperative_groups.h>", "")
-    src = src.replace("extern __shared__ float4 smem4[];", "float4* smem4 = ::emu::smem();")
+    src = _shared_decls(src)
     out, pos = "", 0
     for m in re.finditer(r"([A-Za-z_]\w*(?:<\w+>)?)<<<", src):
         if m.start() < pos:
@@ -87,6 +107,7 @@ def build(out_dir: str | None = None, mutate: dict | None = None) -> str:
     """Compile the emulated kernels; returns the shared library's path.  ``mutate`` maps a kernel
     file name to (text, replacement): a planted mistake, for the tests that show one is caught."""
     out_dir = out_dir or tempfile.mkdtemp(prefix="more_emulation_")
+    os.makedirs(out_dir, exist_ok=True)
     srcs = [os.path.join(HERE, "fibers.cpp"), os.path.join(HERE, "entry.cpp")]
     for name in KERNELS:
         with open(os.path.join(CSRC, name)) as f:
@@ -125,6 +146,18 @@ class Emulated:
         lib.emu_backward.argtypes = [P, P, P, I64, I, I, I, I] + [P] * 11
         lib.emu_route_cluster.restype = I
         lib.emu_route_cluster.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, P, P]
+        lib.emu_route_small.restype = I
+        lib.emu_route_small.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, P, P]
+        lib.emu_unfused_scratch_bytes.restype = ctypes.c_long
+        lib.emu_unfused_scratch_bytes.argtypes = [I64, I, I]
+        lib.emu_route_unfused.restype = I
+        lib.emu_route_unfused.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, P, P, P]
+        lib.emu_train_stats.restype = I
+        lib.emu_train_stats.argtypes = [P, P, P, I64, I, I, I, P, P, P, P]
+        lib.emu_dispatch_scratch_bytes.restype = ctypes.c_long
+        lib.emu_dispatch_scratch_bytes.argtypes = [I64, I]
+        lib.emu_dispatch.restype = I
+        lib.emu_dispatch.argtypes = [P, I64, I, P, P, P, P]
         self._live = []
 
     def put(self, a) -> int | None:

@@ -1,5 +1,5 @@
-// C entry points of the emulated library: the backward and the cluster routing call, with the
-// arguments the C ABI takes (host pointers here).
+// C entry points of the emulated library: the CUDA-core kernels' launchers, with the arguments
+// the C ABI takes (host pointers here).  Each zeroes what the C ABI zeroes before launching.
 #include "prelude.h"
 #include "more_internal.cuh"
 
@@ -56,4 +56,55 @@ extern "C" int emu_route_cluster(const void* X, const void* R1, const void* R2, 
   const int rc = (int)more::launch_cluster(a);
   emu::cluster_size = 1;
   return rc;
+}
+
+namespace {
+more::RouteArgs route_args(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                           int32_t* idx, float* gate, int32_t* cnt, float* logits, unsigned* status) {
+  more::RouteArgs a;
+  a.X = (const __nv_bfloat16*)X;
+  a.R1 = (const __nv_bfloat16*)R1;
+  a.R2 = (const __nv_bfloat16*)R2;
+  a.N = N;
+  a.h = h;
+  a.r = r;
+  a.M = M;
+  a.k = k;
+  a.out_idx = idx;
+  a.out_gate = gate;
+  a.out_count = cnt;
+  a.out_logits = logits;
+  a.status = status;
+  a.stream = nullptr;
+  if (cnt) memset(cnt, 0, sizeof(int32_t) * M);
+  return a;
+}
+}  // namespace
+
+extern "C" int emu_route_small(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                               int32_t* idx, float* gate, int32_t* cnt, float* logits, unsigned* status) {
+  return (int)more::launch_small_n(route_args(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, status));
+}
+
+extern "C" long emu_unfused_scratch_bytes(int64_t N, int r, int M) { return (long)more::unfused_scratch_bytes(N, r, M); }
+
+extern "C" int emu_route_unfused(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                                 int32_t* idx, float* gate, int32_t* cnt, float* logits, void* scratch,
+                                 unsigned* status) {
+  return (int)more::launch_unfused(route_args(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, status), scratch);
+}
+
+extern "C" int emu_train_stats(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
+                               float* out_m, float* out_Z, float* out_psum, unsigned* status) {
+  memset(out_psum, 0, sizeof(float) * M);
+  return (int)more::launch_train_stats(route_args(X, R1, R2, N, h, r, M, 1, nullptr, nullptr, nullptr, nullptr,
+                                                  status),
+                                       out_m, out_Z, out_psum);
+}
+
+extern "C" long emu_dispatch_scratch_bytes(int64_t S, int M) { return (long)more::dispatch_scratch_bytes(S, M); }
+
+extern "C" int emu_dispatch(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted, void* scratch,
+                            unsigned* status) {
+  return (int)more::launch_dispatch(idx, S, M, offsets, sorted, scratch, status, nullptr);
 }

@@ -35,6 +35,7 @@ long progress = 0;
 std::vector<Barrier> cta_bar, warp_bar;
 Barrier cl_bar;
 std::vector<uint64_t> xbuf;
+std::vector<std::map<int, std::vector<float4>>> statics;  // per CTA: static shared declarations
 std::function<void()>* body_ptr = nullptr;
 std::vector<std::vector<float4>> bufs;
 size_t smem_size = 0;
@@ -88,6 +89,25 @@ uint64_t xchg(uint64_t bits, int src, bool xor_mode) {
   return r;
 }
 float4* smem() { return bufs[fibers[cur].cta].data(); }
+void* shared_static_bytes(int id, size_t bytes) {
+  std::vector<float4>& v = statics[fibers[cur].cta][id];
+  const size_t n = (bytes + sizeof(float4) - 1) / sizeof(float4);
+  if (v.size() != n) {
+    v.assign(n, float4());
+    memset(v.data(), 0xFF, n * sizeof(float4));  // NaN: unwritten reads show up
+  }
+  return v.data();
+}
+unsigned match_any(unsigned long long v) {
+  const int me = cur;
+  xbuf[me] = v;
+  (void)wait_on(warp_bar[me / 32], 32, 0);
+  unsigned mask = 0;
+  for (int l = 0; l < 32; ++l)
+    if (xbuf[(me & ~31) | l] == v) mask |= 1u << l;
+  (void)wait_on(warp_bar[me / 32], 32, 0);
+  return mask;
+}
 
 void launch(dim3 grid, dim3 block, size_t smem_bytes, std::function<void()> body) {
   per_cta = (int)(block.x * block.y * block.z);
@@ -121,6 +141,7 @@ void launch(dim3 grid, dim3 block, size_t smem_bytes, std::function<void()> body
         warp_bar.assign(n / 32, Barrier());
         cl_bar = Barrier();
         xbuf.assign(n, 0);
+        statics.assign(cs, {});
         body_ptr = &body;
         for (int i = 0; i < n; ++i) {
           Fiber& f = fibers[i];

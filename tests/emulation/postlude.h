@@ -4,3 +4,4 @@
 #define cudaMemsetAsync(p, v, n, s) (memset((p), (v), (n)), cudaSuccess)
 #define cudaGetLastError() cudaSuccess
 #define cudaGetDevice(p) (*(p) = 0, cudaSuccess)
+#define cudaDeviceGetAttribute(p, attr, dev) (*(p) = 148, cudaSuccess)

@@ -29,6 +29,9 @@ template <class T> T shfl(unsigned, T v, int src) {
   uint64_t b = 0; memcpy(&b, &v, sizeof(T)); b = xchg(b, src, false); T r; memcpy(&r, &b, sizeof(T)); return r;
 }
 float4* smem();
+void* shared_static_bytes(int id, size_t bytes);
+template <class T> T& shared_static(int id) { return *static_cast<T*>(shared_static_bytes(id, sizeof(T))); }
+unsigned match_any(unsigned long long v);
 void launch(dim3 grid, dim3 block, size_t smem_bytes, std::function<void()> body);
 }
 namespace cooperative_groups {
@@ -49,6 +52,9 @@ inline cluster_group this_cluster() { return {}; }
 #define __shfl_xor_sync(m, v, l) ::emu::shfl_xor(m, v, l)
 #define __shfl_sync(m, v, l) ::emu::shfl(m, v, l)
 #define __ldg(p) (*(p))
+#define __ldcs(p) (*(p))
+#define __popc(x) __builtin_popcount(x)
+#define __match_any_sync(m, v) ::emu::match_any((unsigned long long)(long long)(v))
 inline unsigned atomicOr(unsigned* p, unsigned v) { unsigned o = *p; *p |= v; return o; }
 inline int atomicAdd(int* p, int v) { int o = *p; *p += v; return o; }
 inline float atomicAdd(float* p, float v) { float o = *p; *p += v; return o; }

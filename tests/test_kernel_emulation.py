@@ -1,14 +1,15 @@
-"""The CUDA-core kernels of the backward and of the cluster routing variant, run on the CPU under
-the test-only thread emulation (tests/emulation), against the fp64 oracle.
+"""The library's CUDA-core kernels run on the CPU under the test-only thread emulation
+(tests/emulation), against the fp64 oracle.
 
-The sources are the library's own (``csrc/backward.cu``, ``csrc/route_cluster.cu``), compiled
-with g++; each CTA's threads, or each cluster's, run as fibers.  Checks, with the tolerances of
-the GPU tests:
+The sources are the library's own, compiled with g++: backward, cluster and small-N routing,
+training statistics, dispatch, and the unfused path.  Each CTA's threads, or each cluster's, run
+as fibers.  Checks, with the tolerances of the GPU tests:
 - the backward's gradients ("MoRE: Scaling mixture of experts with hardware-aware low-rank
   routing", App. F, Algorithm 3) within 2e-3 of the magnitude bound S
   (tests/test_gpu_training_backward.py);
-- the cluster variant's routing (App. F, Algorithm 1, Fig. 12) by the parity rules
-  (tests/parity.py).
+- routing (App. F, Algorithm 1, Fig. 12) by the parity rules (tests/parity.py);
+- the training statistics (Algorithm 2) within the bounds of tests/test_gpu_train_stats.py;
+- dispatch (Fig. 9) bit-exact.
 Every host array ends against an inaccessible page, and the runtime aborts on a deadlock, a write
 past a CTA's shared memory, or a DSMEM address outside it.  These checks catch the kernels'
 index, barrier and arithmetic mistakes before any GPU runs them; the GPU tests remain the
@@ -126,3 +127,91 @@ def test_planted_kernel_mistake_is_caught(tmp_path, name, old, new):
             X, R1, R2 = syn.router_inputs(13, 256, 32, 512, seed=13)
             cluster(e, X, R1, R2, 13, 256, 32, 512, 8)
     e.free_all()
+
+
+def route_with(e, entry, X, R1, R2, N, h, r, M, k, exact=False):
+    out = [e.empty(N * k * 4), e.empty(N * k * 4), e.empty(M * 4), e.empty(N * k * 4)]
+    status = ctypes.c_uint(0)
+    args = [e.put(X), e.put(R1), e.put(R2), N, h, r, M, k, *out]
+    if entry == "unfused":
+        args.append(e.empty(e.lib.emu_unfused_scratch_bytes(N, r, M)))
+    fn = e.lib.emu_route_unfused if entry == "unfused" else e.lib.emu_route_small
+    assert fn(*args, ctypes.addressof(status)) == 0
+    idx, gate = e.get(out[0], (N, k), np.int32), e.get(out[1], (N, k), np.float32)
+    cnt, logits = e.get(out[2], (M,), np.int32), e.get(out[3], (N, k), np.float32)
+    e.free_all()
+    assert status.value == 0
+    return parity.compare(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, exact=exact)
+
+
+@pytest.mark.parametrize("entry", ["small_n", "unfused"])
+@pytest.mark.parametrize("N,h,r,M,k", [(7, 2048, 32, 4096, 8), (33, 136, 48, 64, 8), (20, 72, 16, 200, 1),
+                                       (9, 256, 64, 16, 16)])
+def test_routing_kernels_match_oracle(emu, entry, N, h, r, M, k):
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=N)
+    route_with(emu, entry, X, R1, R2, N, h, r, M, k)
+
+
+@pytest.mark.parametrize("entry", ["small_n", "unfused"])
+def test_routing_kernels_tie_heavy_exact(emu, entry):
+    M, N, k = 64, 60, 8
+    X = syn.f32_to_bf16_bits(np.random.default_rng(9).integers(-3, 4, size=(N, M)).astype(np.float32))
+    eye = syn.f32_to_bf16_bits(np.eye(M, dtype=np.float32))
+    route_with(emu, entry, X, eye, eye, N, M, M, M, k, exact=True)
+
+
+@pytest.mark.parametrize("N,h,r,M", [(23, 128, 32, 192), (6, 512, 16, 1000), (1, 64, 128, 64)])
+def test_train_stats_kernel_matches_oracle(emu, N, h, r, M):
+    e = emu
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=N + 1)
+    pm, pz, pp = e.empty(N * 4), e.empty(N * 4), e.empty(M * 4)
+    status = ctypes.c_uint(0)
+    assert e.lib.emu_train_stats(e.put(X), e.put(R1), e.put(R2), N, h, r, M, pm, pz, pp,
+                                 ctypes.addressof(status)) == 0
+    gm, gz, gp = e.get(pm, (N,), np.float32), e.get(pz, (N,), np.float32), e.get(pp, (M,), np.float32)
+    e.free_all()
+    o = oracle.train_stats(X, R1, R2, N, h, r, M)
+    tol = parity.LOGIT_TOL * oracle.route(X, R1, R2, N, h, r, M, 1).rms
+    assert np.all(np.abs(gm - o.m) <= tol)
+    assert np.all(np.abs(np.log(gz.astype(np.float64)) - np.log(o.Z)) <= 2 * tol + 1e-5)
+    assert np.all(np.abs(gp - o.psum) / o.psum <= 4 * tol.max() + 1e-5)
+
+
+@pytest.mark.parametrize("N,k,M,seed", [(1, 1, 8, 0), (37, 3, 16, 1), (3000, 8, 1000, 2), (700, 4, 4096, 3)])
+def test_dispatch_kernels_match_oracle(emu, N, k, M, seed):
+    e = emu
+    idx = np.random.default_rng(seed).integers(0, M, size=(N, k)).astype(np.int32)
+    S = N * k
+    off, srt = e.empty((M + 1) * 4), e.empty(S * 4)
+    status = ctypes.c_uint(0)
+    assert e.lib.emu_dispatch(e.put(idx), S, M, off, srt, e.empty(e.lib.emu_dispatch_scratch_bytes(S, M)),
+                              ctypes.addressof(status)) == 0
+    got_off, got_srt = e.get(off, (M + 1,), np.int32), e.get(srt, (S,), np.int32)
+    e.free_all()
+    o = oracle.dispatch(idx, M)
+    np.testing.assert_array_equal(got_off, o.offsets)
+    np.testing.assert_array_equal(got_srt, o.sorted)
+    assert status.value == 0
+
+
+def test_dispatch_kernels_skip_out_of_range(emu):
+    e = emu
+    M = 16
+    idx = np.random.default_rng(4).integers(0, M, size=(50, 4)).astype(np.int32)
+    bad = idx.copy()
+    bad[::7, 1] = M + 3
+    bad[::11, 2] = -1
+    S = bad.size
+    off, srt = e.empty((M + 1) * 4), e.empty(S * 4)
+    status = ctypes.c_uint(0)
+    assert e.lib.emu_dispatch(e.put(bad), S, M, off, srt, e.empty(e.lib.emu_dispatch_scratch_bytes(S, M)),
+                              ctypes.addressof(status)) == 0
+    got_off = e.get(off, (M + 1,), np.int32)
+    ok = (bad >= 0) & (bad < M)
+    expect = np.concatenate([[0], np.cumsum(np.bincount(bad[ok], minlength=M))])
+    np.testing.assert_array_equal(got_off, expect)
+    valid_slots = np.flatnonzero(ok.ravel())
+    got_srt = e.get(srt, (S,), np.int32)[: got_off[M]]
+    e.free_all()
+    np.testing.assert_array_equal(np.sort(got_srt), valid_slots)
+    assert status.value == 4  # MORE_DEVERR_BAD_INPUT
