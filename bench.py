@@ -8,7 +8,7 @@ workload: prefill, N = 262,144 tokens (256 sequences x 1024), h = 2048, M = 4096
 r = 32, k = 8, X rows at unit RMS, R1 ~ N(0, 1/h), R2 ~ N(0, 1/r), seed 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--variant auto|fused_tc|small_n|cluster|unfused|train|dispatch|backward]
+                  [--variant auto|fused_tc|small_n|cluster|unfused|train|dispatch|dispatch_shared|backward]
                   [--workload NAME]
 
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank routes its own
@@ -253,9 +253,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto",
-                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "train", "dispatch", "backward"],
+                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "train", "dispatch", "dispatch_shared",
+                             "backward"],
                     help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum); "
-                         "dispatch: routing followed by more_dispatch of its indices; "
+                         "dispatch: routing followed by more_dispatch of its indices (dispatch_shared: with the "
+                         "shared-memory dispatch kernels); "
                          "backward: more_route_backward (Algorithm 3) given the forward's selections, m and Z")
     ap.add_argument("--workload", default="prefill_r32", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample size, in CPU seconds")
@@ -306,7 +308,7 @@ def main():
         m_buf = torch.empty((N,), dtype=torch.float32, device="cuda")
         z_buf = torch.empty((N,), dtype=torch.float32, device="cuda")
         psum_buf = torch.empty((M,), dtype=torch.float32, device="cuda")
-    if args.variant == "dispatch":
+    if args.variant in ("dispatch", "dispatch_shared"):
         d_scratch = torch.empty(max(more.dispatch_scratch_bytes(N, k, M), 16), dtype=torch.uint8, device="cuda")
         d_off = torch.empty((M + 1,), dtype=torch.int32, device="cuda")
         d_sorted = torch.empty((N * k,), dtype=torch.int32, device="cuda")
@@ -333,9 +335,10 @@ def main():
         if args.variant == "train":
             more.route_train(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
                              out_m=m_buf, out_Z=z_buf, out_psum=psum_buf, stream=st)
-        elif args.variant == "dispatch":
+        elif args.variant in ("dispatch", "dispatch_shared"):
             more.route(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits, stream=st)
-            more.dispatch(idx, M, scratch=d_scratch, out_offsets=d_off, out_sorted=d_sorted, stream=st)
+            more.dispatch(idx, M, scratch=d_scratch, out_offsets=d_off, out_sorted=d_sorted,
+                          variant="shared" if args.variant == "dispatch_shared" else "auto", stream=st)
         elif args.variant == "backward":
             more.route_backward(X, R1, R2, k, top_idx=idx, top_vals_bar=b_tvb, pbar=b_pbar, m=b_m, Z=b_Z,
                                 scratch=b_scratch, out_Xbar=b_out[0], out_R1bar=b_out[1], out_R2bar=b_out[2],
@@ -355,7 +358,8 @@ def main():
         except more.MoreError:
             variant_used = "small_n"
         variant_used = variant_used if N >= 512 else "small_n"
-    launches_per_step = {"unfused": 3, "train": 2, "dispatch": 5, "backward": 5}.get(args.variant, 1)
+    launches_per_step = {"unfused": 3, "train": 2, "dispatch": 5, "dispatch_shared": 5,
+                         "backward": 5}.get(args.variant, 1)
 
     def barrier():
         if dist is not None:

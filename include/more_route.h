@@ -195,6 +195,24 @@ more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* 
                           int32_t* out_sorted, void* scratch, size_t scratch_bytes, void* stream);
 
 /*
+ * more_dispatch with an explicit kernel variant; same arguments, scratch and result.
+ *   MORE_DISPATCH_GLOBAL: histograms of 2048-slot chunks in global memory (as more_dispatch);
+ *   MORE_DISPATCH_SHARED: about two chunks per SM, each counted in a shared-memory histogram of
+ *     M counters; requires M <= MORE_DISPATCH_SHARED_MMAX (else MORE_ERR_UNSUPPORTED).
+ *   MORE_DISPATCH_AUTO:   the variant more_dispatch uses (GLOBAL).
+ * Any other value returns MORE_ERR_INVALID_ARG.
+ */
+#define MORE_DISPATCH_SHARED_MMAX 32768
+typedef enum more_dispatch_kernel {
+  MORE_DISPATCH_AUTO = 0,
+  MORE_DISPATCH_GLOBAL = 1,
+  MORE_DISPATCH_SHARED = 2
+} more_dispatch_kernel;
+more_status more_dispatch_variant(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
+                                  int32_t* out_sorted, void* scratch, size_t scratch_bytes, int variant,
+                                  void* stream);
+
+/*
  * Backward of the router ("MoRE", App. F, F.2.2, Algorithm 3 and eqs. (10)-(12)), with z
  * recomputed from X (activation recompute), in fp32 on the CUDA cores.  With z = X R1,
  * l = z R2 (fp32) and P_ni = exp(l_ni - saved_m[n]) / saved_Z[n]:

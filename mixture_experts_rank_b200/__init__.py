@@ -27,6 +27,7 @@ __all__ = ["route", "route_train", "route_backward", "route_backward_scratch_byt
 KMAX = 16
 STATS_MMAX = 32768
 VARIANTS = {"auto": 0, "fused_tc": 1, "small_n": 2, "cluster": 3}
+DISPATCH_VARIANTS = {"auto": 0, "global": 1, "shared": 2}
 STATUS = {0: "MORE_OK", 1: "MORE_ERR_INVALID_ARG", 2: "MORE_ERR_UNSUPPORTED", 3: "MORE_ERR_CUDA",
           4: "MORE_ERR_DEVICE"}
 
@@ -54,6 +55,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_dispatch_scratch_bytes.argtypes = [I64, I, I]
     lib.more_dispatch.restype = I
     lib.more_dispatch.argtypes = [P, I64, I, I, P, P, P, ctypes.c_size_t, P]
+    lib.more_dispatch_variant.restype = I
+    lib.more_dispatch_variant.argtypes = [P, I64, I, I, P, P, P, ctypes.c_size_t, I, P]
     lib.more_route_train.restype = I
     lib.more_route_train.argtypes = route_args + [P, P, P, P]
     lib.more_route_backward_scratch_bytes.restype = ctypes.c_size_t
@@ -231,7 +234,7 @@ def dispatch_scratch_bytes(N: int, k: int, M: int) -> int:
 
 
 def dispatch(idx: torch.Tensor, M: int, *, scratch: torch.Tensor | None = None, out_offsets=None,
-             out_sorted=None, stream=None):
+             out_sorted=None, variant: str = "auto", stream=None):
     """Dispatch bookkeeping for routing indices ``idx`` (int32 [N, k], CUDA): returns
     ``(offsets int32 [M + 1], sorted int32 [N k])``; expert e owns ``sorted[offsets[e]:offsets[e+1]]``,
     the flat slots n k + j naming it, in increasing order."""
@@ -244,8 +247,8 @@ def dispatch(idx: torch.Tensor, M: int, *, scratch: torch.Tensor | None = None, 
         out_offsets = torch.empty((M + 1,), dtype=torch.int32, device=idx.device)
     if out_sorted is None:
         out_sorted = torch.empty((N * k,), dtype=torch.int32, device=idx.device)
-    st = _lib.more_dispatch(_ptr(idx), N, k, M, _ptr(out_offsets), _ptr(out_sorted), _ptr(scratch),
-                            scratch.numel(), _stream_handle(stream))
+    st = _lib.more_dispatch_variant(_ptr(idx), N, k, M, _ptr(out_offsets), _ptr(out_sorted), _ptr(scratch),
+                                    scratch.numel(), DISPATCH_VARIANTS[variant], _stream_handle(stream))
     _check(st, "more_dispatch")
     return out_offsets, out_sorted
 

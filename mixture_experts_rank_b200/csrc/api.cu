@@ -150,20 +150,30 @@ size_t more_dispatch_scratch_bytes(int64_t N, int k, int M) {
   return (size_t)dispatch_scratch_bytes(N * (int64_t)k, M);
 }
 
-more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
-                          int32_t* out_sorted, void* scratch, size_t scratch_bytes, void* stream) {
+more_status more_dispatch_variant(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
+                                  int32_t* out_sorted, void* scratch, size_t scratch_bytes, int variant,
+                                  void* stream) {
   if (N < 0 || k < 1 || M < 1 || !out_offsets || !aligned16(out_offsets)) return MORE_ERR_INVALID_ARG;
+  if (variant < MORE_DISPATCH_AUTO || variant > MORE_DISPATCH_SHARED) return MORE_ERR_INVALID_ARG;
   if (k > MORE_KMAX || M > MORE_MMAX || N * (int64_t)k > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
+  if (variant == MORE_DISPATCH_SHARED && !dispatch_shared_supports(M)) return MORE_ERR_UNSUPPORTED;
   const int64_t S = N * (int64_t)k;
   if (S > 0 && (!idx || !out_sorted || !scratch || !aligned16(idx) || !aligned16(out_sorted) ||
                 !aligned16(scratch) || scratch_bytes < (size_t)dispatch_scratch_bytes(S, M)))
     return MORE_ERR_INVALID_ARG;
   unsigned int* status = status_word();
   if (!status) return MORE_ERR_CUDA;
-  return launch_dispatch(idx, S, M, out_offsets, out_sorted, scratch, status,
-                         static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MORE_OK
-             : MORE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t err = variant == MORE_DISPATCH_SHARED
+                              ? launch_dispatch_shared(idx, S, M, out_offsets, out_sorted, scratch, status, s)
+                              : launch_dispatch(idx, S, M, out_offsets, out_sorted, scratch, status, s);
+  return err == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
+more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* out_offsets,
+                          int32_t* out_sorted, void* scratch, size_t scratch_bytes, void* stream) {
+  return more_dispatch_variant(idx, N, k, M, out_offsets, out_sorted, scratch, scratch_bytes, MORE_DISPATCH_AUTO,
+                               stream);
 }
 
 size_t more_route_backward_scratch_bytes(int64_t N, int h, int r, int M) {

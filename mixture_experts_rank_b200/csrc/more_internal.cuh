@@ -29,6 +29,9 @@ cudaError_t launch_cluster(const RouteArgs& a);
 int64_t dispatch_scratch_bytes(int64_t S, int M);
 cudaError_t launch_dispatch(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted,
                             void* scratch, unsigned int* status, cudaStream_t stream);
+bool dispatch_shared_supports(int M);
+cudaError_t launch_dispatch_shared(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted,
+                                   void* scratch, unsigned int* status, cudaStream_t stream);
 cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, float* out_psum);
 
 // Arguments of one backward call after validation (pointers as in more_route_backward).

@@ -158,6 +158,8 @@ class Emulated:
         lib.emu_dispatch_scratch_bytes.argtypes = [I64, I]
         lib.emu_dispatch.restype = I
         lib.emu_dispatch.argtypes = [P, I64, I, P, P, P, P]
+        lib.emu_dispatch_shared.restype = I
+        lib.emu_dispatch_shared.argtypes = [P, I64, I, P, P, P, P]
         self._live = []
 
     def put(self, a) -> int | None:

@@ -108,3 +108,8 @@ extern "C" int emu_dispatch(const int32_t* idx, int64_t S, int M, int32_t* offse
                             unsigned* status) {
   return (int)more::launch_dispatch(idx, S, M, offsets, sorted, scratch, status, nullptr);
 }
+
+extern "C" int emu_dispatch_shared(const int32_t* idx, int64_t S, int M, int32_t* offsets, int32_t* sorted,
+                                   void* scratch, unsigned* status) {
+  return (int)more::launch_dispatch_shared(idx, S, M, offsets, sorted, scratch, status, nullptr);
+}

@@ -54,6 +54,7 @@ inline cluster_group this_cluster() { return {}; }
 #define __ldg(p) (*(p))
 #define __ldcs(p) (*(p))
 #define __popc(x) __builtin_popcount(x)
+#define __ffs(x) __builtin_ffs(x)
 #define __match_any_sync(m, v) ::emu::match_any((unsigned long long)(long long)(v))
 inline unsigned atomicOr(unsigned* p, unsigned v) { unsigned o = *p; *p |= v; return o; }
 inline int atomicAdd(int* p, int v) { int o = *p; *p += v; return o; }

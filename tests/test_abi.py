@@ -160,3 +160,11 @@ def test_backward_scratch_size():
     assert m.route_backward_scratch_bytes(0, 64, 32, 64) >= 0
     assert m.route_backward_scratch_bytes(-1, 64, 32, 64) == 0
     assert m.route_backward_scratch_bytes(10, 64, 144, 64) == 0
+
+
+@pytest.mark.parametrize("variant,M,expected", [(3, 64, 1), (-1, 64, 1), (2, 32776, 2), (1, 262152, 2)])
+def test_dispatch_variant_rejects_invalid_arguments(lib, variant, M, expected):
+    P = ctypes.c_void_p
+    need = lib.more_dispatch_scratch_bytes(100, 4, min(M, 262144))
+    st = lib.more_dispatch_variant(P(16), 100, 4, M, P(16), P(16), P(16), need, variant, None)
+    assert st == expected

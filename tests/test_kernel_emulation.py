@@ -177,15 +177,18 @@ def test_train_stats_kernel_matches_oracle(emu, N, h, r, M):
     assert np.all(np.abs(gp - o.psum) / o.psum <= 4 * tol.max() + 1e-5)
 
 
-@pytest.mark.parametrize("N,k,M,seed", [(1, 1, 8, 0), (37, 3, 16, 1), (3000, 8, 1000, 2), (700, 4, 4096, 3)])
-def test_dispatch_kernels_match_oracle(emu, N, k, M, seed):
+@pytest.mark.parametrize("variant", ["global", "shared"])
+@pytest.mark.parametrize("N,k,M,seed", [(1, 1, 8, 0), (37, 3, 16, 1), (3000, 8, 1000, 2), (700, 4, 4096, 3),
+                                        (9000, 8, 64, 5)])
+def test_dispatch_kernels_match_oracle(emu, variant, N, k, M, seed):
     e = emu
     idx = np.random.default_rng(seed).integers(0, M, size=(N, k)).astype(np.int32)
     S = N * k
     off, srt = e.empty((M + 1) * 4), e.empty(S * 4)
     status = ctypes.c_uint(0)
-    assert e.lib.emu_dispatch(e.put(idx), S, M, off, srt, e.empty(e.lib.emu_dispatch_scratch_bytes(S, M)),
-                              ctypes.addressof(status)) == 0
+    fn = e.lib.emu_dispatch_shared if variant == "shared" else e.lib.emu_dispatch
+    assert fn(e.put(idx), S, M, off, srt, e.empty(e.lib.emu_dispatch_scratch_bytes(S, M)),
+              ctypes.addressof(status)) == 0
     got_off, got_srt = e.get(off, (M + 1,), np.int32), e.get(srt, (S,), np.int32)
     e.free_all()
     o = oracle.dispatch(idx, M)
@@ -194,7 +197,8 @@ def test_dispatch_kernels_match_oracle(emu, N, k, M, seed):
     assert status.value == 0
 
 
-def test_dispatch_kernels_skip_out_of_range(emu):
+@pytest.mark.parametrize("variant", ["global", "shared"])
+def test_dispatch_kernels_skip_out_of_range(emu, variant):
     e = emu
     M = 16
     idx = np.random.default_rng(4).integers(0, M, size=(50, 4)).astype(np.int32)
@@ -204,8 +208,9 @@ def test_dispatch_kernels_skip_out_of_range(emu):
     S = bad.size
     off, srt = e.empty((M + 1) * 4), e.empty(S * 4)
     status = ctypes.c_uint(0)
-    assert e.lib.emu_dispatch(e.put(bad), S, M, off, srt, e.empty(e.lib.emu_dispatch_scratch_bytes(S, M)),
-                              ctypes.addressof(status)) == 0
+    fn = e.lib.emu_dispatch_shared if variant == "shared" else e.lib.emu_dispatch
+    assert fn(e.put(bad), S, M, off, srt, e.empty(e.lib.emu_dispatch_scratch_bytes(S, M)),
+              ctypes.addressof(status)) == 0
     got_off = e.get(off, (M + 1,), np.int32)
     ok = (bad >= 0) & (bad < M)
     expect = np.concatenate([[0], np.cumsum(np.bincount(bad[ok], minlength=M))])
