@@ -197,6 +197,11 @@ def test_dispatch_kernels_match_oracle(emu, variant, N, k, M, seed):
     assert status.value == 0
 
 
+def test_shared_dispatch_at_its_chunk_cap(emu):
+    """700,000 slots: the shared-memory variant's full 296 chunks, several batches each."""
+    test_dispatch_kernels_match_oracle(emu, "shared", 87500, 8, 4096, 11)
+
+
 @pytest.mark.parametrize("variant", ["global", "shared"])
 def test_dispatch_kernels_skip_out_of_range(emu, variant):
     e = emu
