@@ -1,4 +1,4 @@
-// CUDA-core building blocks shared by the small-N kernel and the unfused path.
+// CUDA-core building blocks shared by the small-N and cluster kernels and the unfused path.
 #pragma once
 #include "more_internal.cuh"
 
