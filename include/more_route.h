@@ -125,7 +125,10 @@ more_status more_route_unfused(const void* X, const void* R1, const void* R2, in
  *     on every device that loads it, whether or not this call is used.
  *   - The first call on a device looks up the array's device address (one
  *     cudaGetSymbolAddress with that device current); make that first call
- *     before starting any stream capture.
+ *     before starting any stream capture.  The address is kept for the life of
+ *     the process: after a cudaDeviceReset of that device (which discards the
+ *     library's module and the array with it) this entry point must not be
+ *     called again in the same process.
  *   - All calls share the array and it keeps the last call's contents (every
  *     call overwrites the part it reads).  Calls that may overlap on the GPU
  *     (different streams, or different host threads without ordering) race on

@@ -27,20 +27,6 @@ unsigned int* status_word() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-more_status validate(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
-                     int k, const int32_t* out_idx, const float* out_gate,
-                     const int32_t* out_count, const float* out_logits) {
-  if (N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1)
-    return MORE_ERR_INVALID_ARG;
-  if (!R1 || !R2 || !out_count || (N > 0 && (!X || !out_idx || !out_gate))) return MORE_ERR_INVALID_ARG;
-  if ((X && !aligned16(X)) || !aligned16(R1) || !aligned16(R2) || (out_idx && !aligned16(out_idx)) ||
-      (out_gate && !aligned16(out_gate)) || !aligned16(out_count) || (out_logits && !aligned16(out_logits)))
-    return MORE_ERR_INVALID_ARG;
-  if (N > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
-  if (k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX) return MORE_ERR_UNSUPPORTED;
-  return MORE_OK;
-}
-
 RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
                     int k, int32_t* out_idx, float* out_gate, int32_t* out_count,
                     float* out_logits, void* stream) {
@@ -67,6 +53,22 @@ RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, in
 constexpr int64_t kSmallNThreshold = 512;
 
 }  // namespace
+
+// Argument checks shared by every routing entry point (see more_route.h).
+more_status validate_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                           const int32_t* out_idx, const float* out_gate, const int32_t* out_count,
+                           const float* out_logits) {
+  if (N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1)
+    return MORE_ERR_INVALID_ARG;
+  if (!R1 || !R2 || !out_count || (N > 0 && (!X || !out_idx || !out_gate))) return MORE_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || !aligned16(R1) || !aligned16(R2) || (out_idx && !aligned16(out_idx)) ||
+      (out_gate && !aligned16(out_gate)) || !aligned16(out_count) || (out_logits && !aligned16(out_logits)))
+    return MORE_ERR_INVALID_ARG;
+  if (N > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
+  if (k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX) return MORE_ERR_UNSUPPORTED;
+  return MORE_OK;
+}
+
 }  // namespace more
 
 using namespace more;
@@ -95,7 +97,7 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
                                int M, int k, int32_t* out_idx, float* out_gate,
                                int32_t* out_expert_count, float* out_logits, int variant,
                                void* stream) {
-  more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  more_status st = validate_route(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
   if (st != MORE_OK) return st;
   if (variant < MORE_VARIANT_AUTO || variant > MORE_VARIANT_CLUSTER) return MORE_ERR_INVALID_ARG;
   RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
@@ -130,7 +132,7 @@ more_status more_route(const void* X, const void* R1, const void* R2, int64_t N,
 more_status more_route_train(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
                              int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
                              float* out_logits, float* out_m, float* out_Z, float* out_psum, void* stream) {
-  more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  more_status st = validate_route(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
   if (st != MORE_OK) return st;
   if (!out_psum || !aligned16(out_psum) || (N > 0 && (!out_m || !out_Z)) || (out_m && !aligned16(out_m)) ||
       (out_Z && !aligned16(out_Z)))
@@ -231,7 +233,7 @@ more_status more_route_unfused(const void* X, const void* R1, const void* R2, in
                                int M, int k, int32_t* out_idx, float* out_gate,
                                int32_t* out_expert_count, float* out_logits, void* scratch,
                                size_t scratch_bytes, void* stream) {
-  more_status st = validate(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  more_status st = validate_route(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
   if (st != MORE_OK) return st;
   if (N > 0 && (!scratch || !aligned16(scratch) || scratch_bytes < unfused_scratch_bytes(N, r, M)))
     return MORE_ERR_INVALID_ARG;

@@ -19,6 +19,8 @@
 // row and column against the array's extent; shared-memory tiles are zero-padded.
 #include <algorithm>
 
+#include <atomic>
+
 #include "more_internal.cuh"
 
 namespace more {
@@ -474,11 +476,11 @@ cudaError_t launch_rp(BwdArgs a, cudaStream_t stream) {
   const size_t r2_bytes = sizeof(float) * T::kR2Floats;
   const size_t r1_bytes = sizeof(float) * T::kR1Floats;
   // shared-memory limits, set once per device (a call captured into a CUDA graph then only launches)
-  static int configured[64] = {};
+  static std::atomic<int> configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
+  if (dev < 0 || dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
     if ((e = cudaFuncSetAttribute(bwd_token_block_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)tok_bytes)) != cudaSuccess)
       return e;
@@ -488,7 +490,7 @@ cudaError_t launch_rp(BwdArgs a, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(bwd_r1_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)r1_bytes)) != cudaSuccess)
       return e;
-    if (dev >= 0 && dev < 64) configured[dev] = 1;
+    if (dev >= 0 && dev < 64) configured[dev].store(1, std::memory_order_release);
   }
   const unsigned blocks = (unsigned)ceil_div(a.N, kBN);
   bwd_token_block_kernel<RP><<<blocks, kThreads, tok_bytes, stream>>>(a);

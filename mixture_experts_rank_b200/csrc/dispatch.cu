@@ -22,6 +22,8 @@
 //      (one barrier each), so every expert's slots still land in slot order.
 #include <algorithm>
 
+#include <atomic>
+
 #include "more_internal.cuh"
 
 namespace more {
@@ -233,19 +235,19 @@ cudaError_t launch_dispatch_shared(const int32_t* idx, int64_t S, int M, int32_t
                                    void* scratch, unsigned int* status, cudaStream_t stream) {
   if (S == 0) return cudaMemsetAsync(offsets, 0, sizeof(int32_t) * ((size_t)M + 1), stream);
   if (M > kSharedMMax) return cudaErrorInvalidValue;
-  static int configured[64] = {};
+  static std::atomic<int> configured[64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(int32_t) * kSharedMMax;
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
+  if (dev < 0 || dev >= 64 || !configured[dev].load(std::memory_order_acquire)) {
     if ((err = cudaFuncSetAttribute(dsh_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return err;
     if ((err = cudaFuncSetAttribute(dsh_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return err;
-    if (dev >= 0 && dev < 64) configured[dev] = 1;
+    if (dev >= 0 && dev < 64) configured[dev].store(1, std::memory_order_release);
   }
   const int64_t C = shared_chunk_count(S);
   int32_t* G = static_cast<int32_t*>(scratch);  // C x M, every entry written by the histogram kernel

@@ -23,6 +23,11 @@ struct RouteArgs {
   cudaStream_t stream;
 };
 
+// Argument checks of the routing entry points (more_route.h): MORE_OK or the error to return.
+more_status validate_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
+                           const int32_t* out_idx, const float* out_gate, const int32_t* out_count,
+                           const float* out_logits);
+
 // Launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_small_n(const RouteArgs& a);
 cudaError_t launch_cluster(const RouteArgs& a);

@@ -16,6 +16,8 @@
 //   3. k warp-wide arg-max rounds merge each warp's lanes, then warp 0 merges the
 //      sixteen warp lists in routing order, applies the softmax and writes the outputs
 //      and one atomic count per selection.
+#include <atomic>
+
 #include "more_internal.cuh"
 #include "warp_simt.cuh"
 
@@ -297,12 +299,12 @@ cudaError_t launch_train_stats(const RouteArgs& a, float* out_m, float* out_Z, f
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = sizeof(float) * (size_t)a.M;
-  static int configured[64] = {};
-  if (dev >= 0 && dev < 64 && !configured[dev]) {
+  static std::atomic<int> configured[64] = {};
+  if (dev >= 0 && dev < 64 && !configured[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(train_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(sizeof(float) * MORE_STATS_MMAX));
     if (e != cudaSuccess) return e;
-    configured[dev] = 1;
+    configured[dev].store(1, std::memory_order_release);
   }
   // tokens are independent; a CTA keeps its column sums over its tokens (one CTA per SM fits)
   int64_t blocks = (a.N + kStatTokens - 1) / kStatTokens;

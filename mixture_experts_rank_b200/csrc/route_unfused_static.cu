@@ -13,7 +13,8 @@ namespace {
 // that loads it, and is shared by all calls.
 static __device__ __align__(256) unsigned char g_static_scratch[MORE_STATIC_SCRATCH_BYTES];
 
-// Device address of g_static_scratch on the current device, looked up once per device.
+// Device address of g_static_scratch on the current device, looked up once per device and
+// kept for the life of the process (a device reset invalidates it; see more_route.h).
 void* static_scratch_address(cudaError_t* err) {
   static std::mutex mu;
   static void* addr[64] = {};
@@ -41,8 +42,13 @@ extern "C" more_status more_route_unfused_static(const void* X, const void* R1, 
                                                  int h, int r, int M, int k, int32_t* out_idx,
                                                  float* out_gate, int32_t* out_expert_count,
                                                  float* out_logits, void* stream) {
+  // the arguments are checked first, as more_route_unfused checks them; only a valid
+  // problem that does not fit the fixed scratch is reported as unsupported
+  const more_status st =
+      more::validate_route(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  if (st != MORE_OK) return st;
   if (N > 0 && more_route_unfused_scratch_bytes(N, r, M) > (size_t)MORE_STATIC_SCRATCH_BYTES)
-    return MORE_ERR_UNSUPPORTED;  // the problem does not fit the fixed scratch
+    return MORE_ERR_UNSUPPORTED;
   cudaError_t err = cudaSuccess;
   void* scratch = more::static_scratch_address(&err);
   if (!scratch) return MORE_ERR_CUDA;

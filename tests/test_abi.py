@@ -168,3 +168,23 @@ def test_dispatch_variant_rejects_invalid_arguments(lib, variant, M, expected):
     need = lib.more_dispatch_scratch_bytes(100, 4, min(M, 262144))
     st = lib.more_dispatch_variant(P(16), 100, 4, M, P(16), P(16), P(16), need, variant, None)
     assert st == expected
+
+
+def test_static_entry_point_checks_arguments_before_its_size_limit(lib):
+    """A call with bad arguments returns MORE_ERR_INVALID_ARG even when the problem would also
+    be too large for the fixed scratch (the arguments are checked first, as for
+    more_route_unfused); a valid but too-large problem is MORE_ERR_UNSUPPORTED only then."""
+    P = ctypes.c_void_p
+    N, h, r, M, k = 1 << 20, 64, 32, 4096, 4           # far beyond the 32 MiB scratch
+    assert lib.more_route_unfused_scratch_bytes(N, r, M) > (32 << 20)
+    # null X
+    assert lib.more_route_unfused_static(None, P(16), P(16), N, h, r, M, k, P(16), P(16), P(16), None,
+                                         None) == 1
+    # h not a multiple of 8, k > M
+    assert lib.more_route_unfused_static(P(16), P(16), P(16), N, 66, r, M, k, P(16), P(16), P(16), None,
+                                         None) == 1
+    assert lib.more_route_unfused_static(P(16), P(16), P(16), N, h, r, 16, 17, P(16), P(16), P(16), None,
+                                         None) == 1
+    # misaligned output
+    assert lib.more_route_unfused_static(P(16), P(16), P(16), N, h, r, M, k, P(20), P(16), P(16), None,
+                                         None) == 1

@@ -64,12 +64,23 @@ def run(variant, Xd, R1d, R2d, k):
     return [None if t is None else t.cpu().numpy() for t in out]
 
 
-def check(variant, N, h, r, M, k, seed=0, unit_rms=False, n_sample=None):
+def check(variant, N, h, r, M, k, seed=0, unit_rms=False, n_sample=None, near_scan=0, near_count=0):
+    """Route on the GPU and compare with the oracle.  With ``n_sample`` the comparison takes
+    that many rows: the first and last rows, three whole 128-token tiles from the middle of
+    the batch, random rows, and the ``near_count`` rows with the smallest oracle margins
+    among ``near_scan`` scanned rows (all N when near_scan >= N)."""
     if not supported(variant, N, h, r, M, k):
         pytest.skip(f"{variant} does not take this shape")
     X, R1, R2, Xd, R1d, R2d = inputs(N, h, r, M, seed, unit_rms)
     idx, gate, cnt, logits = run(variant, Xd, R1d, R2d, k)
-    rows = None if n_sample is None else parity.sample_rows(N, n_sample, seed)
+    rows = None
+    if n_sample is not None:
+        extra = ()
+        if near_count:
+            scan = None if near_scan >= N else np.random.default_rng(seed + 1).choice(N, near_scan, replace=False)
+            extra = parity.near_tie_rows(X, R1, R2, N, h, r, M, k, near_count, scan=scan)
+        tiles = (N // 256, N // 384 + 1, (5 * N) // 768) if N >= 1024 else ()
+        rows = parity.sample_rows(N, n_sample, seed, tiles=tiles, extra=extra)
     return parity.compare(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, rows=rows)
 
 
@@ -84,13 +95,15 @@ def test_tiny_full_oracle(variant):
 @pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
 @pytest.mark.parametrize("M", [1024, 2048, 4096, 8192, 16384])
 def test_expert_sweep_sampled(variant, M):
-    check(variant, 65536, 512, 32, M, 8, n_sample=384)
+    check(variant, 65536, 512, 32, M, 8, n_sample=4096, near_scan=16384, near_count=256)
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("r", [16, 32, 64, 128])
 def test_prefill_sampled(variant, r):
-    check(variant, 262144, 2048, r, 4096, 8, unit_rms=True, n_sample=384)
+    # the headline shape (r = 32) scans every token's margin for the 1024 closest near-ties
+    check(variant, 262144, 2048, r, 4096, 8, unit_rms=True, n_sample=8192,
+          near_scan=262144 if r == 32 else 32768, near_count=1024 if r == 32 else 256)
 
 
 def test_prefill_unfused_sampled():
@@ -99,7 +112,7 @@ def test_prefill_unfused_sampled():
 
 @pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
 def test_many_experts_sampled(variant):
-    check(variant, 32768, 4096, 64, 65536, 8, n_sample=128)
+    check(variant, 32768, 4096, 64, 65536, 8, n_sample=1024, near_scan=4096, near_count=128)
 
 
 @pytest.mark.parametrize("variant", VARIANTS + ["unfused"])

@@ -5,7 +5,7 @@ external allocator or memory budget that forbids raw allocations, or a latency-c
 path where an allocation is not acceptable): it runs the materialise-then-top-k kernels
 on a fixed scratch array inside the library.  Two calls in a row, on different inputs,
 must match more_route_unfused within the parity tolerances.  tests/conftest.py runs
-this file right after the routing parity tests, ahead of the rows built on routing.
+this file after every other GPU test file.
 """
 import ctypes
 
