@@ -8,45 +8,49 @@
 // the (N, k) selection written), Fig. 12 (gates) and eq. (9) (counts).  The N x M
 // logits exist only in TMEM.
 //
-// How (one persistent CTA per SM, 128-token tiles, 20 warps):
-//   warp 0  TMA producer of X (128 x BK bf16, swizzled) and R1 (BK x r) stages.
+// How (one persistent CTA per SM, 128-token tiles, 20 warps, each with one role):
+//   warp 0  TMA producer of the X (128 x BK bf16, swizzled) and R1 (BK x r) stages and of
+//           the R2 tiles (r x 128 experts); R2 stays resident in shared memory when it
+//           fits, else it is streamed from L2 once per sweep.  It polls both rings.
 //   warp 1  MMA issuer for Z = X R1: M=128 tokens, N=r, K=16 steps over h, into a
-//           double-buffered TMEM accumulator (the next tile streams while the
-//           current one is routed, so HBM never waits on the top-k).
-//   warp 2  MMA issuer for the logit tiles: pass 1 D[tok, exp] = z_hi R2 (K = r),
-//           pass 2 D^T[exp, tok] = R2^T [z_hi | z_lo]^T (K = 2r, exact to ~16 bits of z).
-//   warp 3  TMA producer of R2 tiles (r x 128 experts); R2 stays resident in
-//           shared memory when it fits, else it is streamed from L2.
-//   warps 4-19  four consumer warpgroups (TMEM lanes = tokens in pass 1, experts
-//           in pass 2; warpgroup g takes lane group warp % 4):
+//           double-buffered TMEM accumulator (the next tiles stream while the
+//           current ones are routed, so HBM never waits on the top-k).
+//   warp 2  MMA issuer of pass A: D[tok, exp] = z_hi R2 (K = r), 128 experts a job.
+//   warp 3  MMA issuer of pass B: D^T[exp, tok] = R2^T [z_hi | z_lo]^T (K = 2r, exact
+//           to ~16 bits of z), 128 experts a job.
+//   warps 4-11   group A (two warps per TMEM lane group): per tile
 //     epilogue  Z from TMEM -> (z_hi, z_lo) bf16 pair -> shared memory (K-major),
-//               plus |z_hi|, |z_lo| per token and the largest column norm of R2.
-//     pass 1    every 32-expert chunk of a token is reduced to the maximum of its
-//               z_hi logits, packed into a 32-bit key (order-preserving value bits
-//               above the chunk id); a branch-free sorted list keeps the best
-//               k + 6 keys per warpgroup.
-//     select    the four lists are merged.  z_hi logits differ from the exact ones
-//               by at most eps (|z_lo| times the largest R2 column norm, plus fp32
+//               plus |z_hi|, |z_lo| per token and (first tile) the largest column norm
+//               of R2.
+//     pass A    every 32-expert chunk of a token is reduced to the maximum of its z_hi
+//               logits, packed into a 32-bit key (order-preserving value bits above the
+//               chunk id); a branch-free sorted list keeps the best k + 6 keys per warp.
+//     select    the two lists of a token are merged.  z_hi logits differ from the exact
+//               ones by at most eps (|z_lo| times the largest R2 column norm, plus fp32
 //               rounding), so the exact k-th logit is at least tlow - eps (tlow: the
-//               k-th chunk maximum) and only chunks whose maximum reaches
-//               tlow - 2 eps can hold a top-k expert.  (token, chunk) pairs are
-//               bucketed by chunk with a counting sort.
-//     pass 2    a tile is worked by two warpgroups (0-1 for even tiles, 2-3 for odd):
-//               the two warps of a lane group split the pairs of their chunk, read
-//               each pair's token column and ballot the experts whose exact logit
-//               reaches tlow - eps (the candidates).
-//     finalize  four threads per token rank its few candidates in routing order
-//               (larger logit, then lower expert) into a shared-memory staging of the
-//               outputs, which the tile writes with coalesced stores; softmax, counts.
-//               A list too short to certify the cut, or more candidates than the
-//               slots hold, sends the token to an exact recomputation on CUDA
-//               cores shared by all sixteen consumer warps.
-// Every consumer warp waits for every logit tile and arrives once on its empty
-// barrier, so no warp can fall two phases behind a buffer (a parity wait cannot tell
-// those apart).  Every barrier wait, the consumers' own barrier included, is bounded
-// (a few seconds); on expiry the kernel records MORE_DEVERR_WAIT_TIMEOUT in the
-// library's device error word and every role unwinds.
+//               k-th chunk maximum) and only chunks whose maximum reaches tlow - 2 eps
+//               can hold a top-k expert.  (token, chunk) pairs are bucketed by chunk
+//               with a counting sort into one of two pair buffers, handed to group B.
+//   warps 12-19  group B (two warps per TMEM lane group): per tile
+//     pass B    the two warps of a lane group split the pairs of their chunk, read each
+//               pair's token column and ballot the experts whose exact logit reaches
+//               tlow - eps (the candidates).
+//     finalize  two threads per token rank its few candidates in routing order (larger
+//               logit, then lower expert) into a shared-memory staging of the outputs,
+//               which the tile writes with coalesced stores; softmax, counts.  A list too
+//               short to certify the cut, or more candidates than the slots hold, sends
+//               the token to an exact recomputation on CUDA cores shared by the group.
+// The logit MMAs run in sweeps over the expert tiles: each sweep streams R2 once and every
+// R2 tile feeds pass B of tile t and pass A of tile t + 1 (with two z buffers; otherwise a
+// sweep carries one pass), so group B works on tile t while group A works on tile t + 1.
+// Every mbarrier wait is bounded (a few seconds); on expiry the kernel records
+// MORE_DEVERR_WAIT_TIMEOUT in the library's device error word and every role unwinds.  A
+// group's select or finalize is entered through a bounded barrier of its eight warps; inside
+// it the warps synchronise with a named barrier and nothing waits on another role, so every
+// warp that enters reaches every named barrier.
 #include <cudaTypedefs.h>
+
+#include <atomic>
 
 #include "more_internal.cuh"
 #include "sm100_ptx.cuh"
@@ -57,13 +61,16 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int kBT = 128;        // tokens per tile (MMA M of Z and pass 1, N of pass 2)
+constexpr int kBT = 128;        // tokens per tile (MMA M of Z and pass A, N of pass B)
 constexpr int kBE = 128;        // experts per logit tile
-constexpr int kThreads = 640;   // 4 role warps + 16 consumer warps
-constexpr int kConsumerThreads = 512;
-constexpr int kConsumerWarps = 16;
-constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass 2
-constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than S candidates
+constexpr int kRoleWarps = 4;
+constexpr int kGroupWarps = 8;  // warps of group A and of group B
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kWarpA0 = kRoleWarps, kWarpB0 = kRoleWarps + kGroupWarps;
+constexpr int kThreads = (kRoleWarps + 2 * kGroupWarps) * 32;  // 640: five warps per SMSP, 96 registers
+constexpr int kNamedBarA = 1, kNamedBarB = 2;                  // bar.sync ids of the groups
+constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass B
+constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than one candidate
 constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -81,16 +88,24 @@ struct Params {
   int x_stages;
   int r2_stages;
   int r2_resident;   // every expert tile stays in shared memory
-  uint32_t off_x, off_r1, off_r2, off_zs, off_lists, off_cand, off_thr, off_flag, off_nq, off_fb, off_pc, off_pairs,
-      off_ccount, off_cbase, off_scan, off_pool, off_poolcnt, off_znorm, off_cnorm, off_bar;
+  int interleave;    // two z buffers: a sweep carries pass B of one tile and pass A of the next
+  uint32_t off_x, off_r1, off_r2, off_zs;
+  // group A only
+  uint32_t off_lists, off_ccount, off_scan, off_znorm, off_cnorm;
+  // handed from group A to group B, two buffers each
+  uint32_t off_pairs, off_cbase, off_flag, off_nq;
+  // group B only
+  uint32_t off_cand, off_pc, off_pool, off_poolcnt, off_fb, off_part;
+  uint32_t off_bar;
 };
 
 template <int R, int KCAP>
 struct Cfg {
-  static constexpr int KL = KCAP + 6;                  // chunk keys kept per token
+  static constexpr int KL = KCAP + 6;                  // chunk keys kept per token and warp
   static constexpr int KLP = (KL + 15) & ~15;          // row stride of the candidate slots and counts
-  static constexpr int S = 1;                          // candidate slots per (token, needed chunk)
   static constexpr int RK = 2 * R;                     // z_hi | z_lo columns of the z buffer
+  // one pair buffer: the (token, chunk) pairs of a tile, later its output staging (3 x 128 x k words)
+  static constexpr uint32_t PAIR_BYTES = kBT * KL * 8 > 3 * kBT * KCAP * 4 ? kBT * KL * 8 : 3 * kBT * KCAP * 4;
   static constexpr int BK = R >= 128 ? 32 : 64;        // hidden elements per X stage
   static constexpr uint32_t X_STAGE = kBT * BK * 2;    // 16 KB (8 KB at BK = 32)
   static constexpr uint32_t X_LAYOUT = BK == 64 ? kSwizzle128B : kSwizzle64B;
@@ -106,27 +121,51 @@ struct Cfg {
   static constexpr uint32_t ZS_BYTES = kBT * RK * 2;   // z pair of 128 tokens, K-major core matrices
   static constexpr uint32_t ZS_SBO = (RK / 8) * 128;   // byte stride of 8-token groups
   static constexpr int ZCOLS = R < 32 ? 32 : R;        // TMEM columns per Z accumulator
-  static constexpr int ND = (512 - 2 * ZCOLS) / 128 < 3 ? (512 - 2 * ZCOLS) / 128 : 3;  // logit tile buffers
-  static constexpr int ZCOL0 = ND * 128;               // first TMEM column of the Z accumulators
+  static constexpr int NBUF = (512 - 2 * ZCOLS) / 128 < 3 ? (512 - 2 * ZCOLS) / 128 : 3;
+  static constexpr int NA = 1;                         // TMEM buffers of pass A jobs
+  static constexpr int NB = NBUF - NA;                 // TMEM buffers of pass B jobs (longer MMAs)
+  static constexpr int ZCOL0 = NBUF * 128;             // first TMEM column of the Z accumulators
   static constexpr uint32_t IDESC_Z = idesc_bf16_f32(128, R, 0, 1);    // A = X (K-major), B = R1 (MN-major)
-  static constexpr uint32_t IDESC_P1 = idesc_bf16_f32(128, 128, 0, 1); // A = z pair, B = R2 tile
-  static constexpr uint32_t IDESC_P2 = idesc_bf16_f32(128, 128, 1, 0); // A = R2 tile^T, B = z pair^T
+  static constexpr uint32_t IDESC_PA = idesc_bf16_f32(128, 128, 0, 1); // A = z pair, B = R2 tile
+  static constexpr uint32_t IDESC_PB = idesc_bf16_f32(128, 128, 1, 0); // A = R2 tile^T, B = z pair^T
+  static_assert(NB >= 1, "TMEM holds at least one buffer per pass");
 };
+
+// Jobs of one sweep over the expert tiles: pass A of local tile ta and pass B of local
+// tile tb (-1: none).  Interleaved: sweep q carries A(q) and B(q - 1), so T tiles take
+// T + 1 sweeps; otherwise sweep 2j carries A(j) and sweep 2j + 1 carries B(j).
+struct Sweep {
+  int ta, tb;
+};
+__host__ __device__ __forceinline__ Sweep sweep_jobs(int q, int T, int interleave) {
+  if (interleave) return Sweep{q < T ? q : -1, q >= 1 ? q - 1 : -1};
+  return (q & 1) ? Sweep{-1, q >> 1} : Sweep{q >> 1, -1};
+}
+__host__ __device__ __forceinline__ int sweep_count(int T, int interleave) {
+  return T == 0 ? 0 : (interleave ? T + 1 : 2 * T);
+}
+// z buffer of local tile j and its use count on that buffer.
+__device__ __forceinline__ int zs_buf(int j, int interleave) { return interleave ? (j & 1) : 0; }
+__device__ __forceinline__ int zs_use(int j, int interleave) { return interleave ? (j >> 1) : j; }
 
 // Barrier block layout (uint64_t slots).
 struct Bars {
-  uint64_t* x_full;
-  uint64_t* x_empty;
-  uint64_t* r2_full;
-  uint64_t* r2_empty;
-  uint64_t* zacc_full;   // [2]
+  uint64_t* x_full;      // [8]
+  uint64_t* x_empty;     // [8]
+  uint64_t* r2_full;     // [64]
+  uint64_t* r2_empty;    // [64]
+  uint64_t* zacc_full;   // [2] Z accumulators
   uint64_t* zacc_empty;  // [2]
-  uint64_t* zsm_full;
-  uint64_t* zsm_empty;
-  uint64_t* d_full;      // [3]
-  uint64_t* d_empty;     // [3]
-  uint64_t* drain;       // [2]
-  uint64_t* cbar;        // consumer-warp barrier (16 arrivals per phase)
+  uint64_t* zsm_full;    // [2] z buffers in shared memory
+  uint64_t* zsm_empty;   // [2]
+  uint64_t* a_full;      // [2] pass A TMEM buffers
+  uint64_t* a_empty;     // [2]
+  uint64_t* b_full;      // [2] pass B TMEM buffers
+  uint64_t* b_empty;     // [2]
+  uint64_t* pairs_full;  // [2] pair buffers (group A -> group B)
+  uint64_t* pairs_empty; // [2]
+  uint64_t* gbar;        // [2] bounded entry barriers of groups A and B
+  uint64_t* drain;       // [3]
   uint32_t* tmem_slot;
   int* abort_flag;
 };
@@ -141,16 +180,21 @@ __device__ __forceinline__ Bars bars_at(uint8_t* smem, const Params& p) {
   r.zacc_full = r.r2_empty + 64;
   r.zacc_empty = r.zacc_full + 2;
   r.zsm_full = r.zacc_empty + 2;
-  r.zsm_empty = r.zsm_full + 1;
-  r.d_full = r.zsm_empty + 1;
-  r.d_empty = r.d_full + 3;
-  r.drain = r.d_empty + 3;
-  r.cbar = r.drain + 2;
-  r.tmem_slot = reinterpret_cast<uint32_t*>(r.cbar + 1);
+  r.zsm_empty = r.zsm_full + 2;
+  r.a_full = r.zsm_empty + 2;
+  r.a_empty = r.a_full + 2;
+  r.b_full = r.a_empty + 2;
+  r.b_empty = r.b_full + 2;
+  r.pairs_full = r.b_empty + 2;
+  r.pairs_empty = r.pairs_full + 2;
+  r.gbar = r.pairs_empty + 2;
+  r.drain = r.gbar + 2;
+  r.tmem_slot = reinterpret_cast<uint32_t*>(r.drain + 3);
   r.abort_flag = reinterpret_cast<int*>(r.tmem_slot + 1);
   return r;
 }
-constexpr uint32_t kBarBytes = (16 + 128 + 15) * 8 + 16;
+constexpr uint32_t kBarSlots = 16 + 128 + 2 * 12 + 3;  // up to and with drain
+constexpr uint32_t kBarBytes = kBarSlots * 8 + 16;
 
 // Slow path of the bounded mbarrier wait: false once the limit passes or another
 // thread gave up.
@@ -178,17 +222,22 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return wait_bar_slow(bar, parity, abort_flag, status);
 }
 
-
-// Barrier of the 16 consumer warps on an mbarrier, so that it is bounded like every
-// other wait: if any role gives up (and raises the abort flag), a warp waiting here
-// leaves too instead of waiting for a warp that has already returned.  `phase` is
+// Bounded entry barrier of one group's eight warps (an mbarrier, so that a warp of the
+// group that gave up elsewhere cannot leave the others waiting without limit).  `phase` is
 // the calling thread's parity of the barrier, flipped at every use.
-__device__ __forceinline__ bool consumer_sync(const Bars& b, uint32_t& phase, unsigned int* status) {
+__device__ __forceinline__ bool group_enter(uint64_t* gbar, uint32_t& phase, volatile int* abort_flag,
+                                            unsigned int* status) {
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(b.cbar);
-  const bool ok = wait_bar(b.cbar, phase, b.abort_flag, status);
+  if ((threadIdx.x & 31) == 0) mbar_arrive(gbar);
+  const bool ok = wait_bar(gbar, phase, abort_flag, status);
   phase ^= 1u;
   return ok;
+}
+
+// Named barrier of one group's 256 threads.  Used only between a group_enter and the end
+// of the same phase, where no thread waits on anything else.
+__device__ __forceinline__ void group_bar(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kGroupThreads) : "memory");
 }
 
 // Order-preserving map of fp32 onto uint32 and its inverse.
@@ -241,59 +290,99 @@ __device__ __forceinline__ float zs_value(const uint8_t* zs, int t, int i) {
   return __bfloat162float(*hi) + __bfloat162float(*lo);
 }
 
-// ---- role: TMA producer of X and R1 -----------------------------------------------
-
-template <int R, int KCAP>
-__device__ void producer_x(const Params& p, const Bars& b, uint8_t* smem, const CUtensorMap* tmX,
-                           const CUtensorMap* tmR1) {
-  using C = Cfg<R, KCAP>;
-  int s = 0;
-  uint32_t ph = 0;
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-    for (int kb = 0; kb < p.kb_count; ++kb) {
-      if (!wait_bar(&b.x_empty[s], ph ^ 1u, b.abort_flag, p.a.status)) return;
-      mbar_arrive_expect_tx(&b.x_full[s], C::X_STAGE + C::R1_STAGE);
-      tma_load_2d(smem + p.off_x + s * C::X_STAGE, tmX, &b.x_full[s], kb * C::BK, tile * kBT);
-#pragma unroll
-      for (int q = 0; q < C::R1_BOXES; ++q)
-        tma_load_2d(smem + p.off_r1 + s * C::R1_STAGE + q * C::R1_BOX_BYTES, tmR1, &b.x_full[s], q * 64,
-                    kb * C::BK);
-      if (++s == p.x_stages) {
-        s = 0;
-        ph ^= 1u;
-      }
-    }
-  }
+// Byte offset of R2 element (row i, expert e_local of a 128-expert stage) in the
+// MN-major 128B-swizzled stage written by TMA (two boxes of 64 experts x R rows).
+template <int R>
+__device__ __forceinline__ uint32_t r2_offset(int i, int e_local) {
+  const int box = e_local >> 6, col = e_local & 63;
+  return (uint32_t)(box * (64 * R * 2) + i * 128 + ((((col >> 3) ^ (i & 7))) << 4) + (col & 7) * 2);
 }
 
-// ---- role: TMA producer of R2 tiles ----------------------------------------------------
+// Number of 128-token tiles this CTA routes (tiles blockIdx.x, blockIdx.x + gridDim.x, ...).
+__device__ __forceinline__ int local_tiles(const Params& p) {
+  return (int)blockIdx.x < p.num_tiles ? (p.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+}
+
+// Position of one thread in a ring of mbarrier-guarded buffers.
+struct Ring {
+  int i = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++i == n) {
+      i = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// ---- role: TMA producer of X, R1 and R2 ---------------------------------------------
+//
+// One thread keeps both rings full: X and R1 stages in tile order, R2 tiles in sweep order
+// (or, when R2 is resident, all of them once).  It polls the rings' empty barriers without
+// blocking and backs off briefly when neither has room, so a slow ring never holds up the
+// other.  It gives up like every bounded wait: after kTimeoutNs without progress, or when
+// another role has raised the abort flag.
 
 template <int R, int KCAP>
-__device__ void producer_r2(const Params& p, const Bars& b, uint8_t* smem, const CUtensorMap* tmR2) {
+__device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CUtensorMap* tmX,
+                         const CUtensorMap* tmR1, const CUtensorMap* tmR2) {
   using C = Cfg<R, KCAP>;
-  if (p.r2_resident) {
-    for (int t = 0; t < p.p_count; ++t) {
-      uint8_t* dst = smem + p.off_r2 + t * C::R2_STAGE;
-      mbar_arrive_expect_tx(&b.r2_full[t], C::R2_STAGE);
-      tma_load_2d(dst, tmR2, &b.r2_full[t], t * kBE, 0);
-      tma_load_2d(dst + C::R2_BOX_BYTES, tmR2, &b.r2_full[t], t * kBE + 64, 0);
+  auto load_r2 = [&](int slot, int t) {
+    uint8_t* dst = smem + p.off_r2 + slot * C::R2_STAGE;
+    mbar_arrive_expect_tx(&b.r2_full[slot], C::R2_STAGE);
+    tma_load_2d(dst, tmR2, &b.r2_full[slot], t * kBE, 0);
+    tma_load_2d(dst + C::R2_BOX_BYTES, tmR2, &b.r2_full[slot], t * kBE + 64, 0);
+  };
+  if (p.r2_resident)
+    for (int t = 0; t < p.p_count; ++t) load_r2(t, t);
+  // X side: local tile xt, hidden block kb
+  Ring sx, sr;
+  int xt = 0, kb = 0;
+  const int T = local_tiles(p);
+  // R2 side: stage t of sweep q
+  int q = 0, rt = 0;
+  const int nsw = p.r2_resident ? 0 : sweep_count(T, p.interleave);
+  uint64_t idle_since = global_timer_ns();
+  uint32_t polls = 0;
+  while (xt < T || q < nsw) {
+    bool progress = false;
+    if (xt < T && mbar_test_wait(&b.x_empty[sx.i], sx.phase ^ 1u)) {
+      const int tile = (int)blockIdx.x + xt * (int)gridDim.x;
+      mbar_arrive_expect_tx(&b.x_full[sx.i], C::X_STAGE + C::R1_STAGE);
+      tma_load_2d(smem + p.off_x + sx.i * C::X_STAGE, tmX, &b.x_full[sx.i], kb * C::BK, tile * kBT);
+#pragma unroll
+      for (int r = 0; r < C::R1_BOXES; ++r)
+        tma_load_2d(smem + p.off_r1 + sx.i * C::R1_STAGE + r * C::R1_BOX_BYTES, tmR1, &b.x_full[sx.i], r * 64,
+                    kb * C::BK);
+      sx.next(p.x_stages);
+      if (++kb == p.kb_count) {
+        kb = 0;
+        ++xt;
+      }
+      progress = true;
     }
-    return;
-  }
-  int s = 0;
-  uint32_t ph = 0;
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-    for (int pass = 0; pass < 2; ++pass) {
-      for (int t = 0; t < p.p_count; ++t) {
-        if (!wait_bar(&b.r2_empty[s], ph ^ 1u, b.abort_flag, p.a.status)) return;
-        uint8_t* dst = smem + p.off_r2 + s * C::R2_STAGE;
-        mbar_arrive_expect_tx(&b.r2_full[s], C::R2_STAGE);
-        tma_load_2d(dst, tmR2, &b.r2_full[s], t * kBE, 0);
-        tma_load_2d(dst + C::R2_BOX_BYTES, tmR2, &b.r2_full[s], t * kBE + 64, 0);
-        if (++s == p.r2_stages) {
-          s = 0;
-          ph ^= 1u;
-        }
+    if (q < nsw && mbar_test_wait(&b.r2_empty[sr.i], sr.phase ^ 1u)) {
+      load_r2(sr.i, rt);
+      sr.next(p.r2_stages);
+      if (++rt == p.p_count) {
+        rt = 0;
+        ++q;
+      }
+      progress = true;
+    }
+    if (progress) {
+      polls = 0;
+      continue;
+    }
+    __nanosleep(64);
+    if ((++polls & 63u) == 0) {
+      if (*reinterpret_cast<volatile int*>(b.abort_flag)) return;
+      const uint64_t now = global_timer_ns();
+      if (polls == 64) idle_since = now;
+      if (now - idle_since > kTimeoutNs) {
+        atomicOr(p.a.status, MORE_DEVERR_WAIT_TIMEOUT);
+        *reinterpret_cast<volatile int*>(b.abort_flag) = 1;
+        return;
       }
     }
   }
@@ -304,8 +393,7 @@ __device__ void producer_r2(const Params& p, const Bars& b, uint8_t* smem, const
 template <int R, int KCAP>
 __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  int s = 0;
-  uint32_t ph = 0;
+  Ring s;
   int lt = 0;
   const uint32_t x0 = smem_u32(smem + p.off_x), r10 = smem_u32(smem + p.off_r1);
   for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
@@ -314,20 +402,17 @@ __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tm
     tc_fence_after();
     const uint32_t d = tmem_base + C::ZCOL0 + buf * C::ZCOLS;
     for (int kb = 0; kb < p.kb_count; ++kb) {
-      if (!wait_bar(&b.x_full[s], ph, b.abort_flag, p.a.status)) goto done;
+      if (!wait_bar(&b.x_full[s.i], s.phase, b.abort_flag, p.a.status)) goto done;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < C::BK / 16; ++kk) {
-        uint64_t ad = smem_desc(x0 + s * C::X_STAGE + kk * 32, 16, C::X_SBO, C::X_LAYOUT);
-        uint64_t bd = smem_desc(r10 + s * C::R1_STAGE + kk * 16 * C::R1_ROW, C::R1_BOX_BYTES, 8 * C::R1_ROW,
+        uint64_t ad = smem_desc(x0 + s.i * C::X_STAGE + kk * 32, 16, C::X_SBO, C::X_LAYOUT);
+        uint64_t bd = smem_desc(r10 + s.i * C::R1_STAGE + kk * 16 * C::R1_ROW, C::R1_BOX_BYTES, 8 * C::R1_ROW,
                                 C::R1_LAYOUT);
         mma_bf16(d, ad, bd, C::IDESC_Z, (kb | kk) != 0);
       }
-      mma_commit(&b.x_empty[s]);
-      if (++s == p.x_stages) {
-        s = 0;
-        ph ^= 1u;
-      }
+      mma_commit(&b.x_empty[s.i]);
+      s.next(p.x_stages);
     }
     mma_commit(&b.zacc_full[buf]);
   }
@@ -336,66 +421,332 @@ done:
   wait_bar(&b.drain[0], 0, b.abort_flag, p.a.status);
 }
 
-// ---- role: MMA issuer of the logit tiles -------------------------------------------------
+// ---- roles: MMA issuers of the logit passes ---------------------------------------------
+//
+// Both issuers walk every sweep's R2 tiles in order.  For each tile they release their
+// share of the R2 stage: a commit when they issued MMAs that read it (it arrives when those
+// MMAs complete), a plain arrival otherwise.  Group A reads the stages of the first sweep
+// for the R2 column norms and arrives then; in later sweeps the pass A issuer arrives for it.
+
+template <int R, int KCAP, bool PASS_B>
+__device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
+  using C = Cfg<R, KCAP>;
+  Ring rs, d;
+  const int T = local_tiles(p), nsw = sweep_count(T, p.interleave);
+  const uint32_t zs0 = smem_u32(smem + p.off_zs), r20 = smem_u32(smem + p.off_r2);
+  uint64_t* full = PASS_B ? b.b_full : b.a_full;
+  uint64_t* empty = PASS_B ? b.b_empty : b.a_empty;
+  constexpr int NBUF = PASS_B ? C::NB : C::NA;
+  constexpr int COL0 = PASS_B ? C::NA * 128 : 0;
+  // pass A reads z_hi only (K = r); pass B reads z_hi | z_lo (K = 2r) for exact logits
+  constexpr int KSTEPS = PASS_B ? C::RK / 16 : R / 16;
+  for (int q = 0; q < nsw; ++q) {
+    const Sweep sw = sweep_jobs(q, T, p.interleave);
+    const int j = PASS_B ? sw.tb : sw.ta;
+    const uint32_t zs = j >= 0 ? zs0 + zs_buf(j, p.interleave) * C::ZS_BYTES : 0u;
+    for (int t = 0; t < p.p_count; ++t) {
+      int st;
+      if (p.r2_resident) {
+        st = t;
+        if (q == 0 && !wait_bar(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
+      } else {
+        st = rs.i;
+        if (!wait_bar(&b.r2_full[rs.i], rs.phase, b.abort_flag, p.a.status)) goto done;
+      }
+      if (j >= 0) {
+        // the tile's z buffer is written by group A's epilogue
+        if (t == 0 && !wait_bar(&b.zsm_full[zs_buf(j, p.interleave)], zs_use(j, p.interleave) & 1, b.abort_flag,
+                                p.a.status))
+          goto done;
+        if (!wait_bar(&empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + COL0 + d.i * 128;
+        const uint32_t r2 = r20 + st * C::R2_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          const uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
+          const uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
+          if (PASS_B)
+            mma_bf16(dt, rd, zd, C::IDESC_PB, kk != 0);
+          else
+            mma_bf16(dt, zd, rd, C::IDESC_PA, kk != 0);
+        }
+        mma_commit(&full[d.i]);
+        d.next(NBUF);
+      }
+      if (!p.r2_resident) {
+        if (j >= 0)
+          mma_commit(&b.r2_empty[rs.i]);
+        else
+          mbar_arrive(&b.r2_empty[rs.i]);
+        if (!PASS_B && q > 0) mbar_arrive_count(&b.r2_empty[rs.i], kGroupWarps);  // for group A
+        rs.next(p.r2_stages);
+      }
+    }
+    // tile tb's z buffer: its pass B MMAs are one of the two releases (group B's finalize is
+    // the other)
+    if (PASS_B && j >= 0) mma_commit(&b.zsm_empty[zs_buf(j, p.interleave)]);
+  }
+done:
+  mma_commit(&b.drain[PASS_B ? 2 : 1]);
+  wait_bar(&b.drain[PASS_B ? 2 : 1], 0, b.abort_flag, p.a.status);
+}
+
+// ---- group A: epilogue, pass A, select ------------------------------------------------------
 
 template <int R, int KCAP>
-__device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
+__device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  int rs = 0;
-  uint32_t rph = 0;
-  int ds = 0;
-  uint32_t dph = 0;
-  int lt = 0;
-  const uint32_t zs = smem_u32(smem + p.off_zs), r20 = smem_u32(smem + p.off_r2);
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
-    if (!wait_bar(b.zsm_full, lt & 1, b.abort_flag, p.a.status)) goto done;
-    for (int pass = 0; pass < 2; ++pass) {
-      for (int t = 0; t < p.p_count; ++t) {
+  constexpr int KL = C::KL;
+  const RouteArgs& a = p.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int aw = warp - kWarpA0;        // 0..7
+  const int sp = warp & 3;              // TMEM lane group: lanes 32 sp .. 32 sp + 31
+  const int hh = aw >> 2;               // which of the lane group's two warps
+  const int gt = aw * 32 + lane;        // 0..255
+  const int t = sp * 32 + lane;         // token of this thread
+  const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+  const uint32_t low = p.low_mask;
+  uint8_t* zs0 = smem + p.off_zs;
+  const uint8_t* r2s = smem + p.off_r2;
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);  // merge exchange, then stage
+  int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
+  int* scan = reinterpret_cast<int*>(smem + p.off_scan);
+  float* znorm = reinterpret_cast<float*>(smem + p.off_znorm);  // [hi h0 | hi h1 | lo h0 | lo h1][token]
+  float* cnorm = reinterpret_cast<float*>(smem + p.off_cnorm);  // [8] per warp, [8] = result
+  uint32_t gph = 0;
+  Ring ad, rs;
+  float colmax2 = 0.f;  // this warp's largest squared R2 column norm (first tile)
+  const int T = local_tiles(p);
+  uint32_t kl[KL];
+
+  for (int j = 0; j < T; ++j) {
+    const int64_t n0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kBT;
+    const bool first = j == 0;
+    // ---------------- epilogue: Z from TMEM -> (z_hi, z_lo) -> shared memory ----------------
+    {
+      const int buf = j & 1;
+      if (!wait_bar(&b.zacc_full[buf], (j >> 1) & 1, b.abort_flag, a.status)) return;
+      tc_fence_after();
+      constexpr int HALF = R / 2;
+      uint32_t zr[HALF];
+      const uint32_t taddr = tmem_base + lane_base + C::ZCOL0 + buf * C::ZCOLS + hh * HALF;
+      if constexpr (HALF == 8) {
+        tmem_ld_x8(taddr, zr);
+      } else if constexpr (HALF == 16) {
+        tmem_ld_x16(taddr, zr);
+      } else {
+#pragma unroll
+        for (int q = 0; q < HALF / 32; ++q) tmem_ld_x32(taddr + q * 32, zr + q * 32);
+      }
+      tmem_wait_ld();
+      reg_fence<HALF>(zr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.zacc_empty[buf]);
+      // the previous tile of this z buffer: its pass B MMAs and its finalize are done
+      const int zb = zs_buf(j, p.interleave), u = zs_use(j, p.interleave);
+      if (u > 0 && !wait_bar(&b.zsm_empty[zb], (u - 1) & 1, b.abort_flag, a.status)) return;
+      uint8_t* zs = zs0 + zb * C::ZS_BYTES;
+      float hi2 = 0.f, lo2 = 0.f;
+#pragma unroll
+      for (int q = 0; q < HALF / 8; ++q) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          float z0 = __uint_as_float(zr[q * 8 + 2 * jj]), z1 = __uint_as_float(zr[q * 8 + 2 * jj + 1]);
+          __nv_bfloat16 h0 = __float2bfloat16_rn(z0), h1 = __float2bfloat16_rn(z1);
+          __nv_bfloat16 l0 = __float2bfloat16_rn(z0 - __bfloat162float(h0));
+          __nv_bfloat16 l1 = __float2bfloat16_rn(z1 - __bfloat162float(h1));
+          const float fh0 = __bfloat162float(h0), fh1 = __bfloat162float(h1);
+          const float fl0 = __bfloat162float(l0), fl1 = __bfloat162float(l1);
+          hi2 = fmaf(fh0, fh0, fmaf(fh1, fh1, hi2));
+          lo2 = fmaf(fl0, fl0, fmaf(fl1, fl1, lo2));
+          hi[jj] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          lo[jj] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        const int i0 = hh * HALF + q * 8;  // first z index of this 8-group
+        *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, i0 >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, (R + i0) >> 3)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      znorm[hh * kBT + t] = hi2;
+      znorm[(2 + hh) * kBT + t] = lo2;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.zsm_full[zb]);
+    }
+
+    // ---------------- pass A: chunk maxima of z_hi . R2 -> top KL chunk keys -------------
+    // warp hh of a lane group owns columns 64 hh .. 64 hh + 63 (chunks 4 pt + 2 hh, + 1)
+#pragma unroll
+    for (int i = 0; i < KL; ++i) kl[i] = 0u;
+    for (int pt = 0; pt < p.p_count; ++pt) {
+      if (!wait_bar(&b.a_full[ad.i], ad.phase, b.abort_flag, a.status)) return;
+      tc_fence_after();
+      const uint32_t col = tmem_base + lane_base + ad.i * 128 + hh * 64;
+      const int c0 = pt * 4 + 2 * hh;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld_x32(col + 32 * half, v);
+        tmem_wait_ld();
+        reg_fence<32>(v);
+        if (half == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b.a_empty[ad.i]);
+        }
+        const int c = c0 + half;
+        if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (32 * c + jj >= a.M) v[jj] = 0xff800000u;
+        }
+        key_insert<KL>(kl, (ord_key(max32(v)) & ~low) | (uint32_t)c);
+      }
+      ad.next(C::NA);
+      if (first) {
+        // squared column norms of R2 (experts 16 aw .. 16 aw + 15 of the stage)
         int st;
         if (p.r2_resident) {
-          st = t;
-          if (lt == 0 && pass == 0 && !wait_bar(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
+          st = pt;
+          if (!wait_bar(&b.r2_full[pt], 0, b.abort_flag, a.status)) return;
         } else {
-          st = rs;
-          if (!wait_bar(&b.r2_full[rs], rph, b.abort_flag, p.a.status)) goto done;
+          st = rs.i;
+          if (!wait_bar(&b.r2_full[rs.i], rs.phase, b.abort_flag, a.status)) return;
         }
-        if (!wait_bar(&b.d_empty[ds], dph ^ 1u, b.abort_flag, p.a.status)) goto done;
-        tc_fence_after();
-        const uint32_t d = tmem_base + ds * 128;
-        const uint32_t r2 = r20 + st * C::R2_STAGE;
-        // pass 1 reads z_hi only (K = r); pass 2 reads z_hi | z_lo (K = 2r) for exact logits
-        const int ksteps = pass == 0 ? R / 16 : C::RK / 16;
-#pragma unroll
-        for (int kk = 0; kk < ksteps; ++kk) {
-          uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
-          uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
-          if (pass == 0)
-            mma_bf16(d, zd, rd, C::IDESC_P1, kk != 0);
-          else
-            mma_bf16(d, rd, zd, C::IDESC_P2, kk != 0);
+        const uint8_t* base = r2s + st * C::R2_STAGE;
+        const int el = 16 * aw + (lane & 15);
+        float acc = 0.f;
+#pragma unroll 4
+        for (int i = lane >> 4; i < R; i += 2) {
+          const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + r2_offset<R>(i, el)));
+          acc = fmaf(w, w, acc);
         }
-        mma_commit(&b.d_full[ds]);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+        colmax2 = fmaxf(colmax2, acc);
         if (!p.r2_resident) {
-          mma_commit(&b.r2_empty[rs]);
-          if (++rs == p.r2_stages) {
-            rs = 0;
-            rph ^= 1u;
-          }
-        }
-        if (++ds == C::ND) {
-          ds = 0;
-          dph ^= 1u;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b.r2_empty[rs.i]);
+          rs.next(p.r2_stages);
         }
       }
     }
-    mma_commit(b.zsm_empty);
+
+    // ---------------- select: merge the lists, certified window, needed pairs --------------
+    const int pb = j & 1, pu = j >> 1;  // pair buffer and its use count
+    // the pair buffer's previous tile (j - 2) is finalized by group B
+    if (pu > 0 && !wait_bar(&b.pairs_empty[pb], (pu - 1) & 1, b.abort_flag, a.status)) return;
+    uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs + pb * C::PAIR_BYTES);
+    int* cbase = reinterpret_cast<int*>(smem + p.off_cbase) + pb * (p.nchunks + 1);
+    uint8_t* flag = smem + p.off_flag + pb * kBT;
+    uint8_t* nq = smem + p.off_nq + pb * kBT;
+    if (hh == 1) {
+#pragma unroll
+      for (int i = 0; i < KL; ++i) lists[i * kBT + t] = kl[i];
+    }
+    if (first) {
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, d));
+      if (lane == 0) cnorm[aw] = colmax2;
+    }
+    if (!group_enter(&b.gbar[0], gph, b.abort_flag, a.status)) return;
+    // from here to the hand-off nothing waits on another role
+    if (hh == 0) {
+#pragma unroll
+      for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[i * kBT + t]);
+    }
+    if (first && gt == 0) {
+      float m = 0.f;
+      for (int w = 0; w < kGroupWarps; ++w) m = fmaxf(m, cnorm[w]);
+      cnorm[kGroupWarps] = sqrtf(m) * (1.f + 0x1p-20f);  // max column norm of R2, rounded up
+    }
+    group_bar(kNamedBarA);  // the merge has read the exchanged lists; cnorm is final
+    uint32_t* stage = lists;  // (chunk, rank) of each needed pair of token t
+    float ccut = -INFINITY;   // candidates: exact logit >= ccut
+    int needed = 0;
+    if (hh == 0) {
+      const bool active = n0 + t < a.N;
+      // Certified window: values from z_hi differ from the z_hi + z_lo values by at most
+      // eps = |z_lo| cmax (Cauchy-Schwarz) plus a bound on fp32 accumulation differences.
+      const float cmax = cnorm[kGroupWarps];
+      const float zh = sqrtf(znorm[t] + znorm[kBT + t]);
+      const float zl = sqrtf(znorm[2 * kBT + t] + znorm[3 * kBT + t]);
+      const float eps = (zl * cmax) * (1.f + 0x1p-8f) + (float)R * 0x1p-20f * zh * cmax + 1e-30f;
+      uint32_t kth = 0;
+#pragma unroll
+      for (int i = 0; i < KL; ++i)
+        if (i == a.k - 1) kth = kl[i];
+      int f = active ? 0 : 2;
+      // The k chunks with the largest z_hi maxima (>= tlow) hold k elements whose exact logit
+      // is >= tlow - eps, so the exact k-th logit is >= tlow - eps (the candidate cut), and an
+      // element reaching it has a z_hi logit >= tlow - 2 eps (the chunk cut).
+      uint32_t cut_key = 0u;  // chunks whose key range reaches cut_key are needed
+      if ((kth & ~low) >= kRealKey) {
+        const float tlow = ord_inv(kth & ~low);  // <= the k-th largest z_hi chunk maximum
+        ccut = __fsub_rd(tlow, eps);
+        cut_key = ord_key(__fsub_rd(tlow, __fmul_ru(2.f, eps)));
+        if ((kl[KL - 1] & ~low) >= kRealKey && (kl[KL - 1] | low) >= cut_key) f |= 1;  // list too short
+      }
+      if (f == 0) {
+#pragma unroll
+        for (int i = 0; i < KL; ++i) {
+          if ((kl[i] & ~low) >= kRealKey && (kl[i] | low) >= cut_key) {
+            const uint32_t cid = kl[i] & low;
+            const int rank = atomicAdd(&ccount[cid], 1);
+            stage[i * kBT + t] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
+            needed = i + 1;
+          }
+        }
+      }
+      flag[t] = (uint8_t)f;
+      nq[t] = (uint8_t)needed;
+    }
+    group_bar(kNamedBarA);
+    // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty),
+    // eight chunks per thread
+    {
+      int vals[8], run = 0;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int i = gt * 8 + jj;
+        vals[jj] = (i < p.nchunks) ? ccount[i] : 0;
+        run += vals[jj];
+      }
+      int incl = run;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      if (lane == 31) scan[aw] = incl;
+      group_bar(kNamedBarA);
+      int before = incl - run;
+      for (int w = 0; w < aw; ++w) before += scan[w];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int i = gt * 8 + jj;
+        if (i <= p.nchunks) cbase[i] = before;
+        if (i < p.nchunks) ccount[i] = 0;
+        before += vals[jj];
+      }
+      // the end of the last bucket (index nchunks lies past the 8 x 256 slots when nchunks == 2048)
+      if (gt == kGroupThreads - 1) cbase[p.nchunks] = before;
+    }
+    group_bar(kNamedBarA);
+    if (hh == 0) {
+      for (int i = 0; i < needed; ++i) {
+        const uint32_t st = stage[i * kBT + t];
+        // {token | needed-chunk index << 8, candidate cut}
+        pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(ccut));
+      }
+    }
+    group_bar(kNamedBarA);  // the pairs are written; the stage area may be reused
+    if (gt == 0) mbar_arrive(&b.pairs_full[pb]);
   }
-done:
-  mma_commit(&b.drain[1]);
-  wait_bar(&b.drain[1], 0, b.abort_flag, p.a.status);
 }
 
-// ---- consumers ----------------------------------------------------------------------------
+// ---- group B: pass B, finalize ------------------------------------------------------------
 
 // Exact recomputation on CUDA cores of the logits of one token (ties at the threshold,
 // candidate overflow), for the 256-expert block eb .. eb + 255: lane l takes experts
@@ -434,10 +785,10 @@ __device__ __forceinline__ void fallback_block(const RouteArgs& a, const float (
 }
 
 // The cooperative fallback's first step: this warp's partial top-k (over the 256-expert
-// blocks cw, cw + 16, ...) of each of the nb tokens in tok, written to part.
+// blocks bw, bw + 8, ...) of each of the nb tokens in tok, written to part.
 template <int R, int KCAP>
 __device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t* zs, const uint8_t* tok, int nb,
-                                           uint2* part, int cw, int lane) {
+                                              uint2* part, int bw, int lane) {
   for (int j = 0; j < nb; ++j) {
     const int tf = tok[j];
     float zr[(R + 31) / 32];
@@ -446,21 +797,21 @@ __device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t*
       zr[q] = (32 * q + lane < R) ? zs_value<R, KCAP>(zs, tf, 32 * q + lane) : 0.f;
     TopList<KCAP> list;
     list.init();
-    for (int eb = 256 * cw; eb < a.M; eb += 256 * kConsumerWarps) fallback_block<R, KCAP>(a, zr, eb, lane, list);
+    for (int eb = 256 * bw; eb < a.M; eb += 256 * kGroupWarps) fallback_block<R, KCAP>(a, zr, eb, lane, list);
     float v;
     int e;
     warp_merge_topk<KCAP>(list, a.k, lane, v, e);
-    if (lane < KCAP) part[(j * kConsumerWarps + cw) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
+    if (lane < KCAP) part[(j * kGroupWarps + bw) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
   }
 }
 
-// The second step: merge the sixteen partial lists of one token (part: warp-major, KCAP
+// The second step: merge the eight partial lists of one token (part: warp-major, KCAP
 // entries each, the first k valid) and write the token's outputs.
 template <int KCAP>
 __device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* part, int64_t n, int lane) {
   TopList<KCAP> list;
   list.init();
-  for (int q = lane; q < kConsumerWarps * KCAP; q += 32) {
+  for (int q = lane; q < kGroupWarps * KCAP; q += 32) {
     const uint2 c = part[q];
     if ((q % KCAP) < a.k) list.insert_any(__uint_as_float(c.x), (int)c.y);
   }
@@ -470,470 +821,209 @@ __device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* 
   warp_write_selection(a, n, lane, v, e);
 }
 
-// Byte offset of R2 element (row i, expert e_local of a 128-expert stage) in the
-// MN-major 128B-swizzled stage written by TMA (two boxes of 64 experts x R rows).
-template <int R>
-__device__ __forceinline__ uint32_t r2_offset(int i, int e_local) {
-  const int box = e_local >> 6, col = e_local & 63;
-  return (uint32_t)(box * (64 * R * 2) + i * 128 + ((((col >> 3) ^ (i & 7))) << 4) + (col & 7) * 2);
-}
-
 template <int R, int KCAP>
-__device__ void consumers(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
+__device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
   constexpr int KL = C::KL;
+  constexpr int NC = KL + kPoolSlots;
   const RouteArgs& a = p.a;
-  uint32_t cph = 0;  // parity of the consumer barrier
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sp = warp & 3;              // TMEM subpartition: lanes 32 sp .. 32 sp + 31
-  const int g = (warp - 4) >> 2;        // consumer warpgroup 0..3
-  const int cw = warp - 4;              // consumer warp 0..15
-  const int ctid = threadIdx.x - 128;   // 0..511
-  const int t = sp * 32 + lane;         // token of this thread in pass 1 and finalize
+  const int bw = warp - kWarpB0;        // 0..7
+  const int sp = warp & 3;              // TMEM lane group: lanes 32 sp .. 32 sp + 31
+  const int hh = bw >> 2;               // which of the lane group's two warps
+  const int gt = bw * 32 + lane;        // 0..255
+  const int t = sp * 32 + lane;         // token of this thread in the finalize
   const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-  uint8_t* zs = smem + p.off_zs;
-  const uint8_t* r2s = smem + p.off_r2;
-  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);
-  uint32_t* stage = lists + 2 * KL * kBT;  // (chunk, rank) of each needed pair, after the two list slots
+  uint8_t* zs0 = smem + p.off_zs;
   uint2* cand = reinterpret_cast<uint2*>(smem + p.off_cand);
-  float* thr = reinterpret_cast<float*>(smem + p.off_thr);
-  int* flag = reinterpret_cast<int*>(smem + p.off_flag);
-  uint8_t* nq = smem + p.off_nq;
+  uint8_t* pc = smem + p.off_pc;
+  uint2* pool = reinterpret_cast<uint2*>(smem + p.off_pool);
+  int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
   int* fbcount = reinterpret_cast<int*>(smem + p.off_fb);
   uint8_t* fblist = smem + p.off_fb + 4;
   uint8_t* fbmark = smem + p.off_fb + 4 + kBT;  // 1: the token's outputs come from the fallback
-  uint2* part = reinterpret_cast<uint2*>(smem + p.off_lists);  // fallback partial lists (finalize only)
-  uint8_t* pc = smem + p.off_pc;
-  uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs);
-  int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
-  int* cbase = reinterpret_cast<int*>(smem + p.off_cbase);
-  int* scan = reinterpret_cast<int*>(smem + p.off_scan);
-  uint2* pool = reinterpret_cast<uint2*>(smem + p.off_pool);
-  int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
-  float* znorm = reinterpret_cast<float*>(smem + p.off_znorm);  // [hi g0 | hi g1 | lo g0 | lo g1][token]
-  float* cnorm = reinterpret_cast<float*>(smem + p.off_cnorm);
-  const uint32_t low = p.low_mask;
-  int ds = 0, rs = 0;
-  uint32_t dph = 0, rph = 0;
-  int lt = 0;
-  float colmax2 = 0.f;  // this warp's largest squared R2 column norm (first tile)
+  uint2* part = reinterpret_cast<uint2*>(smem + p.off_part);
+  uint32_t gph = 0;
+  Ring bd;
+  const int T = local_tiles(p);
 
-  // R2 stage of the current logit tile: wait until it is in shared memory.
-  auto r2_stage = [&](int pt, int& st) -> bool {
-    if (p.r2_resident) {
-      st = pt;
-      return wait_bar(&b.r2_full[pt], 0, b.abort_flag, a.status);
-    }
-    st = rs;
-    return wait_bar(&b.r2_full[rs], rph, b.abort_flag, a.status);
-  };
-  // This warp is done with the R2 stage of the current logit tile; it arrives for
-  // `count` consumer warps (0: only advance the stage counters).
-  auto r2_release = [&](uint32_t count) {
-    if (p.r2_resident) return;
-    if (count) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive_count(&b.r2_empty[rs], count);
-    }
-    if (++rs == p.r2_stages) {
-      rs = 0;
-      rph ^= 1u;
-    }
-  };
+  for (int j = 0; j < T; ++j) {
+    const int64_t n0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kBT;
+    const int pb = j & 1, pu = j >> 1;
+    if (!wait_bar(&b.pairs_full[pb], pu & 1, b.abort_flag, a.status)) return;
+    const uint2* pairs = reinterpret_cast<const uint2*>(smem + p.off_pairs + pb * C::PAIR_BYTES);
+    const int* cbase = reinterpret_cast<const int*>(smem + p.off_cbase) + pb * (p.nchunks + 1);
+    const uint8_t* flag = smem + p.off_flag + pb * kBT;
+    const uint8_t* nq = smem + p.off_nq + pb * kBT;
 
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
-    const int64_t n0 = (int64_t)tile * kBT;
-    const int buf = lt & 1;
-    // ---------------- Z epilogue (warpgroups 0, 1): TMEM -> (z_hi, z_lo) -> smem ----------
-    if (g < 2) {
-      if (!wait_bar(&b.zacc_full[buf], (lt >> 1) & 1, b.abort_flag, a.status)) return;
-      tc_fence_after();
-      constexpr int HALF = R / 2;
-      uint32_t zr[HALF];
-      const uint32_t taddr = tmem_base + lane_base + C::ZCOL0 + buf * C::ZCOLS + g * HALF;
-      if constexpr (HALF == 8) {
-        tmem_ld_x8(taddr, zr);
-      } else if constexpr (HALF == 16) {
-        tmem_ld_x16(taddr, zr);
-      } else {
-#pragma unroll
-        for (int q = 0; q < HALF / 32; ++q) tmem_ld_x32(taddr + q * 32, zr + q * 32);
-      }
-      tmem_wait_ld();
-      reg_fence<HALF>(zr);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b.zacc_empty[buf]);
-      // the previous tile's logit MMAs must be done with the z buffer
-      if (lt > 0 && !wait_bar(b.zsm_empty, (lt - 1) & 1, b.abort_flag, a.status)) return;
-      float hi2 = 0.f, lo2 = 0.f;
-#pragma unroll
-      for (int q = 0; q < HALF / 8; ++q) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float z0 = __uint_as_float(zr[q * 8 + 2 * j]), z1 = __uint_as_float(zr[q * 8 + 2 * j + 1]);
-          __nv_bfloat16 h0 = __float2bfloat16_rn(z0), h1 = __float2bfloat16_rn(z1);
-          __nv_bfloat16 l0 = __float2bfloat16_rn(z0 - __bfloat162float(h0));
-          __nv_bfloat16 l1 = __float2bfloat16_rn(z1 - __bfloat162float(h1));
-          const float fh0 = __bfloat162float(h0), fh1 = __bfloat162float(h1);
-          const float fl0 = __bfloat162float(l0), fl1 = __bfloat162float(l1);
-          hi2 = fmaf(fh0, fh0, fmaf(fh1, fh1, hi2));
-          lo2 = fmaf(fl0, fl0, fmaf(fl1, fl1, lo2));
-          hi[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-          lo[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-        }
-        const int i0 = g * HALF + q * 8;  // first z index of this 8-group
-        *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, i0 >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(zs + zs_offset<R, KCAP>(t, (R + i0) >> 3)) =
-            make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      znorm[g * kBT + t] = hi2;
-      znorm[(2 + g) * kBT + t] = lo2;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b.zsm_full);
-    }
-
-    // ---------------- pass 1: chunk maxima of z_hi . R2 -> top KL chunk keys -------------
-    // warpgroup g owns columns 32 g .. 32 g + 31 of every 128-expert tile.
-    uint32_t kl[KL];
-#pragma unroll
-    for (int i = 0; i < KL; ++i) kl[i] = 0u;
+    // ---------------- pass B: candidates of the needed chunks (exact z_hi + z_lo logits) ----
+    // Lane group sp of the transposed tile is chunk 4 pt + sp; its two warps split the
+    // chunk's pairs in halves.
     for (int pt = 0; pt < p.p_count; ++pt) {
-      if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
+      const int c = pt * 4 + sp;
+      int lo = 0, hi = 0;
+      if (c < p.nchunks) {
+        const int c_lo = cbase[c], n = cbase[c + 1] - c_lo;
+        lo = c_lo + ((n * hh) >> 1);
+        hi = c_lo + ((n * (hh + 1)) >> 1);
+      }
+      if (!wait_bar(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_x32(tmem_base + lane_base + ds * 128 + g * 32, v);
-      tmem_wait_ld();
-      reg_fence<32>(v);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b.d_empty[ds]);
-      if (++ds == C::ND) {
-        ds = 0;
-        dph ^= 1u;
-      }
-      if (lt == 0) {
-        // first tile of this CTA: squared column norms of R2 (experts 8 cw .. 8 cw + 7 of the stage)
-        int st;
-        if (!r2_stage(pt, st)) return;
-        const uint8_t* base = r2s + st * C::R2_STAGE;
-        const int el = 8 * cw + (lane & 7);
-        float acc = 0.f;
-#pragma unroll 4
-        for (int i = lane >> 3; i < R; i += 4) {
-          const float w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + r2_offset<R>(i, el)));
-          acc = fmaf(w, w, acc);
+      const int e = 32 * c + lane;
+      const bool e_ok = e < a.M;
+      const uint32_t col0 = tmem_base + lane_base + (C::NA + bd.i) * 128;
+      const uint32_t lt_mask = (1u << lane) - 1u;
+      for (int pi = lo; pi < hi; pi += kPairBatch) {
+        const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
+        uint2 ent[kPairBatch];
+        uint32_t val[kPairBatch];
+#pragma unroll
+        for (int q = 0; q < kPairBatch; ++q)
+          if (q < nb) ent[q] = pairs[pi + q];  // {token | slot << 8, candidate cut}
+#pragma unroll
+        for (int q = 0; q < kPairBatch; ++q)
+          if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q].x & 0xffu));
+        tmem_wait_ld();
+        reg_fence<kPairBatch>(val);
+        // per pair: ballot the experts at or above the cut; the first one takes the
+        // pair's slot, lane 0 records the count, any further ones go to the pool below
+        uint32_t bal[kPairBatch];
+        uint32_t extra = 0u;
+#pragma unroll
+        for (int q = 0; q < kPairBatch; ++q) {
+          const bool take = q < nb && e_ok && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y);
+          bal[q] = __ballot_sync(0xffffffffu, take);
+          const uint32_t tq = ent[q].x & 0xffu, iq = ent[q].x >> 8;
+          const uint32_t before = bal[q] & lt_mask;
+          if (take && before == 0u) cand[iq * kBT + tq] = make_uint2(val[q], (uint32_t)e);
+          if (lane == 0 && q < nb) pc[tq * C::KLP + iq] = (uint8_t)__popc(bal[q]);
+          extra |= bal[q] & (bal[q] - 1u);  // set iff the pair has two or more candidates
         }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-        colmax2 = fmaxf(colmax2, acc);
-        r2_release(1);
-      } else {
-        r2_release(cw == 0 ? kConsumerWarps : 0);  // nobody reads R2 here: one warp arrives for all
-      }
-      const int c = pt * 4 + g;
-      if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
+        if (extra) {  // rare: more candidates than the pair's slot
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (32 * c + j >= a.M) v[j] = 0xff800000u;
-      }
-      key_insert<KL>(kl, (ord_key(max32(v)) & ~low) | (uint32_t)c);
-    }
-
-    // ---------------- select: merge the lists, certified window, needed pairs --------------
-    // two-round merge of the four partial lists: g2 -> g0 and g3 -> g1, then g1 -> g0
-    if (g >= 2) {
-#pragma unroll
-      for (int i = 0; i < KL; ++i) lists[((g - 2) * KL + i) * kBT + t] = kl[i];
-    }
-    if (lt == 0) {
-      colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 1));
-      colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 2));
-      colmax2 = fmaxf(colmax2, __shfl_xor_sync(0xffffffffu, colmax2, 4));
-      if (lane == 0) cnorm[cw] = colmax2;
-    }
-    if (!consumer_sync(b, cph, a.status)) return;
-    if (lt == 0 && ctid == 0) {
-      float m = 0.f;
-      for (int w = 0; w < kConsumerWarps; ++w) m = fmaxf(m, cnorm[w]);
-      cnorm[kConsumerWarps] = sqrtf(m) * (1.f + 0x1p-20f);  // max column norm of R2, rounded up
-    }
-    if (g < 2) {
-#pragma unroll
-      for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(g * KL + i) * kBT + t]);
-      if (g == 1) {  // each thread rewrites only its own column of slot 1
-#pragma unroll
-        for (int i = 0; i < KL; ++i) lists[(KL + i) * kBT + t] = kl[i];
-      }
-    }
-    if (!consumer_sync(b, cph, a.status)) return;
-    if (g == 0) {
-#pragma unroll
-      for (int i = 0; i < KL; ++i) key_insert<KL>(kl, lists[(KL + i) * kBT + t]);
-      const bool active = n0 + t < a.N;
-      // Certified window: values from z_hi differ from the z_hi + z_lo values by at most
-      // eps = |z_lo| cmax (Cauchy-Schwarz) plus a bound on fp32 accumulation differences.
-      const float cmax = cnorm[kConsumerWarps];
-      const float zh = sqrtf(znorm[t] + znorm[kBT + t]);
-      const float zl = sqrtf(znorm[2 * kBT + t] + znorm[3 * kBT + t]);
-      const float eps = (zl * cmax) * (1.f + 0x1p-8f) + (float)R * 0x1p-20f * zh * cmax + 1e-30f;
-      uint32_t kth = 0;
-#pragma unroll
-      for (int i = 0; i < KL; ++i)
-        if (i == a.k - 1) kth = kl[i];
-      int f = active ? 0 : 2;
-      // The k chunks with the largest z_hi maxima (>= tlow) hold k elements whose exact logit
-      // is >= tlow - eps, so the exact k-th logit is >= tlow - eps (the candidate cut), and an
-      // element reaching it has a z_hi logit >= tlow - 2 eps (the chunk cut).
-      float ccut = -INFINITY;                  // candidates: exact logit >= ccut
-      uint32_t cut_key = 0u;                   // chunks whose key range reaches cut_key are needed
-      if ((kth & ~low) >= kRealKey) {
-        const float tlow = ord_inv(kth & ~low);  // <= the k-th largest z_hi chunk maximum
-        ccut = __fsub_rd(tlow, eps);
-        cut_key = ord_key(__fsub_rd(tlow, __fmul_ru(2.f, eps)));
-        if ((kl[KL - 1] & ~low) >= kRealKey && (kl[KL - 1] | low) >= cut_key) f |= 1;  // list too short
-      }
-      int needed = 0;
-      if (f == 0) {
-#pragma unroll
-        for (int i = 0; i < KL; ++i) {
-          if ((kl[i] & ~low) >= kRealKey && (kl[i] | low) >= cut_key) {
-            const uint32_t cid = kl[i] & low;
-            const int rank = atomicAdd(&ccount[cid], 1);
-            stage[i * kBT + t] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
-            needed = i + 1;
-          }
-        }
-      }
-      thr[t] = ccut;
-      flag[t] = f;
-      nq[t] = (uint8_t)needed;
-      poolcnt[t] = 0;
-      if (t == 0 && g == 0) *fbcount = 0;
-    }
-    if (!consumer_sync(b, cph, a.status)) return;
-    // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty)
-    {
-      int vals[4], run = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = ctid * 4 + j;
-        vals[j] = (i < p.nchunks) ? ccount[i] : 0;
-        run += vals[j];
-      }
-      int incl = run;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
-      }
-      if (lane == 31) scan[ctid >> 5] = incl;
-      if (!consumer_sync(b, cph, a.status)) return;
-      int before = incl - run;
-      for (int w = 0; w < (ctid >> 5); ++w) before += scan[w];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = ctid * 4 + j;
-        if (i <= p.nchunks) cbase[i] = before;
-        if (i < p.nchunks) ccount[i] = 0;
-        before += vals[j];
-      }
-      // the end of the last bucket (index nchunks lies past the 4 x 512 slots when nchunks == 2048)
-      if (ctid == kConsumerThreads - 1) cbase[p.nchunks] = before;
-    }
-    if (!consumer_sync(b, cph, a.status)) return;
-    if (g == 0) {
-      const int needed = nq[t];
-      const float cut = thr[t];
-      for (int i = 0; i < needed; ++i) {
-        const uint32_t st = stage[i * kBT + t];
-        // {token | needed-chunk index << 8, candidate cut}
-        pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(cut));
-      }
-    }
-    if (!consumer_sync(b, cph, a.status)) return;
-
-    // ---------------- pass 2: candidates of the needed chunks (exact z_hi + z_lo logits) ----
-    // Lane group sp of the transposed tile is chunk 4 pt + sp.  Tile pt belongs to
-    // warpgroups 0-1 when pt is even, 2-3 when odd: the two warps of a lane group split the
-    // pairs of their chunk (first and second half), so a tile is worked by eight warps and
-    // two tiles at once.  Every warp waits for every tile and arrives once on its empty
-    // barrier (the owners when done, the others at once): a buffer is refilled only after
-    // all sixteen warps have seen its current phase, so no warp can fall two phases
-    // behind, which a parity wait could not tell from the phase it waits for.
-    for (int pt = 0; pt < p.p_count; ++pt) {
-      if (!wait_bar(&b.d_full[ds], dph, b.abort_flag, a.status)) return;
-      if ((pt & 1) == (g >> 1)) {
-        tc_fence_after();
-        const int c = pt * 4 + sp;
-        if (c < p.nchunks) {
-          const int e = 32 * c + lane;
-          const bool e_ok = e < a.M;
-          const uint32_t col0 = tmem_base + lane_base + ds * 128;
-          const uint32_t lt_mask = (1u << lane) - 1u;
-          const int c_lo = cbase[c], c_hi = cbase[c + 1], c_mid = (c_lo + c_hi + 1) >> 1;
-          const int lo = (g & 1) ? c_mid : c_lo, hi = (g & 1) ? c_hi : c_mid;
-          for (int pi = lo; pi < hi; pi += kPairBatch) {
-            const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
-            uint2 ent[kPairBatch];
-            uint32_t val[kPairBatch];
-#pragma unroll
-            for (int q = 0; q < kPairBatch; ++q)
-              if (q < nb) ent[q] = pairs[pi + q];  // {token | slot << 8, candidate cut}
-#pragma unroll
-            for (int q = 0; q < kPairBatch; ++q)
-              if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q].x & 0xffu));
-            tmem_wait_ld();
-            reg_fence<kPairBatch>(val);
-            // per pair: ballot the experts at or above the cut; the first one takes the
-            // pair's slot, lane 0 records the count, any further ones go to the pool below
-            uint32_t bal[kPairBatch];
-            uint32_t extra = 0u;
-#pragma unroll
-            for (int q = 0; q < kPairBatch; ++q) {
-              const bool take = q < nb && e_ok && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y);
-              bal[q] = __ballot_sync(0xffffffffu, take);
-              const uint32_t tq = ent[q].x & 0xffu, iq = ent[q].x >> 8;
-              const uint32_t before = bal[q] & lt_mask;
-              if (take && before == 0u) cand[iq * kBT + tq] = make_uint2(val[q], (uint32_t)e);
-              if (lane == 0 && q < nb) pc[tq * C::KLP + iq] = (uint8_t)__popc(bal[q]);
-              extra |= bal[q] & (bal[q] - 1u);  // set iff the pair has two or more candidates
-            }
-            if (extra) {  // rare: more candidates than the pair's slot
-#pragma unroll
-              for (int q = 0; q < kPairBatch; ++q) {
-                if (((bal[q] >> lane) & 1u) && (bal[q] & lt_mask)) {
-                  const int tok = ent[q].x & 0xff;
-                  const int ps = atomicAdd(&poolcnt[tok], 1);
-                  if (ps < kPoolSlots) pool[ps * kBT + tok] = make_uint2(val[q], (uint32_t)e);
-                }
-              }
+          for (int q = 0; q < kPairBatch; ++q) {
+            if (((bal[q] >> lane) & 1u) && (bal[q] & lt_mask)) {
+              const int tok = ent[q].x & 0xff;
+              const int ps = atomicAdd(&poolcnt[tok], 1);
+              if (ps < kPoolSlots) pool[ps * kBT + tok] = make_uint2(val[q], (uint32_t)e);
             }
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b.d_empty[ds]);
-        r2_release(kConsumerWarps / 8);  // the tile's eight warps stand for all sixteen
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b.d_empty[ds]);
-        r2_release(0);
       }
-      if (++ds == C::ND) {
-        ds = 0;
-        dph ^= 1u;
-      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.b_empty[bd.i]);
+      bd.next(C::NB);
     }
-    if (!consumer_sync(b, cph, a.status)) return;
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
-    // Four threads per token (one per warpgroup).  Every thread loads all of the token's
-    // candidates (the slots of its needed chunks, then its pool entries); thread g ranks
-    // candidates g, g + 4, ... in routing order (larger logit, then lower expert) and the
-    // ones of rank < k go to the output staging at their rank, with exp(logit - max).
-    {
-      constexpr int NC = KL + kPoolSlots;
-      int32_t* sidx = reinterpret_cast<int32_t*>(pairs);  // staging: [token][k], like the outputs
-      float* sex = reinterpret_cast<float*>(sidx + kBT * a.k);
-      float* slog = sex + kBT * a.k;
-      const int f = flag[t];
-      if ((f & 2) == 0) {
-        const int jn = nq[t], np = poolcnt[t];
-        uint32_t cnt[C::KLP / 4];
+    // Two threads per token (the lane group's two warps).  Every thread loads all of the
+    // token's candidates (the slots of its needed chunks, then its pool entries) into
+    // registers; thread hh ranks candidates hh, hh + 2, ... in routing order (larger logit,
+    // then lower expert) and the ones of rank < k go to the output staging at their rank,
+    // with exp(logit - max).  The staging reuses the tile's pair buffer, which pass B has
+    // finished reading.
+    if (!group_enter(&b.gbar[1], gph, b.abort_flag, a.status)) return;
+    // from here to the hand-off nothing waits on another role
+    int32_t* sidx = reinterpret_cast<int32_t*>(smem + p.off_pairs + pb * C::PAIR_BYTES);  // [token][k]
+    float* sex = reinterpret_cast<float*>(sidx + kBT * a.k);
+    float* slog = sex + kBT * a.k;
+    const int f = flag[t];
+    bool fb = false;
+    if ((f & 2) == 0) {
+      uint32_t o[NC], e[NC];
+      const int jn = nq[t], np = poolcnt[t];
+      uint32_t cnt[C::KLP / 4];
 #pragma unroll
-        for (int w = 0; w < C::KLP / 16; ++w) {
-          const uint4 q4 = *reinterpret_cast<const uint4*>(pc + t * C::KLP + 16 * w);
-          cnt[4 * w] = q4.x;
-          cnt[4 * w + 1] = q4.y;
-          cnt[4 * w + 2] = q4.z;
-          cnt[4 * w + 3] = q4.w;
+      for (int w = 0; w < C::KLP / 16; ++w) {
+        const uint4 q4 = *reinterpret_cast<const uint4*>(pc + t * C::KLP + 16 * w);
+        cnt[4 * w] = q4.x;
+        cnt[4 * w + 1] = q4.y;
+        cnt[4 * w + 2] = q4.z;
+        cnt[4 * w + 3] = q4.w;
+      }
+      // -0 and +0 are equal in routing order: both take the key of +0.  Empty slots take
+      // key 0, below every real value, so they never outrank a candidate.
+      int total = 0;
+#pragma unroll
+      for (int q = 0; q < NC; ++q) {
+        bool has;
+        uint2 cv = make_uint2(0u, 0u);
+        if (q < KL) {
+          const int nc = q < jn ? (int)((cnt[q >> 2] >> (8 * (q & 3))) & 0xffu) : 0;
+          total += nc;
+          has = nc > 0;
+          if (has) cv = cand[q * kBT + t];
+        } else {
+          has = q - KL < np;
+          if (has) cv = pool[(q - KL) * kBT + t];
         }
-        // -0 and +0 are equal in routing order: both take the key of +0.  Empty slots take
-        // key 0, below every real value, so they never outrank a candidate.
-        uint32_t o[NC], e[NC];
-        int total = 0;
+        o[q] = has ? ord_key(__uint_as_float(cv.x) + 0.f) : 0u;
+        e[q] = cv.y;
+      }
+      fb = (f & 1) || np > kPoolSlots || total < a.k;
+      if (hh == 0) {
+        fbmark[t] = fb ? 1 : 0;
+        if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
+      }
+      if (!fb) {
+        uint32_t top = 0u;
+#pragma unroll
+        for (int q = 0; q < NC; ++q) top = max(top, o[q]);
+        const float vtop = ord_inv(top);
 #pragma unroll
         for (int q = 0; q < NC; ++q) {
-          bool has;
-          uint2 cv = make_uint2(0u, 0u);
-          if (q < KL) {
-            const int nc = q < jn ? (int)((cnt[q >> 2] >> (8 * (q & 3))) & 0xffu) : 0;
-            total += nc;
-            has = nc > 0;
-            if (has) cv = cand[q * kBT + t];
-          } else {
-            has = q - KL < np;
-            if (has) cv = pool[(q - KL) * kBT + t];
-          }
-          o[q] = has ? ord_key(__uint_as_float(cv.x) + 0.f) : 0u;
-          e[q] = cv.y;
-        }
-        const bool fb = (f & 1) || np > kPoolSlots || total < a.k;
-        if (g == 0) {
-          fbmark[t] = fb ? 1 : 0;
-          if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
-        }
-        if (!fb) {
-          uint32_t top = 0u;
+          if ((q & 1) != hh || o[q] == 0u) continue;  // this thread's share; empty slots
+          int rank = 0;
 #pragma unroll
-          for (int q = 0; q < NC; ++q) top = max(top, o[q]);
-          const float vtop = ord_inv(top);
-          for (int q = g; q < NC; q += 4) {
-            uint2 cv = make_uint2(0u, 0u);
-            bool has;
-            if (q < KL) {
-              has = q < jn && pc[t * C::KLP + q] != 0;
-              if (has) cv = cand[q * kBT + t];
-            } else {
-              has = q - KL < np;
-              if (has) cv = pool[(q - KL) * kBT + t];
-            }
-            if (!has) continue;
-            const uint32_t om = ord_key(__uint_as_float(cv.x) + 0.f), em = cv.y;
-            int rank = 0;
-#pragma unroll
-            for (int j = 0; j < NC; ++j) rank += (o[j] > om || (o[j] == om && e[j] < em)) ? 1 : 0;
-            if (rank < a.k) {
-              const float v = ord_inv(om);
-              sidx[t * a.k + rank] = (int)em;
-              sex[t * a.k + rank] = expf(v - vtop);
-              slog[t * a.k + rank] = v;
-              if (em < (uint32_t)a.M) atomicAdd(a.out_count + em, 1);
-            }
+          for (int jj = 0; jj < NC; ++jj) rank += (o[jj] > o[q] || (o[jj] == o[q] && e[jj] < e[q])) ? 1 : 0;
+          if (rank < a.k) {
+            const float v = ord_inv(o[q]);
+            sidx[t * a.k + rank] = (int)e[q];
+            sex[t * a.k + rank] = expf(v - vtop);
+            slog[t * a.k + rank] = v;
+            if (e[q] < (uint32_t)a.M) atomicAdd(a.out_count + e[q], 1);
           }
         }
-      }
-      if (!consumer_sync(b, cph, a.status)) return;
-      // gates: each selected exp divided by its token's sum
-      if (g == 0 && (f & 2) == 0 && !fbmark[t]) {
-        float sum = 0.f;
-        for (int j = 0; j < a.k; ++j) sum += sex[t * a.k + j];
-        const float inv = 1.f / sum;
-        for (int j = 0; j < a.k; ++j) sex[t * a.k + j] *= inv;
-      }
-      if (!consumer_sync(b, cph, a.status)) return;
-      // the tile's outputs are contiguous: copy the staging out with coalesced stores
-      const int rows = a.N - n0 < kBT ? (int)(a.N - n0) : kBT;
-      const size_t ob = (size_t)n0 * a.k;
-      for (int x = ctid; x < rows * a.k; x += kConsumerThreads) {
-        if (fbmark[x / a.k]) continue;
-        a.out_idx[ob + x] = sidx[x];
-        a.out_gate[ob + x] = sex[x];
-        if (a.out_logits) a.out_logits[ob + x] = slog[x];
       }
     }
-    // fallback tokens, kFbBatch at a time: every consumer warp ranks its 256-expert blocks
-    // (blocks cw, cw + 16, ...) for each token, then warp j merges the 16 partial lists of
-    // the batch's token j and writes it
-    for (int fb0 = 0, nfb = *fbcount; fb0 < nfb; fb0 += kFbBatch) {
-      const int nb = nfb - fb0 < kFbBatch ? nfb - fb0 : kFbBatch;
-      fallback_rank<R, KCAP>(a, zs, fblist + fb0, nb, part, cw, lane);
-      if (!consumer_sync(b, cph, a.status)) return;
-      if (cw < nb) fallback_merge<KCAP>(a, part + cw * kConsumerWarps * KCAP, n0 + fblist[fb0 + cw], lane);
-      if (!consumer_sync(b, cph, a.status)) return;
+    group_bar(kNamedBarB);
+    // gates: each selected exp divided by its token's sum
+    if (hh == 0 && (f & 2) == 0 && !fb) {
+      float sum = 0.f;
+      for (int jj = 0; jj < a.k; ++jj) sum += sex[t * a.k + jj];
+      const float inv = 1.f / sum;
+      for (int jj = 0; jj < a.k; ++jj) sex[t * a.k + jj] *= inv;
+    }
+    group_bar(kNamedBarB);
+    // the tile's outputs are contiguous: copy the staging out with coalesced stores
+    const int rows = a.N - n0 < kBT ? (int)(a.N - n0) : kBT;
+    const size_t ob = (size_t)n0 * a.k;
+    for (int x = gt; x < rows * a.k; x += kGroupThreads) {
+      if (fbmark[x / a.k]) continue;
+      a.out_idx[ob + x] = sidx[x];
+      a.out_gate[ob + x] = sex[x];
+      if (a.out_logits) a.out_logits[ob + x] = slog[x];
+    }
+    // fallback tokens, kFbBatch at a time: every warp of the group ranks its 256-expert
+    // blocks (blocks bw, bw + 8, ...) for each token, then warp jj merges the 8 partial lists
+    // of the batch's token jj and writes it
+    const uint8_t* zs = zs0 + zs_buf(j, p.interleave) * C::ZS_BYTES;
+    const int nfb = *fbcount;
+    for (int fb0 = 0; fb0 < nfb; fb0 += kFbBatch) {
+      const int nbt = nfb - fb0 < kFbBatch ? nfb - fb0 : kFbBatch;
+      fallback_rank<R, KCAP>(a, zs, fblist + fb0, nbt, part, bw, lane);
+      group_bar(kNamedBarB);
+      if (bw < nbt) fallback_merge<KCAP>(a, part + bw * kGroupWarps * KCAP, n0 + fblist[fb0 + bw], lane);
+      group_bar(kNamedBarB);
+    }
+    // reset the per-tile counters for the next tile
+    if (hh == 0) poolcnt[t] = 0;
+    group_bar(kNamedBarB);  // every warp has read fbcount, the staging and the fallback lists
+    if (gt == 0) {
+      *fbcount = 0;
+      mbar_arrive(&b.pairs_empty[pb]);
+      mbar_arrive(&b.zsm_empty[zs_buf(j, p.interleave)]);  // the fallback is done with the z buffer
     }
   }
 }
@@ -957,20 +1047,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nr2 = p.r2_resident ? p.p_count : p.r2_stages;
     for (int i = 0; i < nr2; ++i) {
       mbar_init(&b.r2_full[i], 1);
-      mbar_init(&b.r2_empty[i], 1 + kConsumerWarps);  // the MMA commit and every consumer warp
+      // both logit issuers and group A's eight warps (the pass A issuer stands in for them
+      // after the first sweep)
+      mbar_init(&b.r2_empty[i], 2 + kGroupWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b.zacc_full[i], 1);
-      mbar_init(&b.zacc_empty[i], 8);
-      mbar_init(&b.drain[i], 1);
+      mbar_init(&b.zacc_empty[i], kGroupWarps);
+      mbar_init(&b.zsm_full[i], kGroupWarps);
+      mbar_init(&b.zsm_empty[i], 2);  // pass B MMAs done, finalize done
+      mbar_init(&b.a_full[i], 1);
+      mbar_init(&b.a_empty[i], kGroupWarps);
+      mbar_init(&b.b_full[i], 1);
+      mbar_init(&b.b_empty[i], kGroupWarps);
+      mbar_init(&b.pairs_full[i], 1);
+      mbar_init(&b.pairs_empty[i], 1);
+      mbar_init(&b.gbar[i], kGroupWarps);
     }
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(&b.d_full[i], 1);
-      mbar_init(&b.d_empty[i], kConsumerWarps);
-    }
-    mbar_init(b.zsm_full, 8);
-    mbar_init(b.zsm_empty, 1);
-    mbar_init(b.cbar, kConsumerWarps);
+    for (int i = 0; i < 3; ++i) mbar_init(&b.drain[i], 1);
     *b.abort_flag = 0;
     fence_mbar_init();
   }
@@ -983,9 +1077,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(b.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= 4) {  // clear the per-chunk pair counters
+  if (warp >= kWarpA0 && warp < kWarpB0) {  // clear the per-chunk pair counters
     int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
-    for (int i = threadIdx.x - 128; i < p.nchunks; i += kConsumerThreads) ccount[i] = 0;
+    for (int i = threadIdx.x - kWarpA0 * 32; i < p.nchunks; i += kGroupThreads) ccount[i] = 0;
+  }
+  if (warp >= kWarpB0) {  // clear the per-token pool counters and the fallback count
+    int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
+    const int i = threadIdx.x - kWarpB0 * 32;
+    if (i < kBT) poolcnt[i] = 0;
+    if (i == 0) *reinterpret_cast<int*>(smem + p.off_fb) = 0;
   }
   tc_fence_before();
   __syncthreads();
@@ -993,19 +1093,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *b.tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer_x<R, KCAP>(p, b, smem, &tmX, &tmR1);
+    if (lane == 0) producer<R, KCAP>(p, b, smem, &tmX, &tmR1, &tmR2);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) mma_z<R, KCAP>(p, b, smem, tmem_base);
     __syncwarp();
   } else if (warp == 2) {
-    if (lane == 0) mma_scores<R, KCAP>(p, b, smem, tmem_base);
+    if (lane == 0) mma_pass<R, KCAP, false>(p, b, smem, tmem_base);
     __syncwarp();
   } else if (warp == 3) {
-    if (lane == 0) producer_r2<R, KCAP>(p, b, smem, &tmR2);
+    if (lane == 0) mma_pass<R, KCAP, true>(p, b, smem, tmem_base);
     __syncwarp();
+  } else if (warp < kWarpB0) {
+    group_a<R, KCAP>(p, b, smem, tmem_base);
   } else {
-    consumers<R, KCAP>(p, b, smem, tmem_base);
+    group_b<R, KCAP>(p, b, smem, tmem_base);
   }
 
   tc_fence_before();
@@ -1047,71 +1149,96 @@ constexpr uint32_t kSmemLimit = 227 * 1024;
 
 uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Shared-memory plan; returns the total bytes (0 when nothing fits).
+// Shared-memory layout for xs X stages, r2n R2 stages (all p_count when resident) and nz z
+// buffers; returns the total bytes.
+template <int R, int KCAP>
+uint32_t layout(Params& p, int xs, int r2n, int nz) {
+  using C = Cfg<R, KCAP>;
+  uint32_t off = 0;
+  p.off_x = off;
+  off += xs * C::X_STAGE;
+  p.off_r1 = off = align_up(off, 1024);
+  off += xs * C::R1_STAGE;
+  p.off_r2 = off = align_up(off, 1024);
+  off += r2n * C::R2_STAGE;
+  p.off_zs = off = align_up(off, 1024);
+  off += nz * C::ZS_BYTES;
+  // group A: list exchange, later the (chunk, rank) stage of the needed pairs
+  p.off_lists = off = align_up(off, 16);
+  off += C::KL * kBT * 4;
+  p.off_ccount = off;
+  off += p.nchunks * 4;
+  p.off_scan = off = align_up(off, 16);
+  off += kGroupWarps * 4;
+  p.off_znorm = off;  // per token: |z_hi|^2 and |z_lo|^2 partial sums of both halves
+  off += 4 * kBT * 4;
+  p.off_cnorm = off;  // per warp: max squared column norm of R2; [8] = the result
+  off += (kGroupWarps + 1) * 4;
+  // group A -> group B, two buffers each; in the finalize a pair buffer holds the output
+  // staging
+  p.off_pairs = off = align_up(off, 16);
+  off += 2 * C::PAIR_BYTES;
+  p.off_cbase = off;
+  off += 2 * (p.nchunks + 1) * 4;
+  p.off_flag = off;
+  off += 2 * kBT;
+  p.off_nq = off;
+  off += 2 * kBT;
+  // group B: candidate slots (later the output staging), counts, pool, fallback
+  p.off_cand = off = align_up(off, 16);
+  {
+    const uint32_t cand_bytes = kBT * C::KLP * 8, staging_bytes = 3 * kBT * KCAP * 4;
+    off += cand_bytes > staging_bytes ? cand_bytes : staging_bytes;
+  }
+  p.off_pc = off = align_up(off, 16);
+  off += kBT * C::KLP;
+  p.off_pool = off = align_up(off, 8);
+  off += kBT * kPoolSlots * 8;
+  p.off_poolcnt = off;
+  off += kBT * 4;
+  p.off_fb = off;  // fallback count, the tile's fallback tokens, per-token mark
+  off += 4 + 2 * kBT;
+  // the fallback's partial lists reuse the candidate slots: the finalize has read them by then
+  static_assert(kFbBatch * kGroupWarps * KCAP * 8 <= kBT * C::KLP * 8, "partial lists fit the slots");
+  p.off_part = p.off_cand;
+  p.off_bar = off = align_up(off, 8);
+  off += kBarBytes;
+  return off + 1024;  // alignment slack of the dynamic base
+}
+
+// Shared-memory plan; returns the total bytes (0 when nothing fits).  Preference order:
+// R2 resident (no streaming at all), then two z buffers (one R2 sweep per tile) with at
+// least 3 X stages, then one z buffer (two sweeps per tile); more X stages first.
 template <int R, int KCAP>
 uint32_t plan(Params& p) {
-  using C = Cfg<R, KCAP>;
-  for (int xs = 4; xs >= 2; --xs) {
-    for (int mode = 0; mode < 2; ++mode) {  // 0: R2 resident, 1: streamed
-      const int r2s = mode == 0 ? p.p_count : 8;
-      if (mode == 0 && p.p_count > 64) continue;
-      for (int r2n = r2s; r2n >= 2 || (mode == 0 && r2n == r2s); --r2n) {
-        uint32_t off = 0;
-        p.off_x = off;
-        off += xs * C::X_STAGE;
-        p.off_r1 = off = align_up(off, 1024);
-        off += xs * C::R1_STAGE;
-        p.off_r2 = off = align_up(off, 1024);
-        off += r2n * C::R2_STAGE;
-        p.off_zs = off = align_up(off, 1024);
-        off += C::ZS_BYTES;
-        // candidate slots and the list exchange + pair staging share memory (disjoint lifetimes)
-        // (and, after the finalize, the partial lists of the cooperative fallback)
-        const uint32_t cand_bytes = kBT * C::KLP * C::S * 8, list_bytes = 3 * kBT * C::KL * 4;
-        const uint32_t part_bytes = kFbBatch * kConsumerWarps * KCAP * 8;
-        uint32_t shared_bytes = cand_bytes > list_bytes ? cand_bytes : list_bytes;
-        if (part_bytes > shared_bytes) shared_bytes = part_bytes;
-        p.off_cand = p.off_lists = off = align_up(off, 16);
-        off += shared_bytes;
-        p.off_thr = off;
-        off += kBT * 4;
-        p.off_flag = off;
-        off += kBT * 4;
-        p.off_pairs = off = align_up(off, 16);  // pass-2 pairs; in the finalize, the output staging
-        {
-          const uint32_t pair_bytes = kBT * C::KL * 8, staging_bytes = 3 * kBT * KCAP * 4;
-          off += pair_bytes > staging_bytes ? pair_bytes : staging_bytes;
+  struct Try {
+    int nz, xs_min, r2_min;
+  };
+  if (p.p_count <= 64) {
+    for (int nz = 2; nz >= 1; --nz)
+      for (int xs = 4; xs >= 3; --xs) {
+        const uint32_t total = layout<R, KCAP>(p, xs, p.p_count, nz);
+        if (total <= kSmemLimit) {
+          p.x_stages = xs;
+          p.r2_stages = p.p_count;
+          p.r2_resident = 1;
+          p.interleave = nz == 2;
+          return total;
         }
-        p.off_ccount = off;
-        off += p.nchunks * 4;
-        p.off_cbase = off;
-        off += (p.nchunks + 1) * 4;
-        p.off_scan = off = align_up(off, 16);
-        off += kConsumerWarps * 4;
-        p.off_znorm = off;           // per token: |z_hi|^2 and |z_lo|^2 partial sums of both halves
-        off += 4 * kBT * 4;
-        p.off_cnorm = off;           // per consumer warp: max squared column norm of R2; [16] = result
-        off += (kConsumerWarps + 1) * 4;
-        p.off_nq = off;
-        off += kBT;
-        p.off_fb = off = align_up(off, 4);  // fallback count, the tile's fallback tokens, per-token mark
-        off += 4 + 2 * kBT;
-        p.off_poolcnt = off = align_up(off, 4);
-        off += kBT * 4;
-        p.off_pool = off = align_up(off, 8);
-        off += kBT * kPoolSlots * 8;
-        p.off_pc = off = align_up(off, 16);
-        off += kBT * C::KLP;
-        p.off_bar = off = align_up(off, 8);
-        off += kBarBytes;
-        const uint32_t total = off + 1024;  // alignment slack of the dynamic base
+      }
+  }
+  const Try tries[] = {{2, 3, 3}, {1, 2, 2}, {2, 2, 2}};
+  for (const Try& tr : tries) {
+    for (int xs = 4; xs >= tr.xs_min; --xs) {
+      for (int r2n = 8; r2n >= tr.r2_min; --r2n) {
+        const uint32_t total = layout<R, KCAP>(p, xs, r2n, tr.nz);
         if (total <= kSmemLimit) {
           p.x_stages = xs;
           p.r2_stages = r2n;
-          p.r2_resident = mode == 0;
+          p.r2_resident = 0;
+          p.interleave = tr.nz == 2;
           return total;
         }
-        if (mode == 0) break;
       }
     }
   }
@@ -1132,6 +1259,17 @@ bool fill_params(const RouteArgs& a, Params& p, uint32_t& smem) {
   return smem != 0;
 }
 
+// Raises the kernel's dynamic shared-memory limit once per device.
+template <int R, int KCAP>
+cudaError_t configure_once(int dev) {
+  static std::atomic<int> done[64] = {};
+  if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fused_route_kernel<R, KCAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemLimit);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev].store(1, std::memory_order_release);
+  return e;
+}
+
 template <int R, int KCAP>
 cudaError_t launch(const RouteArgs& a) {
   using C = Cfg<R, KCAP>;
@@ -1147,15 +1285,11 @@ cudaError_t launch(const RouteArgs& a) {
       !make_map(&tmR1, a.R1, (uint64_t)R, (uint64_t)a.h, C::R1_BOX, C::BK, r1sw) ||
       !make_map(&tmR2, a.R2, (uint64_t)a.M, (uint64_t)R, 64, R, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static int configured = 0;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fused_route_kernel<R, KCAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured = 1;
-  }
   int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = configure_once<R, KCAP>(dev);
+  if (e != cudaSuccess) return e;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   fused_route_kernel<R, KCAP><<<grid, kThreads, smem, a.stream>>>(tmX, tmR1, tmR2, p);
@@ -1181,7 +1315,7 @@ bool supports_r(const RouteArgs& a) {
 }  // namespace tc
 
 bool fused_tc_supports(const RouteArgs& a) {
-  // 65536 experts = 2048 chunks: the pair-count scan covers 4 chunks per consumer thread
+  // 65536 experts = 2048 chunks: the pair-count scan covers 8 chunks per group-A thread
   if (a.M > 65536 || a.k > 16 || a.N < 1 || a.N > 0x7fffffffLL - tc::kBT) return false;
   if (!tc::encode_fn()) return false;
   switch (a.r) {
