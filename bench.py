@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -52,11 +53,23 @@ WORKLOADS = {
 }
 METRIC = "routed tokens/s (fused low-rank router + top-k)"
 BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X, R1, R2)"
-# DRAM bytes (read + write) per token of the fused kernel, from the ncu capture summarised in
-# profiles/fused_route_kernel_prefill_r32_n65536.md (N = 65,536, scaled by tokens).  Only valid
-# while that kernel is unchanged; workloads without a capture report traffic null.
-NCU_TRAFFIC_PER_TOKEN = {"prefill_r32": (269.635072e6 + 8.524544e6) / 65536}
+# DRAM bytes (read + write) per token of the fused kernel, from one ncu capture at N = 65,536
+# (summarised under profiles/, scaled by tokens), keyed to the SHA-256 of the kernel source that
+# was captured: once route_tc.cu differs from that source the figure is stale and traffic is
+# reported null.  Workloads without a capture report traffic null.
+NCU_TRAFFIC = {}   # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
 L2_BYTES = 126 * 1024 * 1024
+
+
+def kernel_source_digest():
+    """SHA-256 of the fused kernel's source, or None where the source is not shipped."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "mixture_experts_rank_b200", "csrc",
+                        "route_tc.cu")
+    try:
+        with open(path, "rb") as f:
+            return hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
 
 
 def describe(name):
@@ -439,8 +452,10 @@ def main():
         kernel_ms = launch_ms if launch_ms is not None else ms
         achieved = x_bytes / (kernel_ms / 1e3) / 1e9
         traffic = None
-        if variant_used == "fused_tc" and args.workload in NCU_TRAFFIC_PER_TOKEN:
-            traffic = NCU_TRAFFIC_PER_TOKEN[args.workload] * N  # bytes per launch
+        if variant_used == "fused_tc" and args.workload in NCU_TRAFFIC:
+            per_token, digest = NCU_TRAFFIC[args.workload]
+            if kernel_source_digest() == digest:
+                traffic = per_token * N  # bytes per launch
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured"
                 else "fallback 6.65 TB/s",

@@ -64,11 +64,17 @@ using namespace sm100;
 constexpr int kBT = 128;        // tokens per tile (MMA M of Z and pass A, N of pass B)
 constexpr int kBE = 128;        // experts per logit tile
 constexpr int kRoleWarps = 4;
-constexpr int kGroupWarps = 8;  // warps of group A and of group B
-constexpr int kGroupThreads = kGroupWarps * 32;
-constexpr int kWarpA0 = kRoleWarps, kWarpB0 = kRoleWarps + kGroupWarps;
-constexpr int kThreads = (kRoleWarps + 2 * kGroupWarps) * 32;  // 640: five warps per SMSP, 96 registers
-constexpr int kNamedBarA = 1, kNamedBarB = 2;                  // bar.sync ids of the groups
+#ifndef MORE_GROUP_B_WARPS
+#define MORE_GROUP_B_WARPS 8
+#endif
+constexpr int kWarpsA = 8;                       // group A: two warps per TMEM lane group
+constexpr int kWarpsB = MORE_GROUP_B_WARPS;      // group B: kWarpsB / 4 warps per TMEM lane group
+constexpr int kThreadsA = kWarpsA * 32, kThreadsB = kWarpsB * 32;
+constexpr int kPerTokB = kWarpsB / 4;            // group B threads per token in the finalize
+constexpr int kWarpA0 = kRoleWarps, kWarpB0 = kRoleWarps + kWarpsA;
+constexpr int kThreads = (kRoleWarps + kWarpsA + kWarpsB) * 32;
+constexpr int kNamedBarA = 1, kNamedBarB = 2;    // bar.sync ids of the groups
+static_assert(kWarpsB % 4 == 0, "group B covers the four TMEM lane groups evenly");
 constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass B
 constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than one candidate
 constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
@@ -222,7 +228,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return wait_bar_slow(bar, parity, abort_flag, status);
 }
 
-// Bounded entry barrier of one group's eight warps (an mbarrier, so that a warp of the
+// Bounded entry barrier of one group's warps (an mbarrier, so that a warp of the
 // group that gave up elsewhere cannot leave the others waiting without limit).  `phase` is
 // the calling thread's parity of the barrier, flipped at every use.
 __device__ __forceinline__ bool group_enter(uint64_t* gbar, uint32_t& phase, volatile int* abort_flag,
@@ -234,10 +240,10 @@ __device__ __forceinline__ bool group_enter(uint64_t* gbar, uint32_t& phase, vol
   return ok;
 }
 
-// Named barrier of one group's 256 threads.  Used only between a group_enter and the end
-// of the same phase, where no thread waits on anything else.
-__device__ __forceinline__ void group_bar(int id) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kGroupThreads) : "memory");
+// Named barrier of one group's threads.  Used only between a group_enter and the end of the
+// same phase, where no thread waits on anything else.
+__device__ __forceinline__ void group_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Order-preserving map of fp32 onto uint32 and its inverse.
@@ -479,7 +485,7 @@ __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t
           mma_commit(&b.r2_empty[rs.i]);
         else
           mbar_arrive(&b.r2_empty[rs.i]);
-        if (!PASS_B && q > 0) mbar_arrive_count(&b.r2_empty[rs.i], kGroupWarps);  // for group A
+        if (!PASS_B && q > 0) mbar_arrive_count(&b.r2_empty[rs.i], kWarpsA);  // for group A
         rs.next(p.r2_stages);
       }
     }
@@ -658,10 +664,10 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     }
     if (first && gt == 0) {
       float m = 0.f;
-      for (int w = 0; w < kGroupWarps; ++w) m = fmaxf(m, cnorm[w]);
-      cnorm[kGroupWarps] = sqrtf(m) * (1.f + 0x1p-20f);  // max column norm of R2, rounded up
+      for (int w = 0; w < kWarpsA; ++w) m = fmaxf(m, cnorm[w]);
+      cnorm[kWarpsA] = sqrtf(m) * (1.f + 0x1p-20f);  // max column norm of R2, rounded up
     }
-    group_bar(kNamedBarA);  // the merge has read the exchanged lists; cnorm is final
+    group_bar(kNamedBarA, kThreadsA);  // the merge has read the exchanged lists; cnorm is final
     uint32_t* stage = lists;  // (chunk, rank) of each needed pair of token t
     float ccut = -INFINITY;   // candidates: exact logit >= ccut
     int needed = 0;
@@ -669,7 +675,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       const bool active = n0 + t < a.N;
       // Certified window: values from z_hi differ from the z_hi + z_lo values by at most
       // eps = |z_lo| cmax (Cauchy-Schwarz) plus a bound on fp32 accumulation differences.
-      const float cmax = cnorm[kGroupWarps];
+      const float cmax = cnorm[kWarpsA];
       const float zh = sqrtf(znorm[t] + znorm[kBT + t]);
       const float zl = sqrtf(znorm[2 * kBT + t] + znorm[3 * kBT + t]);
       const float eps = (zl * cmax) * (1.f + 0x1p-8f) + (float)R * 0x1p-20f * zh * cmax + 1e-30f;
@@ -702,7 +708,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       flag[t] = (uint8_t)f;
       nq[t] = (uint8_t)needed;
     }
-    group_bar(kNamedBarA);
+    group_bar(kNamedBarA, kThreadsA);
     // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty),
     // eight chunks per thread
     {
@@ -720,7 +726,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         if (lane >= d) incl += o;
       }
       if (lane == 31) scan[aw] = incl;
-      group_bar(kNamedBarA);
+      group_bar(kNamedBarA, kThreadsA);
       int before = incl - run;
       for (int w = 0; w < aw; ++w) before += scan[w];
 #pragma unroll
@@ -731,9 +737,9 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         before += vals[jj];
       }
       // the end of the last bucket (index nchunks lies past the 8 x 256 slots when nchunks == 2048)
-      if (gt == kGroupThreads - 1) cbase[p.nchunks] = before;
+      if (gt == kThreadsA - 1) cbase[p.nchunks] = before;
     }
-    group_bar(kNamedBarA);
+    group_bar(kNamedBarA, kThreadsA);
     if (hh == 0) {
       for (int i = 0; i < needed; ++i) {
         const uint32_t st = stage[i * kBT + t];
@@ -741,7 +747,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(ccut));
       }
     }
-    group_bar(kNamedBarA);  // the pairs are written; the stage area may be reused
+    group_bar(kNamedBarA, kThreadsA);  // the pairs are written; the stage area may be reused
     if (gt == 0) mbar_arrive(&b.pairs_full[pb]);
   }
 }
@@ -785,7 +791,7 @@ __device__ __forceinline__ void fallback_block(const RouteArgs& a, const float (
 }
 
 // The cooperative fallback's first step: this warp's partial top-k (over the 256-expert
-// blocks bw, bw + 8, ...) of each of the nb tokens in tok, written to part.
+// blocks bw, bw + kWarpsB, ...) of each of the nb tokens in tok, written to part.
 template <int R, int KCAP>
 __device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t* zs, const uint8_t* tok, int nb,
                                               uint2* part, int bw, int lane) {
@@ -797,21 +803,21 @@ __device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t*
       zr[q] = (32 * q + lane < R) ? zs_value<R, KCAP>(zs, tf, 32 * q + lane) : 0.f;
     TopList<KCAP> list;
     list.init();
-    for (int eb = 256 * bw; eb < a.M; eb += 256 * kGroupWarps) fallback_block<R, KCAP>(a, zr, eb, lane, list);
+    for (int eb = 256 * bw; eb < a.M; eb += 256 * kWarpsB) fallback_block<R, KCAP>(a, zr, eb, lane, list);
     float v;
     int e;
     warp_merge_topk<KCAP>(list, a.k, lane, v, e);
-    if (lane < KCAP) part[(j * kGroupWarps + bw) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
+    if (lane < KCAP) part[(j * kWarpsB + bw) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
   }
 }
 
-// The second step: merge the eight partial lists of one token (part: warp-major, KCAP
+// The second step: merge the partial lists of one token (part: warp-major, KCAP
 // entries each, the first k valid) and write the token's outputs.
 template <int KCAP>
 __device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* part, int64_t n, int lane) {
   TopList<KCAP> list;
   list.init();
-  for (int q = lane; q < kGroupWarps * KCAP; q += 32) {
+  for (int q = lane; q < kWarpsB * KCAP; q += 32) {
     const uint2 c = part[q];
     if ((q % KCAP) < a.k) list.insert_any(__uint_as_float(c.x), (int)c.y);
   }
@@ -828,10 +834,10 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
   constexpr int NC = KL + kPoolSlots;
   const RouteArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bw = warp - kWarpB0;        // 0..7
+  const int bw = warp - kWarpB0;        // 0 .. kWarpsB - 1
   const int sp = warp & 3;              // TMEM lane group: lanes 32 sp .. 32 sp + 31
-  const int hh = bw >> 2;               // which of the lane group's two warps
-  const int gt = bw * 32 + lane;        // 0..255
+  const int hh = bw >> 2;               // which of the lane group's kPerTokB warps
+  const int gt = bw * 32 + lane;        // 0 .. kThreadsB - 1
   const int t = sp * 32 + lane;         // token of this thread in the finalize
   const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
   uint8_t* zs0 = smem + p.off_zs;
@@ -857,15 +863,15 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     const uint8_t* nq = smem + p.off_nq + pb * kBT;
 
     // ---------------- pass B: candidates of the needed chunks (exact z_hi + z_lo logits) ----
-    // Lane group sp of the transposed tile is chunk 4 pt + sp; its two warps split the
-    // chunk's pairs in halves.
+    // Lane group sp of the transposed tile is chunk 4 pt + sp; its kPerTokB warps split the
+    // chunk's pairs.
     for (int pt = 0; pt < p.p_count; ++pt) {
       const int c = pt * 4 + sp;
       int lo = 0, hi = 0;
       if (c < p.nchunks) {
         const int c_lo = cbase[c], n = cbase[c + 1] - c_lo;
-        lo = c_lo + ((n * hh) >> 1);
-        hi = c_lo + ((n * (hh + 1)) >> 1);
+        lo = c_lo + (n * hh) / kPerTokB;
+        hi = c_lo + (n * (hh + 1)) / kPerTokB;
       }
       if (!wait_bar(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
@@ -917,10 +923,10 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     }
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
-    // Two threads per token (the lane group's two warps).  Every thread loads all of the
+    // kPerTokB threads per token (the lane group's warps).  Every thread loads all of the
     // token's candidates (the slots of its needed chunks, then its pool entries) into
-    // registers; thread hh ranks candidates hh, hh + 2, ... in routing order (larger logit,
-    // then lower expert) and the ones of rank < k go to the output staging at their rank,
+    // registers; thread hh ranks candidates hh, hh + kPerTokB, ... in routing order (larger
+    // logit, then lower expert) and the ones of rank < k go to the output staging at their rank,
     // with exp(logit - max).  The staging reuses the tile's pair buffer, which pass B has
     // finished reading.
     if (!group_enter(&b.gbar[1], gph, b.abort_flag, a.status)) return;
@@ -973,7 +979,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         const float vtop = ord_inv(top);
 #pragma unroll
         for (int q = 0; q < NC; ++q) {
-          if ((q & 1) != hh || o[q] == 0u) continue;  // this thread's share; empty slots
+          if ((q % kPerTokB) != hh || o[q] == 0u) continue;  // this thread's share; empty slots
           int rank = 0;
 #pragma unroll
           for (int jj = 0; jj < NC; ++jj) rank += (o[jj] > o[q] || (o[jj] == o[q] && e[jj] < e[q])) ? 1 : 0;
@@ -987,7 +993,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         }
       }
     }
-    group_bar(kNamedBarB);
+    group_bar(kNamedBarB, kThreadsB);
     // gates: each selected exp divided by its token's sum
     if (hh == 0 && (f & 2) == 0 && !fb) {
       float sum = 0.f;
@@ -995,31 +1001,31 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       const float inv = 1.f / sum;
       for (int jj = 0; jj < a.k; ++jj) sex[t * a.k + jj] *= inv;
     }
-    group_bar(kNamedBarB);
+    group_bar(kNamedBarB, kThreadsB);
     // the tile's outputs are contiguous: copy the staging out with coalesced stores
     const int rows = a.N - n0 < kBT ? (int)(a.N - n0) : kBT;
     const size_t ob = (size_t)n0 * a.k;
-    for (int x = gt; x < rows * a.k; x += kGroupThreads) {
+    for (int x = gt; x < rows * a.k; x += kThreadsB) {
       if (fbmark[x / a.k]) continue;
       a.out_idx[ob + x] = sidx[x];
       a.out_gate[ob + x] = sex[x];
       if (a.out_logits) a.out_logits[ob + x] = slog[x];
     }
     // fallback tokens, kFbBatch at a time: every warp of the group ranks its 256-expert
-    // blocks (blocks bw, bw + 8, ...) for each token, then warp jj merges the 8 partial lists
-    // of the batch's token jj and writes it
+    // blocks (blocks bw, bw + kWarpsB, ...) for each token, then warp jj merges the partial
+    // lists of the batch's token jj and writes it
     const uint8_t* zs = zs0 + zs_buf(j, p.interleave) * C::ZS_BYTES;
     const int nfb = *fbcount;
     for (int fb0 = 0; fb0 < nfb; fb0 += kFbBatch) {
       const int nbt = nfb - fb0 < kFbBatch ? nfb - fb0 : kFbBatch;
       fallback_rank<R, KCAP>(a, zs, fblist + fb0, nbt, part, bw, lane);
-      group_bar(kNamedBarB);
-      if (bw < nbt) fallback_merge<KCAP>(a, part + bw * kGroupWarps * KCAP, n0 + fblist[fb0 + bw], lane);
-      group_bar(kNamedBarB);
+      group_bar(kNamedBarB, kThreadsB);
+      if (bw < nbt) fallback_merge<KCAP>(a, part + bw * kWarpsB * KCAP, n0 + fblist[fb0 + bw], lane);
+      group_bar(kNamedBarB, kThreadsB);
     }
     // reset the per-tile counters for the next tile
     if (hh == 0) poolcnt[t] = 0;
-    group_bar(kNamedBarB);  // every warp has read fbcount, the staging and the fallback lists
+    group_bar(kNamedBarB, kThreadsB);  // every warp has read fbcount, the staging and the fallback lists
     if (gt == 0) {
       *fbcount = 0;
       mbar_arrive(&b.pairs_empty[pb]);
@@ -1049,20 +1055,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&b.r2_full[i], 1);
       // both logit issuers and group A's eight warps (the pass A issuer stands in for them
       // after the first sweep)
-      mbar_init(&b.r2_empty[i], 2 + kGroupWarps);
+      mbar_init(&b.r2_empty[i], 2 + kWarpsA);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b.zacc_full[i], 1);
-      mbar_init(&b.zacc_empty[i], kGroupWarps);
-      mbar_init(&b.zsm_full[i], kGroupWarps);
+      mbar_init(&b.zacc_empty[i], kWarpsA);
+      mbar_init(&b.zsm_full[i], kWarpsA);
       mbar_init(&b.zsm_empty[i], 2);  // pass B MMAs done, finalize done
       mbar_init(&b.a_full[i], 1);
-      mbar_init(&b.a_empty[i], kGroupWarps);
+      mbar_init(&b.a_empty[i], kWarpsA);
       mbar_init(&b.b_full[i], 1);
-      mbar_init(&b.b_empty[i], kGroupWarps);
+      mbar_init(&b.b_empty[i], kWarpsB);
       mbar_init(&b.pairs_full[i], 1);
       mbar_init(&b.pairs_empty[i], 1);
-      mbar_init(&b.gbar[i], kGroupWarps);
+      mbar_init(&b.gbar[i], i == 0 ? kWarpsA : kWarpsB);
     }
     for (int i = 0; i < 3; ++i) mbar_init(&b.drain[i], 1);
     *b.abort_flag = 0;
@@ -1079,7 +1085,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp >= kWarpA0 && warp < kWarpB0) {  // clear the per-chunk pair counters
     int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
-    for (int i = threadIdx.x - kWarpA0 * 32; i < p.nchunks; i += kGroupThreads) ccount[i] = 0;
+    for (int i = threadIdx.x - kWarpA0 * 32; i < p.nchunks; i += kThreadsA) ccount[i] = 0;
   }
   if (warp >= kWarpB0) {  // clear the per-token pool counters and the fallback count
     int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
@@ -1169,11 +1175,11 @@ uint32_t layout(Params& p, int xs, int r2n, int nz) {
   p.off_ccount = off;
   off += p.nchunks * 4;
   p.off_scan = off = align_up(off, 16);
-  off += kGroupWarps * 4;
+  off += kWarpsA * 4;
   p.off_znorm = off;  // per token: |z_hi|^2 and |z_lo|^2 partial sums of both halves
   off += 4 * kBT * 4;
   p.off_cnorm = off;  // per warp: max squared column norm of R2; [8] = the result
-  off += (kGroupWarps + 1) * 4;
+  off += (kWarpsA + 1) * 4;
   // group A -> group B, two buffers each; in the finalize a pair buffer holds the output
   // staging
   p.off_pairs = off = align_up(off, 16);
@@ -1199,7 +1205,7 @@ uint32_t layout(Params& p, int xs, int r2n, int nz) {
   p.off_fb = off;  // fallback count, the tile's fallback tokens, per-token mark
   off += 4 + 2 * kBT;
   // the fallback's partial lists reuse the candidate slots: the finalize has read them by then
-  static_assert(kFbBatch * kGroupWarps * KCAP * 8 <= kBT * C::KLP * 8, "partial lists fit the slots");
+  static_assert(kFbBatch * kWarpsB * KCAP * 8 <= kBT * C::KLP * 8, "partial lists fit the slots");
   p.off_part = p.off_cand;
   p.off_bar = off = align_up(off, 8);
   off += kBarBytes;
