@@ -8,7 +8,8 @@ workload: prefill, N = 262,144 tokens (256 sequences x 1024), h = 2048, M = 4096
 r = 32, k = 8, X rows at unit RMS, R1 ~ N(0, 1/h), R2 ~ N(0, 1/r), seed 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--variant auto|fused_tc|small_n|cluster|unfused|train|dispatch|dispatch_shared|backward]
+                  [--variant auto|fused_tc|small_n|cluster|unfused|unfused_tc|train|dispatch|
+                             dispatch_shared|backward]
                   [--workload NAME]
 
 Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank routes its own
@@ -50,6 +51,11 @@ WORKLOADS = {
     "decode_N8": (8, 2048, 32, 4096, 8, False),
     "decode_N64": (64, 2048, 32, 4096, 8, False),
     "decode_N256": (256, 2048, 32, 4096, 8, False),
+    # fused vs unfused against the batch (App. H.6, Fig. 24): N = B x 1024, h = 2048, M = 4096, r = 16, k = 4
+    "fig24_B2": (2048, 2048, 16, 4096, 4, True),
+    "fig24_B16": (16384, 2048, 16, 4096, 4, True),
+    "fig24_B64": (65536, 2048, 16, 4096, 4, True),
+    "fig24_B256": (262144, 2048, 16, 4096, 4, True),
 }
 METRIC = "routed tokens/s (fused low-rank router + top-k)"
 BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X, R1, R2)"
@@ -57,7 +63,10 @@ BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X,
 # (summarised under profiles/, scaled by tokens), keyed to the SHA-256 of the kernel source that
 # was captured: once route_tc.cu differs from that source the figure is stale and traffic is
 # reported null.  Workloads without a capture report traffic null.
-NCU_TRAFFIC = {}   # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
+NCU_TRAFFIC = {    # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
+    "prefill_r32": ((269225728 + 5350912) / 65536,
+                    "befaa7c6efe03d8fd0009787ce44721960f9f4b126fb1a7f017c051db2454282"),
+}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -266,7 +275,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto",
-                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "train", "dispatch", "dispatch_shared",
+                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "unfused_tc", "train", "dispatch", "dispatch_shared",
                              "backward"],
                     help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum); "
                          "dispatch: routing followed by more_dispatch of its indices (dispatch_shared: with the "
@@ -325,7 +334,7 @@ def main():
         d_scratch = torch.empty(max(more.dispatch_scratch_bytes(N, k, M), 16), dtype=torch.uint8, device="cuda")
         d_off = torch.empty((M + 1,), dtype=torch.int32, device="cuda")
         d_sorted = torch.empty((N * k,), dtype=torch.int32, device="cuda")
-    if args.variant == "unfused":
+    if args.variant in ("unfused", "unfused_tc"):
         scratch = torch.empty(more.unfused_scratch_bytes(N, r, M), dtype=torch.uint8, device="cuda")
     if args.variant == "backward":
         # the forward's selections and statistics (untimed), seeded incoming gradients
@@ -359,6 +368,9 @@ def main():
         elif args.variant == "unfused":
             more.route_unfused(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate, out_expert_count=cnt,
                                out_logits=logits, stream=st)
+        elif args.variant == "unfused_tc":
+            more.route_unfused_tc(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate,
+                                  out_expert_count=cnt, out_logits=logits, stream=st)
         else:
             more.route(X, R1, R2, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
                        variant=args.variant, stream=st)
@@ -371,7 +383,7 @@ def main():
         except more.MoreError:
             variant_used = "small_n"
         variant_used = variant_used if N >= 512 else "small_n"
-    launches_per_step = {"unfused": 3, "train": 2, "dispatch": 5, "dispatch_shared": 5,
+    launches_per_step = {"unfused": 3, "unfused_tc": 2, "train": 2, "dispatch": 5, "dispatch_shared": 5,
                          "backward": 5}.get(args.variant, 1)
 
     def barrier():

@@ -112,6 +112,22 @@ more_status more_route_unfused(const void* X, const void* R1, const void* R2, in
                                size_t scratch_bytes, void* stream);
 
 /*
+ * The materialise-then-top-k comparison on the tensor cores (MoRE App. H.6, Fig. 24, with
+ * the fused kernel's products): z = X . R1 accumulated in TMEM and narrowed to the bf16
+ * pair, then the exact logits of every 128-expert tile as one tcgen05 product of K = 2r,
+ * written to the fp32 [N][M] scores in scratch by TMA tile stores; the row-wise top-k and
+ * softmax of more_route_unfused read them back.  The scores differ from the fused kernel's
+ * only in being written out, so the two calls time the HBM round trip of the N x M tensor.
+ * Same arguments, scratch size (more_route_unfused_scratch_bytes; the z area is unused)
+ * and results as more_route_unfused.  r must be 16, 32, 64 or 128, else
+ * MORE_ERR_UNSUPPORTED.
+ */
+more_status more_route_unfused_tc(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                                  int M, int k, int32_t* out_idx, float* out_gate,
+                                  int32_t* out_expert_count, float* out_logits, void* scratch,
+                                  size_t scratch_bytes, void* stream);
+
+/*
  * more_route_unfused with no scratch argument: its scratch is a fixed array of
  * MORE_STATIC_SCRATCH_BYTES bytes inside the library, so the call allocates
  * nothing.  This entry point has no counterpart in the MoRE paper; it is for

@@ -21,7 +21,7 @@ import torch
 from . import _build
 
 __all__ = ["route", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
-           "dispatch_scratch_bytes", "route_unfused", "route_unfused_static", "unfused_scratch_bytes", "device_status",
+           "dispatch_scratch_bytes", "route_unfused", "route_unfused_tc", "route_unfused_static", "unfused_scratch_bytes", "device_status",
            "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
 KMAX = 16
@@ -49,6 +49,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_variant.argtypes = route_args + [I, P]
     lib.more_route_unfused.restype = I
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
+    lib.more_route_unfused_tc.restype = I
+    lib.more_route_unfused_tc.argtypes = route_args + [P, ctypes.c_size_t, P]
     lib.more_route_unfused_static.restype = I
     lib.more_route_unfused_static.argtypes = route_args + [P]
     lib.more_dispatch_scratch_bytes.restype = ctypes.c_size_t
@@ -271,6 +273,24 @@ def route_unfused(X, R1, R2, k: int, *, scratch: torch.Tensor | None = None, out
                                  _ptr(outs[2]), _ptr(outs[3]), _ptr(scratch), scratch.numel(),
                                  _stream_handle(stream))
     _check(st, "more_route_unfused")
+    return outs
+
+
+def route_unfused_tc(X, R1, R2, k: int, *, scratch: torch.Tensor | None = None, out_idx=None, out_gate=None,
+                     out_expert_count=None, out_logits=None, return_logits: bool = True, stream=None):
+    """The materialise-then-top-k comparison with the scores written by the fused kernel's
+    tensor-core products (``more_route_unfused_tc``); same results as :func:`route`."""
+    X, R1, R2 = _as_bf16(X, "X"), _as_bf16(R1, "R1"), _as_bf16(R2, "R2")
+    N, h = X.shape
+    r, M = R2.shape
+    need = unfused_scratch_bytes(N, r, M)
+    if scratch is None:
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    outs = _outputs(N, k, M, X.device, out_idx, out_gate, out_expert_count, out_logits, return_logits)
+    st = _lib.more_route_unfused_tc(_ptr(X), _ptr(R1), _ptr(R2), N, h, r, M, k, _ptr(outs[0]), _ptr(outs[1]),
+                                    _ptr(outs[2]), _ptr(outs[3]), _ptr(scratch), scratch.numel(),
+                                    _stream_handle(stream))
+    _check(st, "more_route_unfused_tc")
     return outs
 
 

@@ -247,6 +247,26 @@ more_status more_route_unfused(const void* X, const void* R1, const void* R2, in
   return launch_unfused(a, scratch) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
 }
 
+more_status more_route_unfused_tc(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                                  int M, int k, int32_t* out_idx, float* out_gate,
+                                  int32_t* out_expert_count, float* out_logits, void* scratch,
+                                  size_t scratch_bytes, void* stream) {
+  more_status st = validate_route(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  if (st != MORE_OK) return st;
+  if (r != 16 && r != 32 && r != 64 && r != 128) return MORE_ERR_UNSUPPORTED;
+  if (N > 0 && (!scratch || !aligned16(scratch) || scratch_bytes < unfused_scratch_bytes(N, r, M)))
+    return MORE_ERR_INVALID_ARG;
+  RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
+                          stream);
+  a.status = status_word();
+  if (!a.status) return MORE_ERR_CUDA;
+  if (N > 0 && !unfused_tc_supports(a)) return MORE_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
+    return MORE_ERR_CUDA;
+  if (N == 0) return MORE_OK;
+  return launch_unfused_tc(a, scratch) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
 more_status more_device_status(void* stream, uint32_t* detail) {
   if (detail) *detail = 0;
   unsigned int* word = status_word();

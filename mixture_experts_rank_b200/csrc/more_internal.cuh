@@ -65,6 +65,16 @@ cudaError_t launch_fused_tc(const RouteArgs& a);
 bool fused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused(const RouteArgs& a, void* scratch);
 size_t unfused_scratch_bytes(int64_t N, int r, int M);
+// The fp32 [N][M] score tensor inside an unfused scratch buffer (after the z area).
+float* unfused_scores_of(void* scratch, int64_t N, int r);
+// Row-wise top-k and softmax over materialised scores: per-lane running lists (the CUDA-core
+// unfused path), and a running list filtered by its k-th value (the tensor-core unfused path).
+cudaError_t launch_scores_topk(const RouteArgs& a, const float* scores);
+cudaError_t launch_threshold_topk(const RouteArgs& a, const float* scores);
+// Tensor-core materialisation of the scores (same products as the fused kernel), then the
+// row-wise top-k; scratch as for launch_unfused.
+bool unfused_tc_supports(const RouteArgs& a);
+cudaError_t launch_unfused_tc(const RouteArgs& a, void* scratch);
 
 // ---- small device helpers -------------------------------------------------
 

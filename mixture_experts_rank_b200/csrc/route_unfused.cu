@@ -119,13 +119,35 @@ size_t unfused_scratch_bytes(int64_t N, int r, int M) {
   return align_up((size_t)N * r * sizeof(float), 256) + (size_t)N * M * sizeof(float);
 }
 
+float* unfused_scores_of(void* scratch, int64_t N, int r) {
+  return reinterpret_cast<float*>(static_cast<char*>(scratch) + align_up((size_t)N * r * sizeof(float), 256));
+}
+
+cudaError_t launch_scores_topk(const RouteArgs& a, const float* scores) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t tblocks = (a.N + kTopkWarps - 1) / kTopkWarps;
+  if (tblocks > (int64_t)sms * 16) tblocks = (int64_t)sms * 16;
+  switch (a.k) {
+#define MORE_CASE(K) \
+  case K:            \
+    return launch_topk<K>(a, scores, (int)tblocks);
+    MORE_CASE(1) MORE_CASE(2) MORE_CASE(3) MORE_CASE(4) MORE_CASE(5) MORE_CASE(6) MORE_CASE(7)
+    MORE_CASE(8) MORE_CASE(9) MORE_CASE(10) MORE_CASE(11) MORE_CASE(12) MORE_CASE(13)
+    MORE_CASE(14) MORE_CASE(15) MORE_CASE(16)
+#undef MORE_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_unfused(const RouteArgs& a, void* scratch) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   auto* z = static_cast<float*>(scratch);
-  auto* scores = reinterpret_cast<float*>(static_cast<char*>(scratch) +
-                                          align_up((size_t)a.N * a.r * sizeof(float), 256));
+  float* scores = unfused_scores_of(scratch, a.N, a.r);
   int64_t pblocks = (a.N + kProjWarps - 1) / kProjWarps;
   if (pblocks > (int64_t)sms * 8) pblocks = (int64_t)sms * 8;
   unfused_projection_kernel<<<(unsigned)pblocks, kProjWarps * 32, sizeof(float) * kProjWarps * a.r, a.stream>>>(
@@ -141,19 +163,7 @@ cudaError_t launch_unfused(const RouteArgs& a, void* scratch) {
   unfused_scores_kernel<<<grid, 256, smem, a.stream>>>(z, a.R2, a.N, a.r, a.M, scores);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  int64_t tblocks = (a.N + kTopkWarps - 1) / kTopkWarps;
-  if (tblocks > (int64_t)sms * 16) tblocks = (int64_t)sms * 16;
-  switch (a.k) {
-#define MORE_CASE(K) \
-  case K:            \
-    return launch_topk<K>(a, scores, (int)tblocks);
-    MORE_CASE(1) MORE_CASE(2) MORE_CASE(3) MORE_CASE(4) MORE_CASE(5) MORE_CASE(6) MORE_CASE(7)
-    MORE_CASE(8) MORE_CASE(9) MORE_CASE(10) MORE_CASE(11) MORE_CASE(12) MORE_CASE(13)
-    MORE_CASE(14) MORE_CASE(15) MORE_CASE(16)
-#undef MORE_CASE
-    default:
-      return cudaErrorInvalidValue;
-  }
+  return launch_scores_topk(a, scores);
 }
 
 }  // namespace more

@@ -26,7 +26,8 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
 CSRC = os.path.join(ROOT, "mixture_experts_rank_b200", "csrc")
-KERNELS = ("backward.cu", "route_cluster.cu", "route_small.cu", "dispatch.cu", "route_unfused.cu")
+KERNELS = ("backward.cu", "route_cluster.cu", "route_small.cu", "dispatch.cu", "route_unfused.cu",
+           "route_scores_topk.cu")
 
 
 def _split_top(s: str) -> list[str]:
@@ -152,6 +153,8 @@ class Emulated:
         lib.emu_unfused_scratch_bytes.argtypes = [I64, I, I]
         lib.emu_route_unfused.restype = I
         lib.emu_route_unfused.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, P, P, P]
+        lib.emu_threshold_topk.restype = I
+        lib.emu_threshold_topk.argtypes = [P, I64, I, I, P, P, P, P, P]
         lib.emu_train_stats.restype = I
         lib.emu_train_stats.argtypes = [P, P, P, I64, I, I, I, P, P, P, P]
         lib.emu_dispatch_scratch_bytes.restype = ctypes.c_long

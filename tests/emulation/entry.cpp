@@ -94,6 +94,12 @@ extern "C" int emu_route_unfused(const void* X, const void* R1, const void* R2, 
   return (int)more::launch_unfused(route_args(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, status), scratch);
 }
 
+extern "C" int emu_threshold_topk(const float* scores, int64_t N, int M, int k, int32_t* idx, float* gate,
+                                  int32_t* cnt, float* logits, unsigned* status) {
+  return (int)more::launch_threshold_topk(
+      route_args(nullptr, nullptr, nullptr, N, 8, 16, M, k, idx, gate, cnt, logits, status), scores);
+}
+
 extern "C" int emu_train_stats(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
                                float* out_m, float* out_Z, float* out_psum, unsigned* status) {
   memset(out_psum, 0, sizeof(float) * M);

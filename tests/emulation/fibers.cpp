@@ -98,6 +98,17 @@ void* shared_static_bytes(int id, size_t bytes) {
   }
   return v.data();
 }
+unsigned ballot(int p) {
+  const int me = cur;
+  xbuf[me] = p ? 1 : 0;
+  (void)wait_on(warp_bar[me / 32], 32, 0);
+  unsigned mask = 0;
+  for (int l = 0; l < 32; ++l)
+    if (xbuf[(me & ~31) | l]) mask |= 1u << l;
+  (void)wait_on(warp_bar[me / 32], 32, 0);
+  return mask;
+}
+int lane_id() { return cur & 31; }
 unsigned match_any(unsigned long long v) {
   const int me = cur;
   xbuf[me] = v;

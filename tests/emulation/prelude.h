@@ -32,6 +32,12 @@ float4* smem();
 void* shared_static_bytes(int id, size_t bytes);
 template <class T> T& shared_static(int id) { return *static_cast<T*>(shared_static_bytes(id, sizeof(T))); }
 unsigned match_any(unsigned long long v);
+unsigned ballot(int p);
+int lane_id();
+template <class T> T shfl_up(unsigned, T v, int d) {
+  const int lane = lane_id();
+  uint64_t b = 0; memcpy(&b, &v, sizeof(T)); b = xchg(b, lane >= d ? lane - d : lane, false); T r; memcpy(&r, &b, sizeof(T)); return r;
+}
 void launch(dim3 grid, dim3 block, size_t smem_bytes, std::function<void()> body);
 }
 namespace cooperative_groups {
@@ -51,6 +57,8 @@ inline cluster_group this_cluster() { return {}; }
 #define __syncwarp(...) ::emu::syncwarp()
 #define __shfl_xor_sync(m, v, l) ::emu::shfl_xor(m, v, l)
 #define __shfl_sync(m, v, l) ::emu::shfl(m, v, l)
+#define __shfl_up_sync(m, v, d) ::emu::shfl_up(m, v, d)
+#define __ballot_sync(m, p) ::emu::ballot((p) ? 1 : 0)
 #define __ldg(p) (*(p))
 #define __ldcs(p) (*(p))
 #define __popc(x) __builtin_popcount(x)

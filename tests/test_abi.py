@@ -29,7 +29,7 @@ def lib():
 def test_header_declares_the_route_entry_points():
     names = declared_functions()
     for required in ("more_route", "more_route_variant", "more_route_train", "more_route_backward",
-                     "more_route_backward_scratch_bytes", "more_route_unfused",
+                     "more_route_backward_scratch_bytes", "more_route_unfused", "more_route_unfused_tc",
                      "more_route_unfused_scratch_bytes", "more_device_status", "more_status_string",
                      "more_abi_version"):
         assert required in names
@@ -75,6 +75,18 @@ def test_unfused_scratch_size_and_checks(lib):
     st = lib.more_route_unfused(P(16), P(16), P(16), 1000, 64, 32, 256, 4, P(16), P(16), P(16), None, P(16),
                                 n - 1, None)
     assert st == 1
+
+
+def test_unfused_tc_checks_rank_and_scratch(lib):
+    """The tensor-core materialisation takes r in {16, 32, 64, 128} and the unfused scratch size."""
+    n = lib.more_route_unfused_scratch_bytes(1000, 32, 256)
+    P = ctypes.c_void_p
+    args = lambda r, nbytes: (P(16), P(16), P(16), 1000, 64, r, 256, 4, P(16), P(16), P(16), None, P(16), nbytes,
+                              None)
+    assert lib.more_route_unfused_tc(*args(32, n - 1)) == 1
+    assert lib.more_route_unfused_tc(*args(48, 1 << 30)) == 2
+    assert lib.more_route_unfused_tc(*args(96, 1 << 30)) == 2
+    assert lib.more_route_unfused_tc(*args(24, 1 << 30)) == 2   # not a multiple of 16: outside every path
 
 
 @pytest.mark.parametrize("kwargs,expected", [

@@ -16,6 +16,8 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 VARIANTS = ["small_n", "fused_tc"]
+UNFUSED = ["unfused", "unfused_tc"]   # materialise-then-top-k: CUDA-core and tensor-core scores
+TC_RANKS = (16, 32, 64, 128)          # ranks of the tensor-core kernels
 
 _cache = {}
 
@@ -41,6 +43,8 @@ def lib():
 
 def supported(variant, N, h, r, M, k):
     m = lib()
+    if variant == "unfused_tc":
+        return r in TC_RANKS
     if variant == "fused_tc":
         try:
             X = torch.zeros((max(N, 1), h), dtype=torch.bfloat16, device="cuda")
@@ -57,6 +61,8 @@ def run(variant, Xd, R1d, R2d, k):
     m = lib()
     if variant == "unfused":
         out = m.route_unfused(Xd, R1d, R2d, k)
+    elif variant == "unfused_tc":
+        out = m.route_unfused_tc(Xd, R1d, R2d, k)
     else:
         out = m.route(Xd, R1d, R2d, k, variant=variant)
     torch.cuda.synchronize()
@@ -86,13 +92,13 @@ def check(variant, N, h, r, M, k, seed=0, unit_rms=False, n_sample=None, near_sc
 
 # --- the benchmark workloads --------------------------------------------------------
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 def test_tiny_full_oracle(variant):
     rep = check(variant, 4096, 128, 32, 192, 4)
     assert rep.set_fraction > 0.8
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 @pytest.mark.parametrize("M", [1024, 2048, 4096, 8192, 16384])
 def test_expert_sweep_sampled(variant, M):
     check(variant, 65536, 512, 32, M, 8, n_sample=4096, near_scan=16384, near_count=256)
@@ -110,12 +116,18 @@ def test_prefill_unfused_sampled():
     check("unfused", 262144, 2048, 32, 4096, 8, unit_rms=True, n_sample=256)
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("r", [16, 32, 64, 128])
+def test_prefill_unfused_tc_sampled(r):
+    check("unfused_tc", 262144, 2048, r, 4096, 8, unit_rms=True, n_sample=4096,
+          near_scan=32768, near_count=256)
+
+
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 def test_many_experts_sampled(variant):
     check(variant, 32768, 4096, 64, 65536, 8, n_sample=1024, near_scan=4096, near_count=128)
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 @pytest.mark.parametrize("N", [1, 8, 64, 256])
 def test_decode_full_oracle(variant, N):
     check(variant, N, 2048, 32, 4096, 8)
@@ -123,7 +135,7 @@ def test_decode_full_oracle(variant, N):
 
 # --- ragged and degenerate shapes ------------------------------------------------------
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 @pytest.mark.parametrize("N,h,r,M,k", [
     (127, 72, 16, 200, 1),
     (129, 136, 48, 64, 8),
@@ -136,7 +148,7 @@ def test_ragged_shapes_full_oracle(variant, N, h, r, M, k):
     check(variant, N, h, r, M, k, seed=N)
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 def test_empty_batch_zeroes_counts(variant):
     m = lib()
     h, r, M, k = 64, 32, 128, 4
@@ -146,6 +158,8 @@ def test_empty_batch_zeroes_counts(variant):
     cnt = torch.full((M,), 7, dtype=torch.int32, device="cuda")
     if variant == "unfused":
         m.route_unfused(X, R1, R2, k, out_expert_count=cnt)
+    elif variant == "unfused_tc":
+        m.route_unfused_tc(X, R1, R2, k, out_expert_count=cnt)
     else:
         if not supported(variant, 0, h, r, M, k):
             pytest.skip("variant does not take this shape")
@@ -161,7 +175,7 @@ def identity_weights(M):
     return eye, eye
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 @pytest.mark.parametrize("k", [1, 3, 8, 16])
 def test_tie_heavy_exact(variant, k):
     """Small-integer logits (R1 = R2 = I): many exact ties; lower index wins (Alg. 1)."""
@@ -175,7 +189,7 @@ def test_tie_heavy_exact(variant, k):
     parity.compare(X, R1, R2, N, M, M, M, k, idx, gate, cnt, logits, exact=True)
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 def test_jl_construction_exact(variant):
     """App. J, Theorem 4 (uncompressed): x_S = (M-k) on S, -k elsewhere; top-k is S."""
     M, k, N = 64, 4, 600
@@ -205,7 +219,7 @@ def hypercube(h, r, r_impl=None):
     return syn.f32_to_bf16_bits(R1), syn.f32_to_bf16_bits(R2), M
 
 
-@pytest.mark.parametrize("variant", VARIANTS + ["unfused"])
+@pytest.mark.parametrize("variant", VARIANTS + UNFUSED)
 def test_hypercube_top1_is_sign_pattern(variant):
     """Prop. 1 proof (App. J): the k = 1 winner is the sign pattern of z."""
     h, r = 64, 16

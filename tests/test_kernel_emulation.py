@@ -113,9 +113,12 @@ def test_cluster_routing_tie_heavy_exact(emu):
 @pytest.mark.parametrize("name,old,new", [
     ("backward.cu", "(pbt[e] - tg[t])", "(pbt[e] + tg[t])"),                   # the sign of g in ybar
     ("route_cluster.cu", "for (int p = 0; p < kCluster; ++p) z +=", "for (int p = 1; p < kCluster; ++p) z +="),
+    ("route_scores_topk.cu", "lane < k && lv >= xv", "lane < k && lv > xv"),  # equal values: later expert first
+    ("route_scores_topk.cu", "first ? lmax >= floor0", "first ? lmax > floor0"),  # drops values at the floor
 ])
 def test_planted_kernel_mistake_is_caught(tmp_path, name, old, new):
-    """A mistake planted in a kernel source fails these checks (a dropped partial z, a sign)."""
+    """A mistake planted in a kernel source fails these checks (a dropped partial z, a sign, the
+    order of equal scores, a first-chunk filter that drops values at its floor)."""
     reason = emulation.available()
     if reason:
         pytest.skip(reason)
@@ -123,6 +126,9 @@ def test_planted_kernel_mistake_is_caught(tmp_path, name, old, new):
     with pytest.raises(AssertionError):
         if name == "backward.cu":
             backward(e, 70, 128, 32, 192, 4, seed=3)
+        elif name == "route_scores_topk.cu":
+            ties = np.random.default_rng(0).integers(-3, 4, size=(40, 520)).astype(np.float32)
+            check_threshold_topk(e, ties, 4)
         else:
             X, R1, R2 = syn.router_inputs(13, 256, 32, 512, seed=13)
             cluster(e, X, R1, R2, 13, 256, 32, 512, 8)
@@ -158,6 +164,55 @@ def test_routing_kernels_tie_heavy_exact(emu, entry):
     X = syn.f32_to_bf16_bits(np.random.default_rng(9).integers(-3, 4, size=(N, M)).astype(np.float32))
     eye = syn.f32_to_bf16_bits(np.eye(M, dtype=np.float32))
     route_with(emu, entry, X, eye, eye, N, M, M, M, k, exact=True)
+
+
+def threshold_topk(e, scores, k):
+    N, M = scores.shape
+    out = (e.empty(N * k * 4), e.empty(N * k * 4), e.empty(M * 4), e.empty(N * k * 4))
+    status = ctypes.c_uint(0)
+    assert e.lib.emu_threshold_topk(e.put(np.asarray(scores, np.float32)), N, M, k, *out,
+                                    ctypes.addressof(status)) == 0
+    got = (e.get(out[0], (N, k), np.int32), e.get(out[1], (N, k), np.float32), e.get(out[2], (M,), np.int32),
+           e.get(out[3], (N, k), np.float32))
+    e.free_all()
+    assert status.value == 0
+    return got
+
+
+def check_threshold_topk(e, scores, k):
+    """The selection is fixed by the fp32 scores themselves: the k largest in routing order
+    (larger value first, lower expert first on equal values), softmax over them, counts."""
+    N, M = scores.shape
+    idx, gate, cnt, logits = threshold_topk(e, scores, k)
+    order = np.lexsort((np.broadcast_to(np.arange(M), (N, M)), -scores.astype(np.float64)), axis=1)[:, :k]
+    np.testing.assert_array_equal(idx, order)
+    sel = np.take_along_axis(scores, order, axis=1)
+    np.testing.assert_array_equal(logits, sel)
+    ex = np.exp(sel.astype(np.float64) - sel[:, :1])
+    np.testing.assert_allclose(gate, ex / ex.sum(axis=1, keepdims=True), rtol=0, atol=2e-6)
+    np.testing.assert_array_equal(cnt, np.bincount(order.ravel(), minlength=M))
+
+
+@pytest.mark.parametrize("N,M,k", [(50, 8, 8), (64, 40, 3), (33, 128, 16), (40, 200, 1), (25, 1000, 8),
+                                   (6, 4096, 8), (9, 4104, 5), (3, 520, 16)])
+def test_threshold_topk_kernel_on_oracle_scores(emu, N, M, k):
+    """The tensor-core unfused path's top-k kernel on fp32 scores taken from the oracle's logits
+    (ragged chunks: M = 40, 200, 1000, 4104; k = 1 .. 16)."""
+    X, R1, R2 = syn.router_inputs(N, 64, 16, M, seed=M + k)
+    check_threshold_topk(emu, oracle.logits(X, R1, R2, N, 64, 16, M).astype(np.float32), k)
+
+
+@pytest.mark.parametrize("k", [1, 4, 16])
+def test_threshold_topk_kernel_ties_and_orders(emu, k):
+    """Small integers (ties inside and across chunks), then rows in ascending order (every value
+    enters the list), descending order (only the first chunk does), and constant rows."""
+    rng = np.random.default_rng(k)
+    M = 520
+    rows = [rng.integers(-3, 4, size=(40, M)).astype(np.float32),
+            np.tile(np.arange(M, dtype=np.float32), (3, 1)),
+            np.tile(np.arange(M, dtype=np.float32)[::-1].copy(), (3, 1)),
+            np.full((3, M), 2.5, np.float32)]
+    check_threshold_topk(emu, np.concatenate(rows), k)
 
 
 @pytest.mark.parametrize("N,h,r,M", [(23, 128, 32, 192), (6, 512, 16, 1000), (1, 64, 128, 64)])
