@@ -377,12 +377,7 @@ def main():
 
     variant_used = args.variant
     if args.variant == "auto":
-        variant_used = "fused_tc"
-        try:
-            more.route(X[:1024], R1, R2, k, variant="fused_tc")
-        except more.MoreError:
-            variant_used = "small_n"
-        variant_used = variant_used if N >= 512 else "small_n"
+        variant_used = more.auto_variant(N, h, r, M, k)
     launches_per_step = {"unfused": 3, "unfused_tc": 2, "train": 2, "dispatch": 5, "dispatch_shared": 5,
                          "backward": 5}.get(args.variant, 1)
 

@@ -68,7 +68,7 @@ typedef enum more_status {
 
 /* Kernel variants of more_route_variant.  All compute the same function. */
 typedef enum more_variant {
-  MORE_VARIANT_AUTO = 0,     /* the fused tensor-core kernel for large N, the small-N kernel otherwise */
+  MORE_VARIANT_AUTO = 0,     /* chosen per shape: see more_route_auto_variant                         */
   MORE_VARIANT_FUSED_TC = 1, /* persistent kernel: TMA-staged X, tcgen05 MMAs into TMEM             */
   MORE_VARIANT_SMALL_N = 2,  /* CUDA-core kernel, one CTA of 16 warps per token (decode batches)    */
   MORE_VARIANT_CLUSTER = 3   /* CUDA-core kernel, 8 tokens per cluster of 8 CTAs: experts split over
@@ -89,6 +89,24 @@ typedef enum more_variant {
 more_status more_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,
                        int k, int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
                        float* out_logits, void* stream);
+
+/*
+ * The kernel AUTO runs for this shape (a more_variant value), or MORE_VARIANT_AUTO if the shape
+ * fails the argument requirements.  The choice follows per-call times measured on a B200:
+ *   - N < 256: MORE_VARIANT_SMALL_N;
+ *   - otherwise MORE_VARIANT_CLUSTER while its time, which grows with N, stays below the fused
+ *     kernel's floor (the latency of one 128-token tile: Z over h, then two sweeps over the
+ *     M / 128 expert tiles); MORE_VARIANT_FUSED_TC beyond.  At h = 2048, M = 4096 the switch
+ *     falls near N = 1,300 (r = 32) and N = 2,000 (r = 16);
+ *   - MORE_VARIANT_CLUSTER at any N >= 256 for shapes the fused kernel's shared-memory plan
+ *     cannot hold: r = 128 with k > 8 (any M), r = 128 with 4 < k <= 8 and M >= 11752,
+ *     r = 128 with k <= 4 and M >= 39048, r = 64 with k > 8 and M >= 28136, every r not in
+ *     {16, 32, 64, 128}, and M > 65536.  Those shapes run on CUDA cores, far slower per token
+ *     at prefill sizes than the fused kernel (r = 128, k = 16, M = 4096: about 0.26 us per
+ *     token against 2.3 ns for the fused kernel at r = 32).
+ * Host-only; makes no CUDA call.
+ */
+int more_route_auto_variant(int64_t N, int h, int r, int M, int k);
 
 /* more_route with an explicit kernel variant (more_variant); same contract. */
 more_status more_route_variant(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,

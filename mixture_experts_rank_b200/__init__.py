@@ -20,7 +20,7 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
+__all__ = ["route", "auto_variant", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
            "dispatch_scratch_bytes", "route_unfused", "route_unfused_tc", "route_unfused_static", "unfused_scratch_bytes", "device_status",
            "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
@@ -49,6 +49,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_variant.argtypes = route_args + [I, P]
     lib.more_route_unfused.restype = I
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
+    lib.more_route_auto_variant.restype = I
+    lib.more_route_auto_variant.argtypes = [I64, I, I, I, I]
     lib.more_route_unfused_tc.restype = I
     lib.more_route_unfused_tc.argtypes = route_args + [P, ctypes.c_size_t, P]
     lib.more_route_unfused_static.restype = I
@@ -253,6 +255,13 @@ def dispatch(idx: torch.Tensor, M: int, *, scratch: torch.Tensor | None = None, 
                                     scratch.numel(), DISPATCH_VARIANTS[variant], _stream_handle(stream))
     _check(st, "more_dispatch")
     return out_offsets, out_sorted
+
+
+def auto_variant(N: int, h: int, r: int, M: int, k: int) -> str | None:
+    """The kernel ``route(..., variant="auto")`` runs for this shape (``more_route_auto_variant``),
+    or None if the shape fails the argument requirements."""
+    v = int(_lib.more_route_auto_variant(N, h, r, M, k))
+    return {value: name for name, value in VARIANTS.items()}[v] if v else None
 
 
 def unfused_scratch_bytes(N: int, r: int, M: int) -> int:

@@ -48,24 +48,63 @@ RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, in
   return a;
 }
 
-// Below this many tokens the small-N kernel wins: the fused kernel works on
-// 128-token tiles, one per SM, and a handful of tiles leaves the GPU idle.
-constexpr int64_t kSmallNThreshold = 512;
+// AUTO's choice of kernel, from per-call times measured on a B200 (CUDA-graph replays of
+// back-to-back calls; h = 2048, M = 4096 with r = 16, 32 and 128):
+// - below 256 tokens the small-N kernel (one CTA per token) is fastest or level;
+// - from 256 tokens the cluster kernel overtakes it.  Its time grows linearly,
+//   about 12 us + N * 2.3e-7 us * r * (h + M) (r = 32: 58 us at N = 1024, 104 us at 2048);
+// - the fused kernel's time has a floor until every SM holds a tile: the chain of one
+//   128-token tile (Z over h, then two sweeps over the M / 128 expert tiles), about
+//   5 us + 0.0056 us * h + 0.0133 us * M * (0.7 + 0.3 r / 32) (r = 32: 74 us; r = 16: 58 us).
+// AUTO takes the cluster kernel while its estimate is below that floor, the fused kernel
+// beyond (when its shared-memory plan fits the shape), and the cluster kernel at any N for
+// shapes the fused kernel does not take.
+constexpr int64_t kClusterMinTokens = 256;
+
+double cluster_estimate_us(int64_t N, int h, int r, int M) {
+  return 12.0 + (double)N * 2.3e-7 * r * ((double)h + M);
+}
+
+double fused_floor_us(int h, int r, int M) {
+  return 5.0 + 0.0056 * h + 0.0133 * M * (0.7 + 0.3 * r / 32.0);
+}
+
+int auto_variant(const RouteArgs& a) {
+  if (a.N < kClusterMinTokens) return MORE_VARIANT_SMALL_N;
+  if (!fused_tc_fits(a)) return MORE_VARIANT_CLUSTER;
+  return cluster_estimate_us(a.N, a.h, a.r, a.M) < fused_floor_us(a.h, a.r, a.M) ? MORE_VARIANT_CLUSTER
+                                                                                  : MORE_VARIANT_FUSED_TC;
+}
 
 }  // namespace
 
+namespace {
+// Shapes that cannot mean anything (MORE_ERR_INVALID_ARG) and legal shapes outside the
+// library's limits (MORE_ERR_UNSUPPORTED).
+bool shape_invalid(int64_t N, int h, int r, int M, int k) {
+  return N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1;
+}
+bool shape_unsupported(int64_t N, int r, int M, int k) {
+  return N > 0x7fffffffLL || k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX;
+}
+}  // namespace
+
 // Argument checks shared by every routing entry point (see more_route.h).
+more_status validate_shape(int64_t N, int h, int r, int M, int k) {
+  if (shape_invalid(N, h, r, M, k)) return MORE_ERR_INVALID_ARG;
+  if (shape_unsupported(N, r, M, k)) return MORE_ERR_UNSUPPORTED;
+  return MORE_OK;
+}
+
 more_status validate_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
                            const int32_t* out_idx, const float* out_gate, const int32_t* out_count,
                            const float* out_logits) {
-  if (N < 0 || h < 8 || (h & 7) || M < 8 || (M & 7) || k < 1 || k > M || r < 1)
-    return MORE_ERR_INVALID_ARG;
+  if (shape_invalid(N, h, r, M, k)) return MORE_ERR_INVALID_ARG;
   if (!R1 || !R2 || !out_count || (N > 0 && (!X || !out_idx || !out_gate))) return MORE_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || !aligned16(R1) || !aligned16(R2) || (out_idx && !aligned16(out_idx)) ||
       (out_gate && !aligned16(out_gate)) || !aligned16(out_count) || (out_logits && !aligned16(out_logits)))
     return MORE_ERR_INVALID_ARG;
-  if (N > 0x7fffffffLL) return MORE_ERR_UNSUPPORTED;
-  if (k > MORE_KMAX || (r & 15) || r < 16 || r > 128 || M > MORE_MMAX) return MORE_ERR_UNSUPPORTED;
+  if (shape_unsupported(N, r, M, k)) return MORE_ERR_UNSUPPORTED;
   return MORE_OK;
 }
 
@@ -107,9 +146,7 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
   if (cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
     return MORE_ERR_CUDA;
   if (N == 0) return MORE_OK;
-  if (variant == MORE_VARIANT_AUTO)
-    variant = (N >= kSmallNThreshold && fused_tc_supports(a)) ? MORE_VARIANT_FUSED_TC
-                                                              : MORE_VARIANT_SMALL_N;
+  if (variant == MORE_VARIANT_AUTO) variant = auto_variant(a);
   cudaError_t err;
   if (variant == MORE_VARIANT_FUSED_TC) {
     if (!fused_tc_supports(a)) return MORE_ERR_UNSUPPORTED;
@@ -120,6 +157,12 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
     err = launch_small_n(a);
   }
   return err == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
+int more_route_auto_variant(int64_t N, int h, int r, int M, int k) {
+  if (validate_shape(N, h, r, M, k) != MORE_OK) return MORE_VARIANT_AUTO;
+  RouteArgs a = make_args(nullptr, nullptr, nullptr, N, h, r, M, k, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return auto_variant(a);
 }
 
 more_status more_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M,

@@ -24,6 +24,7 @@ struct RouteArgs {
 };
 
 // Argument checks of the routing entry points (more_route.h): MORE_OK or the error to return.
+more_status validate_shape(int64_t N, int h, int r, int M, int k);
 more_status validate_route(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
                            const int32_t* out_idx, const float* out_gate, const int32_t* out_count,
                            const float* out_logits);
@@ -62,6 +63,9 @@ struct BackwardArgs {
 int64_t backward_scratch_bytes(int64_t N, int h, int r, int M);
 cudaError_t launch_backward(const BackwardArgs& b);
 cudaError_t launch_fused_tc(const RouteArgs& a);
+// The fused kernel's shared-memory plan fits the shape (r, M, k); supports: it fits and the
+// driver's tensor-map encoder is available.
+bool fused_tc_fits(const RouteArgs& a);
 bool fused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused(const RouteArgs& a, void* scratch);
 size_t unfused_scratch_bytes(int64_t N, int r, int M);

@@ -75,9 +75,11 @@ constexpr int kWarpA0 = kRoleWarps, kWarpB0 = kRoleWarps + kWarpsA;
 constexpr int kThreads = (kRoleWarps + kWarpsA + kWarpsB) * 32;
 constexpr int kNamedBarA = 1, kNamedBarB = 2;    // bar.sync ids of the groups
 static_assert(kWarpsB % 4 == 0, "group B covers the four TMEM lane groups evenly");
+static_assert((kWarpsB & (kWarpsB - 1)) == 0, "fallback teams divide group B evenly");
 constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass B
 constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than one candidate
 constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
+static_assert(kFbBatch <= kWarpsB, "one merging warp per fallback token of a batch");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint32_t kRealKey = 0x00800000u;  // ordered value of -FLT_MAX: keys below are not real chunks
@@ -102,6 +104,7 @@ struct Params {
   uint32_t off_pairs, off_cbase, off_flag, off_nq;
   // group B only
   uint32_t off_cand, off_pc, off_pool, off_poolcnt, off_fb, off_part;
+  int fb_groups;  // warps per fallback token: min(kWarpsB, 256-expert blocks rounded up to a power of two)
   uint32_t off_bar;
 };
 
@@ -790,12 +793,15 @@ __device__ __forceinline__ void fallback_block(const RouteArgs& a, const float (
   }
 }
 
-// The cooperative fallback's first step: this warp's partial top-k (over the 256-expert
-// blocks bw, bw + kWarpsB, ...) of each of the nb tokens in tok, written to part.
+// The cooperative fallback's first step.  The group's warps form kWarpsB / G teams of G
+// warps (G = p.fb_groups, a power of two no larger than the number of 256-expert blocks):
+// team js takes tokens js, js + kWarpsB / G, ... of the nb tokens in tok, and warp g of the
+// team ranks the blocks g, g + G, ... of each, writing its partial top-k to part.
 template <int R, int KCAP>
 __device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t* zs, const uint8_t* tok, int nb,
-                                              uint2* part, int bw, int lane) {
-  for (int j = 0; j < nb; ++j) {
+                                              uint2* part, int G, int bw, int lane) {
+  const int teams = kWarpsB / G, js = bw / G, g = bw % G;
+  for (int j = js; j < nb; j += teams) {
     const int tf = tok[j];
     float zr[(R + 31) / 32];
 #pragma unroll
@@ -803,21 +809,21 @@ __device__ __forceinline__ void fallback_rank(const RouteArgs& a, const uint8_t*
       zr[q] = (32 * q + lane < R) ? zs_value<R, KCAP>(zs, tf, 32 * q + lane) : 0.f;
     TopList<KCAP> list;
     list.init();
-    for (int eb = 256 * bw; eb < a.M; eb += 256 * kWarpsB) fallback_block<R, KCAP>(a, zr, eb, lane, list);
+    for (int eb = 256 * g; eb < a.M; eb += 256 * G) fallback_block<R, KCAP>(a, zr, eb, lane, list);
     float v;
     int e;
     warp_merge_topk<KCAP>(list, a.k, lane, v, e);
-    if (lane < KCAP) part[(j * kWarpsB + bw) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
+    if (lane < KCAP) part[(j * G + g) * KCAP + lane] = make_uint2(__float_as_uint(v), (uint32_t)e);
   }
 }
 
-// The second step: merge the partial lists of one token (part: warp-major, KCAP
-// entries each, the first k valid) and write the token's outputs.
+// The second step: merge the G partial lists of one token (part: list-major, KCAP entries
+// each, the first k valid) and write the token's outputs.
 template <int KCAP>
-__device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* part, int64_t n, int lane) {
+__device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* part, int G, int64_t n, int lane) {
   TopList<KCAP> list;
   list.init();
-  for (int q = lane; q < kWarpsB * KCAP; q += 32) {
+  for (int q = lane; q < G * KCAP; q += 32) {
     const uint2 c = part[q];
     if ((q % KCAP) < a.k) list.insert_any(__uint_as_float(c.x), (int)c.y);
   }
@@ -1011,16 +1017,17 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       a.out_gate[ob + x] = sex[x];
       if (a.out_logits) a.out_logits[ob + x] = slog[x];
     }
-    // fallback tokens, kFbBatch at a time: every warp of the group ranks its 256-expert
-    // blocks (blocks bw, bw + kWarpsB, ...) for each token, then warp jj merges the partial
-    // lists of the batch's token jj and writes it
+    // fallback tokens, kFbBatch at a time: teams of p.fb_groups warps rank the batch's tokens
+    // over their 256-expert blocks, then warp jj merges the partial lists of the batch's token
+    // jj and writes it
     const uint8_t* zs = zs0 + zs_buf(j, p.interleave) * C::ZS_BYTES;
     const int nfb = *fbcount;
     for (int fb0 = 0; fb0 < nfb; fb0 += kFbBatch) {
       const int nbt = nfb - fb0 < kFbBatch ? nfb - fb0 : kFbBatch;
-      fallback_rank<R, KCAP>(a, zs, fblist + fb0, nbt, part, bw, lane);
+      fallback_rank<R, KCAP>(a, zs, fblist + fb0, nbt, part, p.fb_groups, bw, lane);
       group_bar(kNamedBarB, kThreadsB);
-      if (bw < nbt) fallback_merge<KCAP>(a, part + bw * kWarpsB * KCAP, n0 + fblist[fb0 + bw], lane);
+      if (bw < nbt)
+        fallback_merge<KCAP>(a, part + bw * p.fb_groups * KCAP, p.fb_groups, n0 + fblist[fb0 + bw], lane);
       group_bar(kNamedBarB, kThreadsB);
     }
     // reset the per-tile counters for the next tile
@@ -1258,6 +1265,8 @@ bool fill_params(const RouteArgs& a, Params& p, uint32_t& smem) {
   p.kb_count = (a.h + Cfg<R, KCAP>::BK - 1) / Cfg<R, KCAP>::BK;
   p.p_count = (a.M + kBE - 1) / kBE;
   p.nchunks = (a.M + 31) / 32;
+  p.fb_groups = 1;
+  while (p.fb_groups < kWarpsB && 256 * p.fb_groups < a.M) p.fb_groups *= 2;
   int bits = 1;  // chunk ids run up to 4 p_count - 1 (the padded last tile)
   while ((1 << bits) < 4 * p.p_count) ++bits;
   p.low_mask = (1u << bits) - 1u;
@@ -1320,10 +1329,9 @@ bool supports_r(const RouteArgs& a) {
 
 }  // namespace tc
 
-bool fused_tc_supports(const RouteArgs& a) {
+bool fused_tc_fits(const RouteArgs& a) {
   // 65536 experts = 2048 chunks: the pair-count scan covers 8 chunks per group-A thread
   if (a.M > 65536 || a.k > 16 || a.N < 1 || a.N > 0x7fffffffLL - tc::kBT) return false;
-  if (!tc::encode_fn()) return false;
   switch (a.r) {
     case 16: return tc::supports_r<16>(a);
     case 32: return tc::supports_r<32>(a);
@@ -1332,6 +1340,8 @@ bool fused_tc_supports(const RouteArgs& a) {
     default: return false;
   }
 }
+
+bool fused_tc_supports(const RouteArgs& a) { return fused_tc_fits(a) && tc::encode_fn() != nullptr; }
 
 cudaError_t launch_fused_tc(const RouteArgs& a) {
   switch (a.r) {

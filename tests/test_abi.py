@@ -77,6 +77,25 @@ def test_unfused_scratch_size_and_checks(lib):
     assert st == 1
 
 
+@pytest.mark.parametrize("shape,expected", [
+    ((1, 2048, 32, 4096, 8), "small_n"), ((255, 2048, 32, 4096, 8), "small_n"),
+    ((256, 2048, 32, 4096, 8), "cluster"), ((1024, 2048, 32, 4096, 8), "cluster"),
+    ((2048, 2048, 32, 4096, 8), "fused_tc"), ((262144, 2048, 32, 4096, 8), "fused_tc"),
+    ((2048, 2048, 16, 4096, 4), "cluster"), ((4096, 2048, 16, 4096, 4), "fused_tc"),
+    ((262144, 2048, 128, 4096, 16), "cluster"),     # the fused kernel's plan does not hold r = 128, k > 8
+    ((262144, 2048, 128, 8192, 8), "fused_tc"), ((262144, 2048, 128, 11752, 8), "cluster"),
+    ((262144, 2048, 48, 4096, 8), "cluster"),       # r outside the fused kernel's ranks
+    ((32768, 4096, 64, 65536, 8), "fused_tc"),
+    ((16, 64, 32, 64, 0), None), ((16, 64, 24, 64, 4), None),
+])
+def test_auto_variant_follows_the_measured_crossovers(shape, expected):
+    """AUTO's choice (host-only, no GPU): small-N below 256 tokens, the cluster kernel up to the
+    fused kernel's one-tile floor, the fused kernel beyond, and the cluster kernel for shapes the
+    fused kernel's shared-memory plan cannot hold."""
+    import mixture_experts_rank_b200 as m
+    assert m.auto_variant(*shape) == expected
+
+
 def test_unfused_tc_checks_rank_and_scratch(lib):
     """The tensor-core materialisation takes r in {16, 32, 64, 128} and the unfused scratch size."""
     n = lib.more_route_unfused_scratch_bytes(1000, 32, 256)
