@@ -64,8 +64,8 @@ BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X,
 # was captured: once route_tc.cu differs from that source the figure is stale and traffic is
 # reported null.  Workloads without a capture report traffic null.
 NCU_TRAFFIC = {    # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
-    "prefill_r32": ((269225728 + 5350912) / 65536,
-                    "befaa7c6efe03d8fd0009787ce44721960f9f4b126fb1a7f017c051db2454282"),
+    "prefill_r32": ((269207808 + 5669120) / 65536,
+                    "d652dfd40269b1b1101246c61c4142d9c062bd1987b4b5274a9918f2cfe06805"),
 }
 L2_BYTES = 126 * 1024 * 1024
 
