@@ -6,7 +6,8 @@ does, and shares no code with it.  The arithmetic lives in ``more_oracle.c``
 (plain C loops in double precision); this module only marshals numpy arrays.
 
 Source: "MoRE: Scaling mixture of experts with hardware-aware low-rank routing"
-(arXiv 2609.36301), §2 "MoRE layer", App. F eq. (5) and Algorithm 1.
+(arXiv 2609.36301), §2 "MoRE layer", App. F eq. (5) and Algorithm 1; the standard
+(full-rank) router that App. H.3 fuses the same way (``route_fullrank``).
 Parity status of every function: pinned by ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -46,6 +47,12 @@ def _bind(lib):
     lib.oracle_route.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                  ctypes.c_int, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.c_int]
+    lib.oracle_route_fullrank.restype = ctypes.c_int
+    lib.oracle_route_fullrank.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int]
+    lib.oracle_logits_at_fullrank.restype = ctypes.c_int
+    lib.oracle_logits_at_fullrank.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int64, _P, _P, _P]
     lib.oracle_logits.restype = ctypes.c_int
     lib.oracle_logits.argtypes = [_P, _P, _P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   _P, ctypes.c_int64, _P]
@@ -115,6 +122,42 @@ def route(X, R1, R2, N: int, h: int, r: int, M: int, k: int, rows=None,
     if rc != 0:
         raise ValueError("oracle_route: invalid arguments")
     return OracleResult(idx, gate, logit, margin, gaps, rms, counts)
+
+
+def route_fullrank(X, W, N: int, h: int, M: int, k: int, rows=None, threads: int | None = None) -> OracleResult:
+    """The standard router of App. H.3 on tokens ``rows`` (default: all N): logits x . W with a
+    full-rank bf16 W (h x M), then the selection, gates and statistics of :func:`route`."""
+    X = _u16(X, (N, h))
+    W = _u16(W, (h, M))
+    rows, n = _rows(rows, N)
+    idx = np.empty((n, k), np.int32)
+    gate = np.empty((n, k))
+    logit = np.empty((n, k))
+    margin = np.empty(n)
+    gaps = np.empty((n, k))
+    rms = np.empty(n)
+    counts = np.empty(M, np.int64)
+    rc = _load().oracle_route_fullrank(X.ctypes.data, W.ctypes.data, N, h, M, k,
+                                       None if rows is None else rows.ctypes.data, n, idx.ctypes.data,
+                                       gate.ctypes.data, logit.ctypes.data, margin.ctypes.data,
+                                       gaps.ctypes.data, rms.ctypes.data, counts.ctypes.data,
+                                       threads or max(1, min(64, os.cpu_count() or 1)))
+    if rc != 0:
+        raise ValueError("oracle_route_fullrank: invalid arguments")
+    return OracleResult(idx, gate, logit, margin, gaps, rms, counts)
+
+
+def logits_at_fullrank(X, W, N: int, h: int, M: int, rows, experts) -> np.ndarray:
+    """Full-rank logits x_n . W[:, e] of single (row, expert) pairs, fp64."""
+    X = _u16(X, (N, h))
+    W = _u16(W, (h, M))
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    out = np.empty(rows.size)
+    if _load().oracle_logits_at_fullrank(X.ctypes.data, W.ctypes.data, N, h, M, rows.size, rows.ctypes.data,
+                                         experts.ctypes.data, out.ctypes.data) != 0:
+        raise ValueError("oracle_logits_at_fullrank: invalid arguments")
+    return out
 
 
 def logits(X, R1, R2, N: int, h: int, r: int, M: int, rows=None) -> np.ndarray:

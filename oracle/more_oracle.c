@@ -16,6 +16,8 @@
  *   counts[e] = number of (token, slot) pairs naming e  [MoRE App. F eq. (9), f]
  *   training statistics m_n, Z_n and psum of App. F, Algorithm 2, eqs. (6)-(7)
  *           (oracle_train_stats)
+ *   the standard (full-rank) router of the same form, l = x_n . W with W h x M,
+ *           which App. H.3 fuses with the same kernel design (oracle_route_fullrank)
  * plus what the parity checks need: the margin l_(k) - l_(k+1) of Def. 1
  * [MoRE §3, Definition 1] (+inf when k = M), the gaps between consecutive
  * selected logits, and the root-mean-square of the token's M logits.
@@ -62,6 +64,15 @@ void oracle_token_logits(const uint16_t* x, const uint16_t* R1, const uint16_t* 
   }
 }
 
+/* l = x . W for one token, W h x M (the standard router of App. H.3). */
+void oracle_token_logits_full(const uint16_t* x, const uint16_t* W, int h, int M, double* logits) {
+  for (int e = 0; e < M; ++e) {
+    double s = 0.0;
+    for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);
+    logits[e] = s;
+  }
+}
+
 /* The routing order: a goes before b iff l_a > l_b, or l_a == l_b and a < b. */
 typedef struct {
   const double* l;
@@ -102,7 +113,7 @@ void oracle_select(const double* logits, int M, int k, int32_t* idx, double* gat
 }
 
 typedef struct {
-  const uint16_t *X, *R1, *R2;
+  const uint16_t *X, *R1, *R2; /* full rank: R1 is NULL and R2 is W (h x M) */
   int h, r, M, k;
   const int64_t* rows;
   int64_t begin, end;
@@ -113,12 +124,15 @@ typedef struct {
 
 static void* oracle_worker(void* arg) {
   oracle_job* jb = (oracle_job*)arg;
-  double* z = (double*)malloc(sizeof(double) * (size_t)jb->r);
+  double* z = (double*)malloc(sizeof(double) * (size_t)(jb->r > 0 ? jb->r : 1));
   double* l = (double*)malloc(sizeof(double) * (size_t)jb->M);
   oracle_item* scratch = (oracle_item*)malloc(sizeof(oracle_item) * (size_t)jb->M);
   for (int64_t q = jb->begin; q < jb->end; ++q) {
     int64_t n = jb->rows ? jb->rows[q] : q;
-    oracle_token_logits(jb->X + (size_t)n * jb->h, jb->R1, jb->R2, jb->h, jb->r, jb->M, z, l);
+    if (jb->R1)
+      oracle_token_logits(jb->X + (size_t)n * jb->h, jb->R1, jb->R2, jb->h, jb->r, jb->M, z, l);
+    else
+      oracle_token_logits_full(jb->X + (size_t)n * jb->h, jb->R2, jb->h, jb->M, l);
     size_t o = (size_t)q * jb->k;
     oracle_select(l, jb->M, jb->k, jb->idx + o, jb->gate + o, jb->logit + o, jb->margin + q,
                   jb->gaps + o, jb->rms + q, scratch);
@@ -136,11 +150,11 @@ static void* oracle_worker(void* arg) {
  * logit and gaps are n_rows x k; margin and rms are n_rows; counts (length M)
  * counts the selections of these tokens.  Returns 0, or 1 on bad arguments.
  */
-int oracle_route(const uint16_t* X, const uint16_t* R1, const uint16_t* R2, int64_t N, int h,
-                 int r, int M, int k, const int64_t* rows, int64_t n_rows, int32_t* idx,
-                 double* gate, double* logit, double* margin, double* gaps, double* rms,
-                 int64_t* counts, int nthreads) {
-  if (N < 0 || h < 1 || r < 1 || M < 1 || k < 1 || k > M || n_rows < 0) return 1;
+static int oracle_route_rows(const uint16_t* X, const uint16_t* R1, const uint16_t* R2, int64_t N,
+                             int h, int r, int M, int k, const int64_t* rows, int64_t n_rows,
+                             int32_t* idx, double* gate, double* logit, double* margin, double* gaps,
+                             double* rms, int64_t* counts, int nthreads) {
+  if (N < 0 || h < 1 || M < 1 || k < 1 || k > M || n_rows < 0) return 1;
   if (!rows && n_rows > N) return 1;
   if (rows)
     for (int64_t q = 0; q < n_rows; ++q)
@@ -174,6 +188,44 @@ int oracle_route(const uint16_t* X, const uint16_t* R1, const uint16_t* R2, int6
     for (int e = 0; e < M; ++e) counts[e] += priv[(size_t)t * M + e];
   }
   free(priv);
+  return 0;
+}
+
+int oracle_route(const uint16_t* X, const uint16_t* R1, const uint16_t* R2, int64_t N, int h,
+                 int r, int M, int k, const int64_t* rows, int64_t n_rows, int32_t* idx,
+                 double* gate, double* logit, double* margin, double* gaps, double* rms,
+                 int64_t* counts, int nthreads) {
+  if (!R1 || r < 1) return 1;
+  return oracle_route_rows(X, R1, R2, N, h, r, M, k, rows, n_rows, idx, gate, logit, margin, gaps,
+                           rms, counts, nthreads);
+}
+
+/*
+ * The standard router of App. H.3 ("Fusing a standard MoE layer"): the same selection,
+ * gates, counts and parity statistics as oracle_route, with the logits l = x . W of a
+ * full-rank W (h x M) instead of (x . R1) . R2.
+ */
+int oracle_route_fullrank(const uint16_t* X, const uint16_t* W, int64_t N, int h, int M, int k,
+                          const int64_t* rows, int64_t n_rows, int32_t* idx, double* gate,
+                          double* logit, double* margin, double* gaps, double* rms, int64_t* counts,
+                          int nthreads) {
+  return oracle_route_rows(X, NULL, W, N, h, 0, M, k, rows, n_rows, idx, gate, logit, margin, gaps,
+                           rms, counts, nthreads);
+}
+
+/* Full-rank logit of single (token, expert) pairs, fp64: l = sum_t x_t W[t,e]. */
+int oracle_logits_at_fullrank(const uint16_t* X, const uint16_t* W, int64_t N, int h, int M,
+                              int64_t n_pairs, const int64_t* rows, const int32_t* experts,
+                              double* out) {
+  for (int64_t p = 0; p < n_pairs; ++p) {
+    int64_t n = rows[p];
+    int e = experts[p];
+    if (n < 0 || n >= N || e < 0 || e >= M) return 1;
+    const uint16_t* x = X + (size_t)n * h;
+    double s = 0.0;
+    for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);
+    out[p] = s;
+  }
   return 0;
 }
 

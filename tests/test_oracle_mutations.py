@@ -28,6 +28,10 @@ MUTATIONS = {
                           "for (int i = 1; i < r; ++i) s += z[i] * oracle_bf16(R2[(size_t)i * M + e]);\n    logits[e] = s;"),
     "dropped_hidden_term": ("for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(R1[(size_t)t * r + i]);\n    z[i] = s;",
                             "for (int t = 0; t + 1 < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(R1[(size_t)t * r + i]);\n    z[i] = s;"),
+    "fullrank_W_transposed": ("s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);",
+                              "s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)e * h + t]);"),
+    "fullrank_dropped_hidden_term": ("for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);",
+                                     "for (int t = 1; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);"),
     "softmax_sign": ("gate[j] = exp(sel_logit[j] - top) / denom;", "gate[j] = exp(top - sel_logit[j]) / denom;"),
     "softmax_missing_shift": ("denom += exp(sel_logit[j] - top);", "denom += exp(sel_logit[j]);"),
     "margin_wrong_runner_up": ("sel_logit[k - 1] - logits[scratch[k].e]",
@@ -59,6 +63,8 @@ PINS = [
     pins.test_train_stats_closed_forms,
     pins.test_train_stats_against_library_softmax,
     pins.test_train_stats_shift_and_relabelling,
+    pins.test_fullrank_matches_the_factored_router_when_W_is_their_product,
+    pins.test_fullrank_tie_order_and_brute_force_ranks,
 ]
 
 
@@ -68,7 +74,7 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation anchor for {name} not found"
     mutated = tmp_path / "mutant.c"
-    mutated.write_text(src.replace(old, new))
+    mutated.write_text(src.replace(old, new))  # every occurrence
     lib_path = tmp_path / "libmutant.so"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-o",
                            str(lib_path), str(mutated), "-lm", "-lpthread"])

@@ -87,6 +87,51 @@ def test_projection_and_pairs_agree_with_matmul():
     np.testing.assert_allclose(sub, (Xf @ R1f @ R2f)[rows], rtol=1e-11, atol=1e-12)
 
 
+# --- the standard (full-rank) router of App. H.3 -----------------------------------
+
+def test_fullrank_matches_the_factored_router_when_W_is_their_product():
+    """W = R1 R2 with small integer factors is exact in bf16 (|W| <= 4r < 256), so the full-rank
+    router on W and the low-rank router on (R1, R2) define the same logits: the two oracle
+    paths (x . W against (x . R1) . R2) must agree to fp64 rounding and select the same
+    experts."""
+    N, h, r, M, k = 40, 48, 16, 72, 5
+    rng = np.random.default_rng(3)
+    R1f = rng.integers(-2, 3, size=(h, r)).astype(np.float32)
+    R2f = rng.integers(-2, 3, size=(r, M)).astype(np.float32)
+    W = syn.f32_to_bf16_bits(R1f @ R2f)
+    R1, R2 = syn.f32_to_bf16_bits(R1f), syn.f32_to_bf16_bits(R2f)
+    assert np.array_equal(syn.bf16_bits_to_f64(W), (R1f @ R2f).astype(np.float64))
+    X = syn.normal_bf16(7, syn.TENSOR_X, N, h)
+    full = oracle.route_fullrank(X, W, N, h, M, k)
+    low = oracle.route(X, R1, R2, N, h, r, M, k)
+    np.testing.assert_allclose(full.logit, low.logit, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(full.rms, low.rms, rtol=1e-12)
+    np.testing.assert_allclose(full.margin, low.margin, rtol=1e-9, atol=1e-9)
+    clear = low.margin > 1e-9 * low.rms
+    assert clear.mean() > 0.9
+    np.testing.assert_array_equal(full.idx[clear], low.idx[clear])
+    np.testing.assert_array_equal(full.counts, low.counts)
+    rows = np.array([0, 5, 5, 39])
+    experts = np.array([71, 0, 33, 12])
+    np.testing.assert_allclose(oracle.logits_at_fullrank(X, W, N, h, M, rows, experts),
+                               oracle.logits_at(X, R1, R2, N, h, r, M, rows, experts), rtol=1e-12, atol=1e-12)
+
+
+def test_fullrank_tie_order_and_brute_force_ranks():
+    """Small integer logits (x one-hot rows times integer W): many exact ties, which the
+    full-rank router must break towards the lower expert, as brute-force ranks do."""
+    N, h, M, k = 30, 16, 24, 6
+    rng = np.random.default_rng(9)
+    X = syn.f32_to_bf16_bits(np.eye(h, dtype=np.float32)[rng.integers(0, h, N)])
+    Wf = rng.integers(-2, 3, size=(h, M)).astype(np.float32)
+    res = oracle.route_fullrank(X, syn.f32_to_bf16_bits(Wf), N, h, M, k)
+    L = syn.bf16_bits_to_f64(X) @ Wf.astype(np.float64)
+    for n in range(N):
+        rank = [int(np.sum((L[n] > L[n, e]) | ((L[n] == L[n, e]) & (np.arange(M) < e)))) for e in range(M)]
+        expected = sorted(range(M), key=lambda e: rank[e])[:k]
+        assert res.idx[n].tolist() == expected
+
+
 # --- selection: brute force, ties, relabelling ----------------------------------
 
 @pytest.mark.parametrize("M", [1, 2, 7, 13, 33])
