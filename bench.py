@@ -56,8 +56,13 @@ WORKLOADS = {
     "fig24_B16": (16384, 2048, 16, 4096, 4, True),
     "fig24_B64": (65536, 2048, 16, 4096, 4, True),
     "fig24_B256": (262144, 2048, 16, 4096, 4, True),
+    # the standard full-rank router (App. H.3, Figs. 20-21 prefill: N = 262,144, M = 4096, k = 4);
+    # r is that of the MoRE layer the figures compare with and only the low-rank variants use it
+    "fullrank_h1024": (262144, 1024, 64, 4096, 4, True),
+    "fullrank_h2048": (262144, 2048, 64, 4096, 4, True),
 }
 METRIC = "routed tokens/s (fused low-rank router + top-k)"
+FULLRANK_METRIC = "routed tokens/s (fused full-rank router + top-k, App. H.3)"
 BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X, R1, R2)"
 # DRAM bytes (read + write) per token of the fused kernel, from one ncu capture at N = 65,536
 # (summarised under profiles/, scaled by tokens), keyed to the SHA-256 of the kernel source that
@@ -171,12 +176,16 @@ def run_reference(args, world, rank):
     R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
     R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
     backward = args.variant == "backward"
+    fullrank = args.variant == "fullrank"
+    W = syn.normal_bf16(0, syn.TENSOR_R2, h, M, 1.0 / np.sqrt(h)) if fullrank else None
     rng = np.random.default_rng(1)
 
     def one_step(X, S):
         if backward:  # the oracle's Algorithm 3 on the sample, seeded selections and gradients
             oracle.router_backward(X, R1, R2, S, h, r, M, rng.integers(0, M, (S, k)),
                                    rng.standard_normal((S, k)), rng.standard_normal(M))
+        elif fullrank:
+            oracle.route_fullrank(X, W, S, h, M, k, threads=cores)
         else:
             oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
 
@@ -200,7 +209,8 @@ def run_reference(args, world, rank):
     step = sum(times) / len(times)
     value = S / step
     sample = f"first {S} tokens of the workload per step ({S / N:.4%} of N), all M experts"
-    line = {"impl": "reference", "metric": BACKWARD_METRIC if backward else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    metric = BACKWARD_METRIC if backward else (FULLRANK_METRIC if fullrank else METRIC)
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": describe(args.workload), "N": N, "h": h, "r": r,
@@ -212,22 +222,27 @@ def run_reference(args, world, rank):
     return 0
 
 
-def cpu_baseline(workload, seconds):
+def cpu_baseline(workload, seconds, fullrank=False):
     import oracle
     import synthetic as syn
     N, h, r, M, k, unit = WORKLOADS[workload]
     cores = os.cpu_count() or 1
-    R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
-    R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+    if fullrank:
+        W = syn.normal_bf16(0, syn.TENSOR_R2, h, M, 1.0 / np.sqrt(h))
+        route = lambda X, S: oracle.route_fullrank(X, W, S, h, M, k, threads=cores)
+    else:
+        R1 = syn.normal_bf16(0, syn.TENSOR_R1, h, r, 1.0 / np.sqrt(h))
+        R2 = syn.normal_bf16(0, syn.TENSOR_R2, r, M, 1.0 / np.sqrt(r))
+        route = lambda X, S: oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
     probe = max(cores, 16)
     Xp = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, probe)
     t = time.perf_counter()
-    oracle.route(Xp, R1, R2, probe, h, r, M, k, threads=cores)
+    route(Xp, probe)
     per_tok = (time.perf_counter() - t) / probe
     S = int(max(probe, min(N, seconds / max(per_tok, 1e-9))))
     X = syn.normal_bf16(0, syn.TENSOR_X, N, h, 1.0, unit, 0, S)
     t = time.perf_counter()
-    oracle.route(X, R1, R2, S, h, r, M, k, threads=cores)
+    route(X, S)
     el = time.perf_counter() - t
     return {"value": S / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"first {S} of the {N} tokens, all M experts, {el:.1f} s on {cores} threads"}
@@ -275,7 +290,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="auto",
-                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "unfused_tc", "train", "dispatch", "dispatch_shared",
+                    choices=["auto", "fused_tc", "small_n", "cluster", "unfused", "unfused_tc", "fullrank", "train", "dispatch", "dispatch_shared",
                              "backward"],
                     help="train: more_route_train (routing plus the full-softmax statistics m, Z, psum); "
                          "dispatch: routing followed by more_dispatch of its indices (dispatch_shared: with the "
@@ -334,6 +349,8 @@ def main():
         d_scratch = torch.empty(max(more.dispatch_scratch_bytes(N, k, M), 16), dtype=torch.uint8, device="cuda")
         d_off = torch.empty((M + 1,), dtype=torch.int32, device="cuda")
         d_sorted = torch.empty((N * k,), dtype=torch.int32, device="cuda")
+    if args.variant == "fullrank":
+        W = dev(syn.normal_bf16(0, syn.TENSOR_R2, h, M, 1.0 / np.sqrt(h)))   # W ~ N(0, 1/h), h x M
     if args.variant in ("unfused", "unfused_tc"):
         scratch = torch.empty(more.unfused_scratch_bytes(N, r, M), dtype=torch.uint8, device="cuda")
     if args.variant == "backward":
@@ -368,6 +385,9 @@ def main():
         elif args.variant == "unfused":
             more.route_unfused(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate, out_expert_count=cnt,
                                out_logits=logits, stream=st)
+        elif args.variant == "fullrank":
+            more.route_fullrank(X, W, k, out_idx=idx, out_gate=gate, out_expert_count=cnt, out_logits=logits,
+                                stream=st)
         elif args.variant == "unfused_tc":
             more.route_unfused_tc(X, R1, R2, k, scratch=scratch, out_idx=idx, out_gate=gate,
                                   out_expert_count=cnt, out_logits=logits, stream=st)
@@ -468,6 +488,13 @@ def main():
                 else "fallback 6.65 TB/s",
                 "tensor": {"achieved_tflops": flops / (kernel_ms / 1e3) / 1e12, "peak_tflops": tc,
                            "frac": flops / (kernel_ms / 1e3) / 1e12 / tc}}
+        if args.variant == "fullrank":
+            # tensor-bound: 2 N h M FLOP of x . W per launch (X read once: 2 N h bytes)
+            fflops = 2.0 * N * h * M / (kernel_ms / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": fflops, "peak": tc, "unit": "TFLOP/s", "frac": fflops / tc,
+                    "traffic": None, "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops)" if src == "measured"
+                    else "fallback 1.59 PFLOP/s",
+                    "hbm": {"achieved_gbs": achieved, "peak_gbs": hbm, "frac": achieved / hbm}}
         if args.variant == "backward":
             # fp32 FMA work without recompute: z, logits, zbar, Xbar, R1bar, R2bar (6 r (h + M) per
             # token) plus g (2 M); timed over the whole step (five launches)
@@ -477,7 +504,8 @@ def main():
             roof = {"bound": "alu", "achieved": achieved_t, "peak": fp32_peak, "unit": "TFLOP/s",
                     "frac": achieved_t / fp32_peak, "traffic": None, "timed": "whole backward step",
                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz clocks.max.sm"}
-        line = {"metric": METRIC if args.variant != "backward" else BACKWARD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        metric = {"backward": BACKWARD_METRIC, "fullrank": FULLRANK_METRIC}.get(args.variant, METRIC)
+        line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32" if args.variant == "backward" else "bf16", "data": "synthetic",
                 "config": {"workload": describe(args.workload) + (f" (N overridden to {N})" if args.tokens else ""),
@@ -490,8 +518,10 @@ def main():
         if e2e is not None:
             line["e2e"] = e2e
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = (backward_cpu_baseline if args.variant == "backward" else cpu_baseline)(
-                args.workload, args.cpu_seconds)
+            if args.variant == "backward":
+                line["cpu_baseline"] = backward_cpu_baseline(args.workload, args.cpu_seconds)
+            else:
+                line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, args.variant == "fullrank")
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

@@ -175,6 +175,23 @@ more_status more_route_unfused_static(const void* X, const void* R1, const void*
                                       int32_t* out_expert_count, float* out_logits, void* stream);
 
 /*
+ * The standard (full-rank) router, fused.  [MoRE App. H.3 "Fusing a standard MoE layer",
+ * Figs. 20-22]  Per token x: the M logits x . W, the top-k in routing order, softmax gates over
+ * the k and per-expert counts, with the same conventions and outputs as more_route.  W is
+ * streamed past every 128-token tile one 128-expert tile (all h rows) at a time and the N x M
+ * logits stay on chip.
+ *   X  bf16 [N][h]   token hidden vectors
+ *   W  bf16 [h][M]   router weight (one column per expert)
+ * Logits are fp32 sums of the exact bf16 products (tensor cores), ranked as they are.
+ * Requirements: those of more_route without r (h and M multiples of 8, 1 <= k <= M,
+ * k <= MORE_KMAX, M <= MORE_MMAX, pointers 16-byte aligned; X, out_idx and out_gate may be
+ * NULL only when N == 0).
+ */
+more_status more_route_fullrank(const void* X, const void* W, int64_t N, int h, int M, int k,
+                                int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
+                                float* out_logits, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the library's device error word
  * on the current device: MORE_OK if no kernel recorded an error since the last
  * call, MORE_ERR_DEVICE if one did (e.g. a bounded wait gave up), or

@@ -20,7 +20,7 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "auto_variant", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
+__all__ = ["route", "auto_variant", "route_fullrank", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
            "dispatch_scratch_bytes", "route_unfused", "route_unfused_tc", "route_unfused_static", "unfused_scratch_bytes", "device_status",
            "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
@@ -49,6 +49,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_variant.argtypes = route_args + [I, P]
     lib.more_route_unfused.restype = I
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
+    lib.more_route_fullrank.restype = I
+    lib.more_route_fullrank.argtypes = [P, P, I64, I, I, I, P, P, P, P, P]
     lib.more_route_auto_variant.restype = I
     lib.more_route_auto_variant.argtypes = [I64, I, I, I, I]
     lib.more_route_unfused_tc.restype = I
@@ -262,6 +264,22 @@ def auto_variant(N: int, h: int, r: int, M: int, k: int) -> str | None:
     or None if the shape fails the argument requirements."""
     v = int(_lib.more_route_auto_variant(N, h, r, M, k))
     return {value: name for name, value in VARIANTS.items()}[v] if v else None
+
+
+def route_fullrank(X, W, k: int, *, out_idx=None, out_gate=None, out_expert_count=None, out_logits=None,
+                   return_logits: bool = True, stream=None):
+    """The standard full-rank router x . W (W: h x M), fused (``more_route_fullrank``; App. H.3).
+    Same outputs as :func:`route`."""
+    X, W = _as_bf16(X, "X"), _as_bf16(W, "W")
+    N, h = X.shape
+    if W.shape[0] != h:
+        raise ValueError(f"W has {W.shape[0]} rows, X has {h} columns")
+    M = W.shape[1]
+    outs = _outputs(N, k, M, X.device, out_idx, out_gate, out_expert_count, out_logits, return_logits)
+    st = _lib.more_route_fullrank(_ptr(X), _ptr(W), N, h, M, k, _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
+                                  _ptr(outs[3]), _stream_handle(stream))
+    _check(st, "more_route_fullrank")
+    return outs
 
 
 def unfused_scratch_bytes(N: int, r: int, M: int) -> int:

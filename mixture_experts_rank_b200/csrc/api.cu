@@ -310,6 +310,21 @@ more_status more_route_unfused_tc(const void* X, const void* R1, const void* R2,
   return launch_unfused_tc(a, scratch) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
 }
 
+more_status more_route_fullrank(const void* X, const void* W, int64_t N, int h, int M, int k,
+                                int32_t* out_idx, float* out_gate, int32_t* out_expert_count,
+                                float* out_logits, void* stream) {
+  // the shape rules of more_route with the rank check left out (r = 16 stands for "any")
+  more_status st = validate_route(X, W, W, N, h, 16, M, k, out_idx, out_gate, out_expert_count, out_logits);
+  if (st != MORE_OK) return st;
+  RouteArgs a = make_args(X, nullptr, W, N, h, 0, M, k, out_idx, out_gate, out_expert_count, out_logits, stream);
+  a.status = status_word();
+  if (!a.status) return MORE_ERR_CUDA;
+  if (cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
+    return MORE_ERR_CUDA;
+  if (N == 0) return MORE_OK;
+  return launch_fullrank(a) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+}
+
 more_status more_device_status(void* stream, uint32_t* detail) {
   if (detail) *detail = 0;
   unsigned int* word = status_word();

@@ -79,6 +79,8 @@ cudaError_t launch_threshold_topk(const RouteArgs& a, const float* scores);
 // row-wise top-k; scratch as for launch_unfused.
 bool unfused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused_tc(const RouteArgs& a, void* scratch);
+// Fused full-rank router: a.R2 holds W (h x M); a.R1 and a.r are unused.
+cudaError_t launch_fullrank(const RouteArgs& a);
 
 // ---- small device helpers -------------------------------------------------
 

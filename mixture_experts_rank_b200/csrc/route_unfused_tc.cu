@@ -15,6 +15,7 @@
 #include <atomic>
 
 #include "more_internal.cuh"
+#include "mbar_wait.cuh"
 #include "sm100_ptx.cuh"
 
 namespace more {
@@ -28,7 +29,6 @@ constexpr int kRoleWarps = 4;  // producer, Z issuer, score issuer, (idle: keeps
 constexpr int kEpiWarps = 8;   // two warps per TMEM lane group, 64 score columns each
 constexpr int kThreads = (kRoleWarps + kEpiWarps) * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint32_t kStgBytes = 32 * 32 * 4;  // one staged store box: 32 tokens x 32 experts fp32
 constexpr uint32_t kSmemLimit = 227 * 1024;
 constexpr int kMaxR2Stages = 64;
@@ -102,42 +102,6 @@ __device__ __forceinline__ Bars bars_at(uint8_t* smem, const Params& p) {
   return r;
 }
 
-// Bounded mbarrier wait: suspends in hardware first; false once kTimeoutNs pass (the
-// device error word records it and the abort flag stops the other roles) or once another
-// thread has raised the abort flag.
-__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                           unsigned int* status) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
-    if ((spin & 3u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kTimeoutNs) {
-        atomicOr(status, MORE_DEVERR_WAIT_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned int* status) {
-  if (mbar_try_wait_sleep(bar, parity, 65536u)) return true;
-  return wait_bar_slow(bar, parity, abort_flag, status);
-}
-
-struct Ring {
-  int i = 0;
-  uint32_t phase = 0;
-  __device__ __forceinline__ void next(int n) {
-    if (++i == n) {
-      i = 0;
-      phase ^= 1u;
-    }
-  }
-};
-
 __device__ __forceinline__ int local_tiles(const Params& p) {
   return (int)blockIdx.x < p.num_tiles ? (p.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 }
@@ -162,7 +126,7 @@ __device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CU
   };
   if (p.r2_resident)
     for (int t = 0; t < p.p_count; ++t) load_r2(t, t);
-  Ring sx, sr;
+  RingPos sx, sr;
   int xt = 0, kb = 0;
   const int T = local_tiles(p);
   int q = 0, rt = 0;
@@ -204,7 +168,7 @@ __device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CU
       if (*reinterpret_cast<volatile int*>(b.abort_flag)) return;
       const uint64_t now = global_timer_ns();
       if (polls == 64) idle_since = now;
-      if (now - idle_since > kTimeoutNs) {
+      if (now - idle_since > kWaitLimitNs) {
         atomicOr(p.a.status, MORE_DEVERR_WAIT_TIMEOUT);
         *reinterpret_cast<volatile int*>(b.abort_flag) = 1;
         return;
@@ -217,16 +181,16 @@ __device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CU
 template <int R>
 __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R>;
-  Ring s;
+  RingPos s;
   int lt = 0;
   const uint32_t x0 = smem_u32(smem + p.off_x), r10 = smem_u32(smem + p.off_r1);
   for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
     const int buf = lt & 1;
-    if (!wait_bar(&b.zacc_empty[buf], ((lt >> 1) & 1) ^ 1u, b.abort_flag, p.a.status)) break;
+    if (!bounded_wait(&b.zacc_empty[buf], ((lt >> 1) & 1) ^ 1u, b.abort_flag, p.a.status)) break;
     tc_fence_after();
     const uint32_t d = tmem_base + C::ZCOL0 + buf * C::ZCOLS;
     for (int kb = 0; kb < p.kb_count; ++kb) {
-      if (!wait_bar(&b.x_full[s.i], s.phase, b.abort_flag, p.a.status)) goto done;
+      if (!bounded_wait(&b.x_full[s.i], s.phase, b.abort_flag, p.a.status)) goto done;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < C::BK / 16; ++kk) {
@@ -242,7 +206,7 @@ __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tm
   }
 done:
   mma_commit(&b.drain[0]);
-  wait_bar(&b.drain[0], 0, b.abort_flag, p.a.status);
+  bounded_wait(&b.drain[0], 0, b.abort_flag, p.a.status);
 }
 
 // ---- role: MMA issuer of the score tiles ---------------------------------------------------
@@ -250,24 +214,24 @@ done:
 template <int R>
 __device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R>;
-  Ring rs, d;
+  RingPos rs, d;
   const int T = local_tiles(p);
   const uint32_t zs0 = smem_u32(smem + p.off_zs), r20 = smem_u32(smem + p.off_r2);
   for (int j = 0; j < T; ++j) {
     const int zb = p.nz == 2 ? (j & 1) : 0, use = p.nz == 2 ? (j >> 1) : j;
-    if (!wait_bar(&b.zsm_full[zb], use & 1, b.abort_flag, p.a.status)) goto done;
+    if (!bounded_wait(&b.zsm_full[zb], use & 1, b.abort_flag, p.a.status)) goto done;
     {
       const uint32_t zs = zs0 + zb * C::ZS_BYTES;
       for (int t = 0; t < p.p_count; ++t) {
         int st;
         if (p.r2_resident) {
           st = t;
-          if (j == 0 && !wait_bar(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
+          if (j == 0 && !bounded_wait(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
         } else {
           st = rs.i;
-          if (!wait_bar(&b.r2_full[rs.i], rs.phase, b.abort_flag, p.a.status)) goto done;
+          if (!bounded_wait(&b.r2_full[rs.i], rs.phase, b.abort_flag, p.a.status)) goto done;
         }
-        if (!wait_bar(&b.s_empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
+        if (!bounded_wait(&b.s_empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
         tc_fence_after();
         const uint32_t dt = tmem_base + d.i * 128;
         const uint32_t r2 = r20 + st * C::R2_STAGE;
@@ -289,7 +253,7 @@ __device__ void mma_scores(const Params& p, const Bars& b, uint8_t* smem, uint32
   }
 done:
   mma_commit(&b.drain[1]);
-  wait_bar(&b.drain[1], 0, b.abort_flag, p.a.status);
+  bounded_wait(&b.drain[1], 0, b.abort_flag, p.a.status);
 }
 
 // ---- epilogue warps: z pair to shared memory, score tiles to HBM ---------------------------
@@ -306,14 +270,14 @@ __device__ void epilogue(const Params& p, const Bars& b, uint8_t* smem, uint32_t
   uint8_t* stg0 = smem + p.off_stg + (uint32_t)ew * p.nstg * kStgBytes;
   uint8_t* zs0 = smem + p.off_zs;
   int sc = 0;  // score boxes this warp has staged
-  Ring d;
+  RingPos d;
   const int T = local_tiles(p);
   for (int j = 0; j < T; ++j) {
     const int64_t n0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kBT;
     // z from TMEM -> (z_hi, z_lo) bf16 -> shared memory, R / 2 columns per warp
     {
       const int buf = j & 1;
-      if (!wait_bar(&b.zacc_full[buf], (j >> 1) & 1, b.abort_flag, a.status)) goto done;
+      if (!bounded_wait(&b.zacc_full[buf], (j >> 1) & 1, b.abort_flag, a.status)) goto done;
       tc_fence_after();
       constexpr int HALF = R / 2;
       uint32_t zr[HALF];
@@ -332,7 +296,7 @@ __device__ void epilogue(const Params& p, const Bars& b, uint8_t* smem, uint32_t
       __syncwarp();
       if (lane == 0) mbar_arrive(&b.zacc_empty[buf]);
       const int zb = p.nz == 2 ? (j & 1) : 0, use = p.nz == 2 ? (j >> 1) : j;
-      if (use > 0 && !wait_bar(&b.zsm_empty[zb], (use - 1) & 1, b.abort_flag, a.status)) goto done;
+      if (use > 0 && !bounded_wait(&b.zsm_empty[zb], (use - 1) & 1, b.abort_flag, a.status)) goto done;
       uint8_t* zs = zs0 + zb * C::ZS_BYTES;
 #pragma unroll
       for (int q = 0; q < HALF / 8; ++q) {
@@ -358,7 +322,7 @@ __device__ void epilogue(const Params& p, const Bars& b, uint8_t* smem, uint32_t
     const int row0 = (int)(n0 + sp * 32);
     const bool rows_in = n0 + sp * 32 < a.N;
     for (int pt = 0; pt < p.p_count; ++pt) {
-      if (!wait_bar(&b.s_full[d.i], d.phase, b.abort_flag, a.status)) goto done;
+      if (!bounded_wait(&b.s_full[d.i], d.phase, b.abort_flag, a.status)) goto done;
       tc_fence_after();
       uint32_t v[64];
       const uint32_t col = tmem_base + lane_base + d.i * 128 + hh * 64;

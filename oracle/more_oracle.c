@@ -64,12 +64,14 @@ void oracle_token_logits(const uint16_t* x, const uint16_t* R1, const uint16_t* 
   }
 }
 
-/* l = x . W for one token, W h x M (the standard router of App. H.3). */
+/* l = x . W for one token, W h x M (the standard router of App. H.3).  Each l[e] is summed
+   over t in increasing order; the loop runs along W's rows so that W is read in order. */
 void oracle_token_logits_full(const uint16_t* x, const uint16_t* W, int h, int M, double* logits) {
-  for (int e = 0; e < M; ++e) {
-    double s = 0.0;
-    for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);
-    logits[e] = s;
+  for (int e = 0; e < M; ++e) logits[e] = 0.0;
+  for (int t = 0; t < h; ++t) {
+    const double xt = oracle_bf16(x[t]);
+    const uint16_t* w = W + (size_t)t * M;
+    for (int e = 0; e < M; ++e) logits[e] += xt * oracle_bf16(w[e]);
   }
 }
 

@@ -68,25 +68,45 @@ def check_validity(idx, gate, counts, logits, M, k):
 
 def compare(X, R1, R2, N, h, r, M, k, idx, gate, counts, logits, rows=None, exact=False,
             logit_tol=LOGIT_TOL, gate_tol=GATE_TOL, min_set_fraction=0.5) -> ParityReport:
-    """Check GPU outputs (numpy) against the oracle on ``rows`` (default: every token).
+    """Check GPU outputs (numpy) of the low-rank router against the oracle on ``rows``
+    (default: every token).
 
     ``exact`` demands identical indices and counts on every token (for inputs whose
     logits are exact in fp32, e.g. small integers).
     """
+    rows_ = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = oracle.route(X, R1, R2, N, h, r, M, k, rows=rows_)
+    ref_at = lambda rr, ee: oracle.logits_at(X, R1, R2, N, h, r, M, rr, ee)
+    return _compare(o, ref_at, rows, rows_, M, k, idx, gate, counts, logits, exact, logit_tol, gate_tol,
+                    min_set_fraction)
+
+
+def compare_fullrank(X, W, N, h, M, k, idx, gate, counts, logits, rows=None, exact=False,
+                     logit_tol=LOGIT_TOL, gate_tol=GATE_TOL, min_set_fraction=0.5) -> ParityReport:
+    """:func:`compare` for the standard full-rank router x . W (App. H.3), by the same rules."""
+    rows_ = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = oracle.route_fullrank(X, W, N, h, M, k, rows=rows_)
+    ref_at = lambda rr, ee: oracle.logits_at_fullrank(X, W, N, h, M, rr, ee)
+    return _compare(o, ref_at, rows, rows_, M, k, idx, gate, counts, logits, exact, logit_tol, gate_tol,
+                    min_set_fraction)
+
+
+def _compare(o, ref_at, rows_arg, rows, M, k, idx, gate, counts, logits, exact, logit_tol, gate_tol,
+             min_set_fraction) -> ParityReport:
+    """The rules of this module, given the oracle's result ``o`` on ``rows`` and ``ref_at``,
+    the oracle's logits of (row, expert) pairs."""
     idx = np.asarray(idx)
     gate = np.asarray(gate)
     counts = np.asarray(counts)
     logits = None if logits is None else np.asarray(logits)
     check_validity(idx, gate, counts, logits, M, k)
-    all_rows = rows is None
-    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
-    o = oracle.route(X, R1, R2, N, h, r, M, k, rows=rows)
+    all_rows = rows_arg is None
     g_idx, g_gate = idx[rows], gate[rows]
     tol = logit_tol * o.rms
     max_logit = 0.0
     if rows.size:
         # oracle logits of the experts the GPU returned
-        ref = oracle.logits_at(X, R1, R2, N, h, r, M, np.repeat(rows, k), g_idx.ravel()).reshape(-1, k)
+        ref = ref_at(np.repeat(rows, k), g_idx.ravel()).reshape(-1, k)
         if logits is not None:
             err = np.abs(logits[rows] - ref)
             bad = err > tol[:, None]
@@ -169,5 +189,13 @@ def near_tie_rows(X, R1, R2, N, h, r, M, k, count, scan=None) -> np.ndarray:
     tie handling and exact re-check decide the result."""
     scan = np.arange(N) if scan is None else np.asarray(scan, dtype=np.int64)
     o = oracle.route(X, R1, R2, N, h, r, M, k, rows=scan)
+    rel = o.margin / np.maximum(o.rms, 1e-30)
+    return np.sort(scan[np.argsort(rel, kind="stable")[:count]])
+
+
+def near_tie_rows_fullrank(X, W, N, h, M, k, count, scan=None) -> np.ndarray:
+    """:func:`near_tie_rows` for the full-rank router x . W."""
+    scan = np.arange(N) if scan is None else np.asarray(scan, dtype=np.int64)
+    o = oracle.route_fullrank(X, W, N, h, M, k, rows=scan)
     rel = o.margin / np.maximum(o.rms, 1e-30)
     return np.sort(scan[np.argsort(rel, kind="stable")[:count]])

@@ -29,7 +29,7 @@ def lib():
 def test_header_declares_the_route_entry_points():
     names = declared_functions()
     for required in ("more_route", "more_route_variant", "more_route_train", "more_route_backward",
-                     "more_route_backward_scratch_bytes", "more_route_unfused", "more_route_unfused_tc",
+                     "more_route_backward_scratch_bytes", "more_route_unfused", "more_route_unfused_tc", "more_route_fullrank",
                      "more_route_unfused_scratch_bytes", "more_device_status", "more_status_string",
                      "more_abi_version"):
         assert required in names
@@ -94,6 +94,21 @@ def test_auto_variant_follows_the_measured_crossovers(shape, expected):
     fused kernel's shared-memory plan cannot hold."""
     import mixture_experts_rank_b200 as m
     assert m.auto_variant(*shape) == expected
+
+
+@pytest.mark.parametrize("kwargs,expected", [
+    (dict(k=0), 1), (dict(k=65), 1), (dict(N=-1), 1), (dict(h=4), 1), (dict(h=66), 1), (dict(M=70), 1),
+    (dict(X=0), 1), (dict(W=0), 1), (dict(idx=0), 1), (dict(cnt=0), 1), (dict(W=24), 1), (dict(logits=8), 1),
+    (dict(k=17, M=64), 2), (dict(M=262152), 2),
+])
+def test_fullrank_rejects_invalid_arguments(lib, kwargs, expected):
+    P = ctypes.c_void_p
+    args = dict(N=16, h=64, M=64, k=4, X=16, W=16, idx=16, gate=16, cnt=16, logits=None)
+    args.update(kwargs)
+    opt = lambda v: P(v) if v else None
+    st = lib.more_route_fullrank(opt(args["X"]), opt(args["W"]), args["N"], args["h"], args["M"], args["k"],
+                                 opt(args["idx"]), opt(args["gate"]), opt(args["cnt"]), opt(args["logits"]), None)
+    assert st == expected
 
 
 def test_unfused_tc_checks_rank_and_scratch(lib):

@@ -28,10 +28,10 @@ MUTATIONS = {
                           "for (int i = 1; i < r; ++i) s += z[i] * oracle_bf16(R2[(size_t)i * M + e]);\n    logits[e] = s;"),
     "dropped_hidden_term": ("for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(R1[(size_t)t * r + i]);\n    z[i] = s;",
                             "for (int t = 0; t + 1 < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(R1[(size_t)t * r + i]);\n    z[i] = s;"),
-    "fullrank_W_transposed": ("s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);",
-                              "s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)e * h + t]);"),
-    "fullrank_dropped_hidden_term": ("for (int t = 0; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);",
-                                     "for (int t = 1; t < h; ++t) s += oracle_bf16(x[t]) * oracle_bf16(W[(size_t)t * M + e]);"),
+    "fullrank_W_transposed": ("const uint16_t* w = W + (size_t)t * M;\n    for (int e = 0; e < M; ++e) logits[e] += xt * oracle_bf16(w[e]);",
+                              "for (int e = 0; e < M; ++e) logits[e] += xt * oracle_bf16(W[(size_t)e * h + t]);"),
+    "fullrank_dropped_hidden_term": ("for (int t = 0; t < h; ++t) {\n    const double xt",
+                                     "for (int t = 1; t < h; ++t) {\n    const double xt"),
     "softmax_sign": ("gate[j] = exp(sel_logit[j] - top) / denom;", "gate[j] = exp(top - sel_logit[j]) / denom;"),
     "softmax_missing_shift": ("denom += exp(sel_logit[j] - top);", "denom += exp(sel_logit[j]);"),
     "margin_wrong_runner_up": ("sel_logit[k - 1] - logits[scratch[k].e]",
