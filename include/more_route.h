@@ -250,10 +250,11 @@ more_status more_dispatch(const int32_t* idx, int64_t N, int k, int M, int32_t* 
 
 /*
  * more_dispatch with an explicit kernel variant; same arguments, scratch and result.
- *   MORE_DISPATCH_GLOBAL: histograms of 2048-slot chunks in global memory (as more_dispatch);
+ *   MORE_DISPATCH_GLOBAL: histograms of 2048-slot chunks in global memory;
  *   MORE_DISPATCH_SHARED: about two chunks per SM, each counted in a shared-memory histogram of
  *     M counters; requires M <= MORE_DISPATCH_SHARED_MMAX (else MORE_ERR_UNSUPPORTED).
- *   MORE_DISPATCH_AUTO:   the variant more_dispatch uses (GLOBAL).
+ *   MORE_DISPATCH_AUTO:   the variant more_dispatch uses: SHARED when M <= MORE_DISPATCH_SHARED_MMAX
+ *     (the faster of the two where both apply), GLOBAL otherwise.
  * Any other value returns MORE_ERR_INVALID_ARG.
  */
 #define MORE_DISPATCH_SHARED_MMAX 32768
