@@ -192,6 +192,16 @@ more_status more_route_fullrank(const void* X, const void* W, int64_t N, int h, 
                                 float* out_logits, void* stream);
 
 /*
+ * Self-test of the failure path.  Launches one bounded mbarrier wait that nothing completes, the
+ * same bounded wait every persistent kernel of the library uses.  After its limit (4 s) the wait
+ * gives up, records MORE_DEVERR_WAIT_TIMEOUT in the device error word and returns, leaving the
+ * context usable.  *out_result (device int32, 4-byte aligned) is set to 2 when the wait gave up
+ * (1 if it had completed).  Asynchronous on `stream`; read the outcome with more_device_status.
+ * Returns MORE_ERR_INVALID_ARG for a NULL out_result.
+ */
+more_status more_selftest_wait_timeout(int32_t* out_result, void* stream);
+
+/*
  * Synchronise `stream`, then return and clear the library's device error word
  * on the current device: MORE_OK if no kernel recorded an error since the last
  * call, MORE_ERR_DEVICE if one did (e.g. a bounded wait gave up), or

@@ -20,7 +20,7 @@ import torch
 
 from . import _build
 
-__all__ = ["route", "auto_variant", "route_fullrank", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
+__all__ = ["route", "auto_variant", "route_fullrank", "selftest_wait_timeout", "route_train", "route_backward", "route_backward_scratch_bytes", "dispatch",
            "dispatch_scratch_bytes", "route_unfused", "route_unfused_tc", "route_unfused_static", "unfused_scratch_bytes", "device_status",
            "Router", "MoreError", "VARIANTS", "library_path", "abi_version", "KMAX", "STATS_MMAX"]
 
@@ -51,6 +51,8 @@ def _load_library() -> ctypes.CDLL:
     lib.more_route_unfused.argtypes = route_args + [P, ctypes.c_size_t, P]
     lib.more_route_fullrank.restype = I
     lib.more_route_fullrank.argtypes = [P, P, I64, I, I, I, P, P, P, P, P]
+    lib.more_selftest_wait_timeout.restype = I
+    lib.more_selftest_wait_timeout.argtypes = [P, P]
     lib.more_route_auto_variant.restype = I
     lib.more_route_auto_variant.argtypes = [I64, I, I, I, I]
     lib.more_route_unfused_tc.restype = I
@@ -338,6 +340,15 @@ def route_unfused_static(X, R1, R2, k: int, *, out_idx=None, out_gate=None, out_
                                         _ptr(outs[1]), _ptr(outs[2]), _ptr(outs[3]), _stream_handle(stream))
     _check(st, "more_route_unfused_static")
     return outs
+
+
+def selftest_wait_timeout(stream=None) -> torch.Tensor:
+    """Run the failure-path self-test (``more_selftest_wait_timeout``): one bounded wait that
+    nothing completes.  Returns the device int32 result (2 once the wait gave up); the device
+    error word then holds MORE_DEVERR_WAIT_TIMEOUT (read it with :func:`device_status`)."""
+    out = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(_lib.more_selftest_wait_timeout(_ptr(out), _stream_handle(stream)), "more_selftest_wait_timeout")
+    return out
 
 
 def device_status(stream=None) -> int:

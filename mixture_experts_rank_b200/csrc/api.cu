@@ -328,6 +328,15 @@ more_status more_route_fullrank(const void* X, const void* W, int64_t N, int h, 
   return launch_fullrank(a) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
 }
 
+more_status more_selftest_wait_timeout(int32_t* out_result, void* stream) {
+  if (!out_result || (reinterpret_cast<uintptr_t>(out_result) & 3u)) return MORE_ERR_INVALID_ARG;
+  unsigned int* status = status_word();
+  if (!status) return MORE_ERR_CUDA;
+  return launch_wait_timeout_probe(status, out_result, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MORE_OK
+             : MORE_ERR_CUDA;
+}
+
 more_status more_device_status(void* stream, uint32_t* detail) {
   if (detail) *detail = 0;
   unsigned int* word = status_word();

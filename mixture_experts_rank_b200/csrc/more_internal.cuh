@@ -81,6 +81,9 @@ bool unfused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused_tc(const RouteArgs& a, void* scratch);
 // Fused full-rank router: a.R2 holds W (h x M); a.R1 and a.r are unused.
 cudaError_t launch_fullrank(const RouteArgs& a);
+// One bounded wait that nothing completes (the failure path's self-test); writes 2 to
+// *out_result when the wait gave up, 1 if it completed.
+cudaError_t launch_wait_timeout_probe(unsigned int* status, int32_t* out_result, cudaStream_t stream);
 
 // ---- small device helpers -------------------------------------------------
 

@@ -16,7 +16,8 @@ def pytest_configure(config):
 # that under -x a failure in a later row cannot hide an earlier row's results.  The test of
 # the allocation-free entry point runs last of all.
 GPU_FILE_ORDER = ("test_gpu_parity", "test_gpu_train_stats", "test_gpu_dispatch", "test_gpu_variant_cluster",
-                  "test_gpu_training_backward", "test_gpu_variant_dispatch", "test_gpu_fullrank", "test_zz_no_alloc")
+                  "test_gpu_training_backward", "test_gpu_variant_dispatch", "test_gpu_fullrank", "test_gpu_wait_timeout",
+                  "test_zz_no_alloc")
 
 
 def pytest_collection_modifyitems(config, items):

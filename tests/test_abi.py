@@ -111,6 +111,12 @@ def test_fullrank_rejects_invalid_arguments(lib, kwargs, expected):
     assert st == expected
 
 
+def test_selftest_checks_its_output_pointer(lib):
+    P = ctypes.c_void_p
+    assert lib.more_selftest_wait_timeout(None, None) == 1
+    assert lib.more_selftest_wait_timeout(P(18), None) == 1   # not 4-byte aligned
+
+
 def test_unfused_tc_checks_rank_and_scratch(lib):
     """The tensor-core materialisation takes r in {16, 32, 64, 128} and the unfused scratch size."""
     n = lib.more_route_unfused_scratch_bytes(1000, 32, 256)
