@@ -187,7 +187,11 @@ more_status more_route_train(const void* X, const void* R1, const void* R2, int6
   RouteArgs a = make_args(X, R1, R2, N, h, r, M, k, out_idx, out_gate, out_expert_count, out_logits,
                           stream);
   if (cudaMemsetAsync(out_psum, 0, sizeof(float) * (size_t)M, a.stream) != cudaSuccess) return MORE_ERR_CUDA;
-  return launch_train_stats(a, out_m, out_Z, out_psum) == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
+  if (N == 0) return MORE_OK;
+  // the tensor-core statistics where the rank and shared-memory plan allow, else the CUDA-core kernel
+  const cudaError_t err = train_stats_tc_supports(a) ? launch_train_stats_tc(a, out_m, out_Z, out_psum)
+                                                     : launch_train_stats(a, out_m, out_Z, out_psum);
+  return err == cudaSuccess ? MORE_OK : MORE_ERR_CUDA;
 }
 
 size_t more_dispatch_scratch_bytes(int64_t N, int k, int M) {

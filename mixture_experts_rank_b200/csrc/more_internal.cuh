@@ -79,6 +79,10 @@ cudaError_t launch_threshold_topk(const RouteArgs& a, const float* scores);
 // row-wise top-k; scratch as for launch_unfused.
 bool unfused_tc_supports(const RouteArgs& a);
 cudaError_t launch_unfused_tc(const RouteArgs& a, void* scratch);
+// Training statistics (App. F, Algorithm 2) from the same tensor-core logits: m, Z per token
+// and psum per expert (psum accumulated with atomics: zero it first).
+bool train_stats_tc_supports(const RouteArgs& a);
+cudaError_t launch_train_stats_tc(const RouteArgs& a, float* out_m, float* out_Z, float* out_psum);
 // Fused full-rank router: a.R2 holds W (h x M); a.R1 and a.r are unused.
 cudaError_t launch_fullrank(const RouteArgs& a);
 // One bounded wait that nothing completes (the failure path's self-test); writes 2 to
