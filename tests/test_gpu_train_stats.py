@@ -60,7 +60,8 @@ def test_sweep_shape_train_stats():
     check_stats(16384, 512, 32, 2048, 8)
 
 
-@pytest.mark.parametrize("N,h,r,M,k", [(37, 72, 16, 200, 1), (300, 256, 64, 16, 16), (513, 128, 128, 1000, 8)])
+@pytest.mark.parametrize("N,h,r,M,k", [(37, 72, 16, 200, 1), (300, 256, 64, 16, 16), (513, 128, 128, 1000, 8),
+                                       (129, 136, 48, 64, 8)])   # r = 48: the CUDA-core statistics kernel
 def test_ragged_train_stats(N, h, r, M, k):
     check_stats(N, h, r, M, k)
 
