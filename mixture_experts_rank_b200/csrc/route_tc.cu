@@ -53,6 +53,7 @@
 #include <atomic>
 
 #include "more_internal.cuh"
+#include "mbar_wait.cuh"
 #include "sm100_ptx.cuh"
 #include "warp_simt.cuh"
 
@@ -81,7 +82,6 @@ constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more
 constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
 static_assert(kFbBatch <= kWarpsB, "one merging warp per fallback token of a batch");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr uint32_t kRealKey = 0x00800000u;  // ordered value of -FLT_MAX: keys below are not real chunks
 
 // ---- parameters -----------------------------------------------------------------------
@@ -205,32 +205,6 @@ __device__ __forceinline__ Bars bars_at(uint8_t* smem, const Params& p) {
 constexpr uint32_t kBarSlots = 16 + 128 + 2 * 12 + 3;  // up to and with drain
 constexpr uint32_t kBarBytes = kBarSlots * 8 + 16;
 
-// Slow path of the bounded mbarrier wait: false once the limit passes or another
-// thread gave up.
-__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                           unsigned int* status) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
-    if ((spin & 3u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kTimeoutNs) {
-        atomicOr(status, MORE_DEVERR_WAIT_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// The first attempt suspends in hardware until the phase completes (or ~65 us pass),
-// so a normal wait is one instruction and the bounded loop is a rare call.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         unsigned int* status) {
-  if (mbar_try_wait_sleep(bar, parity, 65536u)) return true;
-  return wait_bar_slow(bar, parity, abort_flag, status);
-}
-
 // Bounded entry barrier of one group's warps (an mbarrier, so that a warp of the
 // group that gave up elsewhere cannot leave the others waiting without limit).  `phase` is
 // the calling thread's parity of the barrier, flipped at every use.
@@ -238,7 +212,7 @@ __device__ __forceinline__ bool group_enter(uint64_t* gbar, uint32_t& phase, vol
                                             unsigned int* status) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(gbar);
-  const bool ok = wait_bar(gbar, phase, abort_flag, status);
+  const bool ok = bounded_wait(gbar, phase, abort_flag, status);
   phase ^= 1u;
   return ok;
 }
@@ -312,24 +286,13 @@ __device__ __forceinline__ int local_tiles(const Params& p) {
   return (int)blockIdx.x < p.num_tiles ? (p.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
 }
 
-// Position of one thread in a ring of mbarrier-guarded buffers.
-struct Ring {
-  int i = 0;
-  uint32_t phase = 0;
-  __device__ __forceinline__ void next(int n) {
-    if (++i == n) {
-      i = 0;
-      phase ^= 1u;
-    }
-  }
-};
 
 // ---- role: TMA producer of X, R1 and R2 ---------------------------------------------
 //
 // One thread keeps both rings full: X and R1 stages in tile order, R2 tiles in sweep order
 // (or, when R2 is resident, all of them once).  It polls the rings' empty barriers without
 // blocking and backs off briefly when neither has room, so a slow ring never holds up the
-// other.  It gives up like every bounded wait: after kTimeoutNs without progress, or when
+// other.  It gives up like every bounded wait: after kWaitLimitNs without progress, or when
 // another role has raised the abort flag.
 
 template <int R, int KCAP>
@@ -345,7 +308,7 @@ __device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CU
   if (p.r2_resident)
     for (int t = 0; t < p.p_count; ++t) load_r2(t, t);
   // X side: local tile xt, hidden block kb
-  Ring sx, sr;
+  RingPos sx, sr;
   int xt = 0, kb = 0;
   const int T = local_tiles(p);
   // R2 side: stage t of sweep q
@@ -388,7 +351,7 @@ __device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CU
       if (*reinterpret_cast<volatile int*>(b.abort_flag)) return;
       const uint64_t now = global_timer_ns();
       if (polls == 64) idle_since = now;
-      if (now - idle_since > kTimeoutNs) {
+      if (now - idle_since > kWaitLimitNs) {
         atomicOr(p.a.status, MORE_DEVERR_WAIT_TIMEOUT);
         *reinterpret_cast<volatile int*>(b.abort_flag) = 1;
         return;
@@ -402,16 +365,16 @@ __device__ void producer(const Params& p, const Bars& b, uint8_t* smem, const CU
 template <int R, int KCAP>
 __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  Ring s;
+  RingPos s;
   int lt = 0;
   const uint32_t x0 = smem_u32(smem + p.off_x), r10 = smem_u32(smem + p.off_r1);
   for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
     const int buf = lt & 1;
-    if (!wait_bar(&b.zacc_empty[buf], ((lt >> 1) & 1) ^ 1u, b.abort_flag, p.a.status)) break;
+    if (!bounded_wait(&b.zacc_empty[buf], ((lt >> 1) & 1) ^ 1u, b.abort_flag, p.a.status)) break;
     tc_fence_after();
     const uint32_t d = tmem_base + C::ZCOL0 + buf * C::ZCOLS;
     for (int kb = 0; kb < p.kb_count; ++kb) {
-      if (!wait_bar(&b.x_full[s.i], s.phase, b.abort_flag, p.a.status)) goto done;
+      if (!bounded_wait(&b.x_full[s.i], s.phase, b.abort_flag, p.a.status)) goto done;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < C::BK / 16; ++kk) {
@@ -427,7 +390,7 @@ __device__ void mma_z(const Params& p, const Bars& b, uint8_t* smem, uint32_t tm
   }
 done:
   mma_commit(&b.drain[0]);
-  wait_bar(&b.drain[0], 0, b.abort_flag, p.a.status);
+  bounded_wait(&b.drain[0], 0, b.abort_flag, p.a.status);
 }
 
 // ---- roles: MMA issuers of the logit passes ---------------------------------------------
@@ -440,7 +403,7 @@ done:
 template <int R, int KCAP, bool PASS_B>
 __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  Ring rs, d;
+  RingPos rs, d;
   const int T = local_tiles(p), nsw = sweep_count(T, p.interleave);
   const uint32_t zs0 = smem_u32(smem + p.off_zs), r20 = smem_u32(smem + p.off_r2);
   uint64_t* full = PASS_B ? b.b_full : b.a_full;
@@ -457,17 +420,17 @@ __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t
       int st;
       if (p.r2_resident) {
         st = t;
-        if (q == 0 && !wait_bar(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
+        if (q == 0 && !bounded_wait(&b.r2_full[t], 0, b.abort_flag, p.a.status)) goto done;
       } else {
         st = rs.i;
-        if (!wait_bar(&b.r2_full[rs.i], rs.phase, b.abort_flag, p.a.status)) goto done;
+        if (!bounded_wait(&b.r2_full[rs.i], rs.phase, b.abort_flag, p.a.status)) goto done;
       }
       if (j >= 0) {
         // the tile's z buffer is written by group A's epilogue
-        if (t == 0 && !wait_bar(&b.zsm_full[zs_buf(j, p.interleave)], zs_use(j, p.interleave) & 1, b.abort_flag,
+        if (t == 0 && !bounded_wait(&b.zsm_full[zs_buf(j, p.interleave)], zs_use(j, p.interleave) & 1, b.abort_flag,
                                 p.a.status))
           goto done;
-        if (!wait_bar(&empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
+        if (!bounded_wait(&empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
         tc_fence_after();
         const uint32_t dt = tmem_base + COL0 + d.i * 128;
         const uint32_t r2 = r20 + st * C::R2_STAGE;
@@ -498,7 +461,7 @@ __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t
   }
 done:
   mma_commit(&b.drain[PASS_B ? 2 : 1]);
-  wait_bar(&b.drain[PASS_B ? 2 : 1], 0, b.abort_flag, p.a.status);
+  bounded_wait(&b.drain[PASS_B ? 2 : 1], 0, b.abort_flag, p.a.status);
 }
 
 // ---- group A: epilogue, pass A, select ------------------------------------------------------
@@ -524,7 +487,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
   float* znorm = reinterpret_cast<float*>(smem + p.off_znorm);  // [hi h0 | hi h1 | lo h0 | lo h1][token]
   float* cnorm = reinterpret_cast<float*>(smem + p.off_cnorm);  // [8] per warp, [8] = result
   uint32_t gph = 0;
-  Ring ad, rs;
+  RingPos ad, rs;
   float colmax2 = 0.f;  // this warp's largest squared R2 column norm (first tile)
   const int T = local_tiles(p);
   uint32_t kl[KL];
@@ -535,7 +498,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     // ---------------- epilogue: Z from TMEM -> (z_hi, z_lo) -> shared memory ----------------
     {
       const int buf = j & 1;
-      if (!wait_bar(&b.zacc_full[buf], (j >> 1) & 1, b.abort_flag, a.status)) return;
+      if (!bounded_wait(&b.zacc_full[buf], (j >> 1) & 1, b.abort_flag, a.status)) return;
       tc_fence_after();
       constexpr int HALF = R / 2;
       uint32_t zr[HALF];
@@ -555,7 +518,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       if (lane == 0) mbar_arrive(&b.zacc_empty[buf]);
       // the previous tile of this z buffer: its pass B MMAs and its finalize are done
       const int zb = zs_buf(j, p.interleave), u = zs_use(j, p.interleave);
-      if (u > 0 && !wait_bar(&b.zsm_empty[zb], (u - 1) & 1, b.abort_flag, a.status)) return;
+      if (u > 0 && !bounded_wait(&b.zsm_empty[zb], (u - 1) & 1, b.abort_flag, a.status)) return;
       uint8_t* zs = zs0 + zb * C::ZS_BYTES;
       float hi2 = 0.f, lo2 = 0.f;
 #pragma unroll
@@ -590,7 +553,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
 #pragma unroll
     for (int i = 0; i < KL; ++i) kl[i] = 0u;
     for (int pt = 0; pt < p.p_count; ++pt) {
-      if (!wait_bar(&b.a_full[ad.i], ad.phase, b.abort_flag, a.status)) return;
+      if (!bounded_wait(&b.a_full[ad.i], ad.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
       const uint32_t col = tmem_base + lane_base + ad.i * 128 + hh * 64;
       const int c0 = pt * 4 + 2 * hh;
@@ -619,10 +582,10 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         int st;
         if (p.r2_resident) {
           st = pt;
-          if (!wait_bar(&b.r2_full[pt], 0, b.abort_flag, a.status)) return;
+          if (!bounded_wait(&b.r2_full[pt], 0, b.abort_flag, a.status)) return;
         } else {
           st = rs.i;
-          if (!wait_bar(&b.r2_full[rs.i], rs.phase, b.abort_flag, a.status)) return;
+          if (!bounded_wait(&b.r2_full[rs.i], rs.phase, b.abort_flag, a.status)) return;
         }
         const uint8_t* base = r2s + st * C::R2_STAGE;
         const int el = 16 * aw + (lane & 15);
@@ -645,7 +608,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     // ---------------- select: merge the lists, certified window, needed pairs --------------
     const int pb = j & 1, pu = j >> 1;  // pair buffer and its use count
     // the pair buffer's previous tile (j - 2) is finalized by group B
-    if (pu > 0 && !wait_bar(&b.pairs_empty[pb], (pu - 1) & 1, b.abort_flag, a.status)) return;
+    if (pu > 0 && !bounded_wait(&b.pairs_empty[pb], (pu - 1) & 1, b.abort_flag, a.status)) return;
     uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs + pb * C::PAIR_BYTES);
     int* cbase = reinterpret_cast<int*>(smem + p.off_cbase) + pb * (p.nchunks + 1);
     uint8_t* flag = smem + p.off_flag + pb * kBT;
@@ -856,13 +819,13 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
   uint8_t* fbmark = smem + p.off_fb + 4 + kBT;  // 1: the token's outputs come from the fallback
   uint2* part = reinterpret_cast<uint2*>(smem + p.off_part);
   uint32_t gph = 0;
-  Ring bd;
+  RingPos bd;
   const int T = local_tiles(p);
 
   for (int j = 0; j < T; ++j) {
     const int64_t n0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kBT;
     const int pb = j & 1, pu = j >> 1;
-    if (!wait_bar(&b.pairs_full[pb], pu & 1, b.abort_flag, a.status)) return;
+    if (!bounded_wait(&b.pairs_full[pb], pu & 1, b.abort_flag, a.status)) return;
     const uint2* pairs = reinterpret_cast<const uint2*>(smem + p.off_pairs + pb * C::PAIR_BYTES);
     const int* cbase = reinterpret_cast<const int*>(smem + p.off_cbase) + pb * (p.nchunks + 1);
     const uint8_t* flag = smem + p.off_flag + pb * kBT;
@@ -879,7 +842,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         lo = c_lo + (n * hh) / kPerTokB;
         hi = c_lo + (n * (hh + 1)) / kPerTokB;
       }
-      if (!wait_bar(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
+      if (!bounded_wait(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
       const int e = 32 * c + lane;
       const bool e_ok = e < a.M;
