@@ -45,13 +45,15 @@ RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, in
   a.out_logits = out_logits;
   a.status = nullptr;
   a.stream = static_cast<cudaStream_t>(stream);
+  a.zero_counts = 0;
   return a;
 }
 
 // AUTO's choice of kernel, from per-call times measured on a B200 (CUDA-graph replays of
 // back-to-back calls; h = 2048, M = 4096 with r = 16, 32 and 128):
-// - below 256 tokens the small-N kernel (one CTA per token) is fastest or level;
-// - from 256 tokens the cluster kernel overtakes it.  Its time grows linearly,
+// - up to 148 tokens the small-N kernel (one CTA per token, one CTA per SM: a single wave on
+//   the 148 SMs of a B200) is fastest or level;
+// - beyond, it needs a second wave and the cluster kernel overtakes it.  Its time grows linearly,
 //   about 12 us + N * 2.3e-7 us * r * (h + M) (r = 32: 58 us at N = 1024, 104 us at 2048);
 // - the fused kernel's time has a floor until every SM holds a tile: the chain of one
 //   128-token tile (Z over h, then two sweeps over the M / 128 expert tiles), about
@@ -59,7 +61,7 @@ RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, in
 // AUTO takes the cluster kernel while its estimate is below that floor, the fused kernel
 // beyond (when its shared-memory plan fits the shape), and the cluster kernel at any N for
 // shapes the fused kernel does not take.
-constexpr int64_t kClusterMinTokens = 256;
+constexpr int64_t kClusterMinTokens = 149;
 
 double cluster_estimate_us(int64_t N, int h, int r, int M) {
   return 12.0 + (double)N * 2.3e-7 * r * ((double)h + M);
@@ -143,10 +145,12 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
                           stream);
   a.status = status_word();
   if (!a.status) return MORE_ERR_CUDA;
-  if (cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
+  if (N > 0 && variant == MORE_VARIANT_AUTO) variant = auto_variant(a);
+  // a single token routed by the small-N kernel runs on one CTA, which zeroes the counts itself
+  a.zero_counts = (N == 1 && variant == MORE_VARIANT_SMALL_N) ? 1 : 0;
+  if (!a.zero_counts && cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
     return MORE_ERR_CUDA;
   if (N == 0) return MORE_OK;
-  if (variant == MORE_VARIANT_AUTO) variant = auto_variant(a);
   cudaError_t err;
   if (variant == MORE_VARIANT_FUSED_TC) {
     if (!fused_tc_supports(a)) return MORE_ERR_UNSUPPORTED;

@@ -21,6 +21,7 @@ struct RouteArgs {
   float* out_logits;  // may be null
   unsigned int* status;  // device error word (MORE_DEVERR_* bits)
   cudaStream_t stream;
+  int zero_counts;  // the kernel zeroes out_count itself (single-CTA calls; no memset issued)
 };
 
 // Argument checks of the routing entry points (more_route.h): MORE_OK or the error to return.

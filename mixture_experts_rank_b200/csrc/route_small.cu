@@ -34,19 +34,68 @@ __device__ __forceinline__ void warp_partial_z16(const __nv_bfloat16* __restrict
   warp_partial_z16_strided(x, R1, h, r, b, warp * 32 + lane, kWarpsPerBlock * 32, lane, value, index);
 }
 
+// The same for 32 columns b .. b + 31 (r a multiple of 32): every hidden row's 64-byte slice of
+// R1 is loaded at once, and the 5-step reduce-scatter leaves column b + lane on lane `lane`.
+__device__ __forceinline__ float warp_partial_z32(const __nv_bfloat16* __restrict__ x,
+                                                  const __nv_bfloat16* __restrict__ R1, int h, int r, int b,
+                                                  int warp, int lane) {
+  constexpr int kStride = kWarpsPerBlock * 32;
+  float acc[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+  for (int t0 = warp * 32 + lane; t0 < h; t0 += 4 * kStride) {
+    float xt[4];
+    uint4 w[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + j * kStride;
+      const bool ok = t < h;
+      xt[j] = ok ? __bfloat162float(x[t]) : 0.f;
+      const uint4* src = reinterpret_cast<const uint4*>(R1 + (size_t)(ok ? t : 0) * r + b);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[j][q] = ok ? __ldg(src + q) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w[j][q]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __bfloat1622float2(wp[u]);
+          acc[8 * q + 2 * u] = fmaf(xt[j], f.x, acc[8 * q + 2 * u]);
+          acc[8 * q + 2 * u + 1] = fmaf(xt[j], f.y, acc[8 * q + 2 * u + 1]);
+        }
+      }
+  }
+  // reduce-scatter: after the step with distance dd a lane keeps the half of its columns
+  // selected by its own bit dd; lane L ends with column L
+#pragma unroll
+  for (int dd = 16, wd = 16; dd >= 1; dd >>= 1, wd >>= 1) {
+    const bool up = lane & dd;
+#pragma unroll
+    for (int q = 0; q < wd; ++q) {
+      const float send = up ? acc[q] : acc[q + wd];
+      acc[q] = (up ? acc[q + wd] : acc[q]) + __shfl_xor_sync(0xffffffffu, send, dd);
+    }
+  }
+  return acc[0];
+}
+
 // Logits of this lane's 8 experts e0 .. e0 + 7 (one 16-byte load per R2 row, batches of
-// 8 rows); zs holds z_i as the bf16 pair sum.  ok is false for a lane past the last expert.
+// 16 rows whose loads are issued together); zs holds z_i as the bf16 pair sum.  ok is false
+// for a lane past the last expert.
 __device__ __forceinline__ void lane_logits8(const RouteArgs& a, const float* zs, int e0, bool ok, float* acc) {
   const uint4* src = reinterpret_cast<const uint4*>(a.R2) + (ok ? (e0 >> 3) : 0);
   const size_t rowv = (size_t)(a.M >> 3);
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-  for (int i0 = 0; i0 < a.r; i0 += 8) {
-    uint4 w[8];
+  for (int i0 = 0; i0 < a.r; i0 += 16) {  // r is a multiple of 16
+    uint4 w[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) w[j] = ok ? __ldg(src + (size_t)(i0 + j) * rowv) : make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < 16; ++j) w[j] = ok ? __ldg(src + (size_t)(i0 + j) * rowv) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 16; ++j) {
       const float zi = zs[i0 + j];
       const __nv_bfloat162* wp = reinterpret_cast<const __nv_bfloat162*>(&w[j]);
 #pragma unroll
@@ -67,14 +116,24 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   __shared__ float pv[kWarpsPerBlock][K];
   __shared__ int pe[kWarpsPerBlock][K];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (a.zero_counts) {
+    // a single-token call on one CTA: the counts are zeroed here instead of by a separate
+    // memset, and this CTA's own atomics below follow the barrier
+    for (int i = threadIdx.x; i < a.M; i += blockDim.x) a.out_count[i] = 0;
+    __syncthreads();
+  }
   for (int64_t n = blockIdx.x; n < a.N; n += gridDim.x) {
-    // 1. z = x . R1
+    // 1. z = x . R1 (32 columns per pass where r allows, else 16)
     const __nv_bfloat16* x = a.X + (size_t)n * a.h;
-    for (int b = 0; b < a.r; b += 16) {
-      float v;
-      int i;
-      warp_partial_z16(x, a.R1, a.h, a.r, b, warp, lane, v, i);
-      if ((lane & 1) == 0) zpart[warp][i] = v;
+    if ((a.r & 31) == 0) {
+      for (int b = 0; b < a.r; b += 32) zpart[warp][b + lane] = warp_partial_z32(x, a.R1, a.h, a.r, b, warp, lane);
+    } else {
+      for (int b = 0; b < a.r; b += 16) {
+        float v;
+        int i;
+        warp_partial_z16(x, a.R1, a.h, a.r, b, warp, lane, v, i);
+        if ((lane & 1) == 0) zpart[warp][i] = v;
+      }
     }
     __syncthreads();
     if (threadIdx.x < a.r) {

@@ -78,7 +78,6 @@ constexpr int kNamedBarA = 1, kNamedBarB = 2;    // bar.sync ids of the groups
 static_assert(kWarpsB % 4 == 0, "group B covers the four TMEM lane groups evenly");
 static_assert((kWarpsB & (kWarpsB - 1)) == 0, "fallback teams divide group B evenly");
 constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass B
-constexpr int kPoolSlots = 4;   // per-token overflow slots for chunks with more than one candidate
 constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
 static_assert(kFbBatch <= kWarpsB, "one merging warp per fallback token of a batch");
 constexpr uint32_t kTmemCols = 512;
@@ -112,6 +111,10 @@ template <int R, int KCAP>
 struct Cfg {
   static constexpr int KL = KCAP + 6;                  // chunk keys kept per token and warp
   static constexpr int KLP = (KL + 15) & ~15;          // row stride of the candidate slots and counts
+  // per-token slots for candidates beyond the first of a chunk: at k <= 4 the few chunks of a
+  // small expert pool hold several candidates each, so eight (an overflow sends the token to the
+  // exact fallback)
+  static constexpr int POOL = KCAP <= 4 ? 8 : 4;
   static constexpr int RK = 2 * R;                     // z_hi | z_lo columns of the z buffer
   // one pair buffer: the (token, chunk) pairs of a tile, later its output staging (3 x 128 x k words)
   static constexpr uint32_t PAIR_BYTES = kBT * KL * 8 > 3 * kBT * KCAP * 4 ? kBT * KL * 8 : 3 * kBT * KCAP * 4;
@@ -800,7 +803,7 @@ template <int R, int KCAP>
 __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
   constexpr int KL = C::KL;
-  constexpr int NC = KL + kPoolSlots;
+  constexpr int NC = KL + C::POOL;
   const RouteArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bw = warp - kWarpB0;        // 0 .. kWarpsB - 1
@@ -880,7 +883,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
             if (((bal[q] >> lane) & 1u) && (bal[q] & lt_mask)) {
               const int tok = ent[q].x & 0xff;
               const int ps = atomicAdd(&poolcnt[tok], 1);
-              if (ps < kPoolSlots) pool[ps * kBT + tok] = make_uint2(val[q], (uint32_t)e);
+              if (ps < C::POOL) pool[ps * kBT + tok] = make_uint2(val[q], (uint32_t)e);
             }
           }
         }
@@ -936,7 +939,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         o[q] = has ? ord_key(__uint_as_float(cv.x) + 0.f) : 0u;
         e[q] = cv.y;
       }
-      fb = (f & 1) || np > kPoolSlots || total < a.k;
+      fb = (f & 1) || np > C::POOL || total < a.k;
       if (hh == 0) {
         fbmark[t] = fb ? 1 : 0;
         if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
@@ -1169,7 +1172,7 @@ uint32_t layout(Params& p, int xs, int r2n, int nz) {
   p.off_pc = off = align_up(off, 16);
   off += kBT * C::KLP;
   p.off_pool = off = align_up(off, 8);
-  off += kBT * kPoolSlots * 8;
+  off += kBT * C::POOL * 8;
   p.off_poolcnt = off;
   off += kBT * 4;
   p.off_fb = off;  // fallback count, the tile's fallback tokens, per-token mark

@@ -51,6 +51,7 @@ extern "C" int emu_route_cluster(const void* X, const void* R1, const void* R2, 
   a.out_logits = logits;
   a.status = status;
   a.stream = nullptr;
+  a.zero_counts = 0;
   memset(cnt, 0, sizeof(int32_t) * M);  // the C entry point zeroes the counts before launching
   emu::cluster_size = 8;                 // cluster_route_kernel's __cluster_dims__
   const int rc = (int)more::launch_cluster(a);
@@ -76,6 +77,7 @@ more::RouteArgs route_args(const void* X, const void* R1, const void* R2, int64_
   a.out_logits = logits;
   a.status = status;
   a.stream = nullptr;
+  a.zero_counts = 0;
   if (cnt) memset(cnt, 0, sizeof(int32_t) * M);
   return a;
 }
@@ -84,6 +86,17 @@ more::RouteArgs route_args(const void* X, const void* R1, const void* R2, int64_
 extern "C" int emu_route_small(const void* X, const void* R1, const void* R2, int64_t N, int h, int r, int M, int k,
                                int32_t* idx, float* gate, int32_t* cnt, float* logits, unsigned* status) {
   return (int)more::launch_small_n(route_args(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, status));
+}
+
+// One token on the small-N kernel with the counts zeroed by the kernel itself (as more_route does
+// for N == 1): the counts start as garbage here.
+extern "C" int emu_route_small_self_zero(const void* X, const void* R1, const void* R2, int h, int r, int M, int k,
+                                         int32_t* idx, float* gate, int32_t* cnt, float* logits, unsigned* status) {
+  more::RouteArgs a = route_args(X, R1, R2, 1, h, r, M, k, idx, gate, nullptr, logits, status);
+  a.out_count = cnt;
+  for (int e = 0; e < M; ++e) cnt[e] = 7;
+  a.zero_counts = 1;
+  return (int)more::launch_small_n(a);
 }
 
 extern "C" long emu_unfused_scratch_bytes(int64_t N, int r, int M) { return (long)more::unfused_scratch_bytes(N, r, M); }

@@ -78,8 +78,8 @@ def test_unfused_scratch_size_and_checks(lib):
 
 
 @pytest.mark.parametrize("shape,expected", [
-    ((1, 2048, 32, 4096, 8), "small_n"), ((255, 2048, 32, 4096, 8), "small_n"),
-    ((256, 2048, 32, 4096, 8), "cluster"), ((1024, 2048, 32, 4096, 8), "cluster"),
+    ((1, 2048, 32, 4096, 8), "small_n"), ((148, 2048, 32, 4096, 8), "small_n"),
+    ((149, 2048, 32, 4096, 8), "cluster"), ((1024, 2048, 32, 4096, 8), "cluster"),
     ((2048, 2048, 32, 4096, 8), "fused_tc"), ((262144, 2048, 32, 4096, 8), "fused_tc"),
     ((2048, 2048, 16, 4096, 4), "cluster"), ((4096, 2048, 16, 4096, 4), "fused_tc"),
     ((262144, 2048, 128, 4096, 16), "cluster"),     # the fused kernel's plan does not hold r = 128, k > 8
@@ -89,7 +89,7 @@ def test_unfused_scratch_size_and_checks(lib):
     ((16, 64, 32, 64, 0), None), ((16, 64, 24, 64, 4), None),
 ])
 def test_auto_variant_follows_the_measured_crossovers(shape, expected):
-    """AUTO's choice (host-only, no GPU): small-N below 256 tokens, the cluster kernel up to the
+    """AUTO's choice (host-only, no GPU): small-N up to 148 tokens, the cluster kernel up to the
     fused kernel's one-tile floor, the fused kernel beyond, and the cluster kernel for shapes the
     fused kernel's shared-memory plan cannot hold."""
     import mixture_experts_rank_b200 as m

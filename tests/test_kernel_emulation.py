@@ -215,6 +215,23 @@ def test_threshold_topk_kernel_ties_and_orders(emu, k):
     check_threshold_topk(emu, np.concatenate(rows), k)
 
 
+@pytest.mark.parametrize("h,r,M,k", [(2048, 32, 4096, 8), (136, 48, 64, 8), (72, 16, 200, 1)])
+def test_small_n_single_token_zeroes_its_counts(emu, h, r, M, k):
+    """A one-token call runs on one CTA, which zeroes the counts itself (no memset is issued):
+    counts that start as garbage end as the bincount of the token's k selections."""
+    e = emu
+    X, R1, R2 = syn.router_inputs(1, h, r, M, seed=h + r)
+    out = [e.empty(k * 4), e.empty(k * 4), e.empty(M * 4), e.empty(k * 4)]
+    status = ctypes.c_uint(0)
+    assert e.lib.emu_route_small_self_zero(e.put(X), e.put(R1), e.put(R2), h, r, M, k, *out,
+                                           ctypes.addressof(status)) == 0
+    idx, gate = e.get(out[0], (1, k), np.int32), e.get(out[1], (1, k), np.float32)
+    cnt, logits = e.get(out[2], (M,), np.int32), e.get(out[3], (1, k), np.float32)
+    e.free_all()
+    assert status.value == 0
+    parity.compare(X, R1, R2, 1, h, r, M, k, idx, gate, cnt, logits)
+
+
 @pytest.mark.parametrize("N,h,r,M", [(23, 128, 32, 192), (6, 512, 16, 1000), (1, 64, 128, 64)])
 def test_train_stats_kernel_matches_oracle(emu, N, h, r, M):
     e = emu
