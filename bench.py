@@ -69,8 +69,8 @@ BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X,
 # was captured: once route_tc.cu differs from that source the figure is stale and traffic is
 # reported null.  Workloads without a capture report traffic null.
 NCU_TRAFFIC = {    # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
-    "prefill_r32": ((269207808 + 5669120) / 65536,
-                    "d652dfd40269b1b1101246c61c4142d9c062bd1987b4b5274a9918f2cfe06805"),
+    "prefill_r32": ((269296128 + 5271808) / 65536,
+                    "81620ba28949d4d2eb3688cbdb92f79cc859d2b0846c1756f81a5d65fcc3dd2d"),
 }
 L2_BYTES = 126 * 1024 * 1024
 
