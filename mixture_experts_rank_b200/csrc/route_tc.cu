@@ -1186,8 +1186,9 @@ uint32_t layout(Params& p, int xs, int r2n, int nz) {
 }
 
 // Shared-memory plan; returns the total bytes (0 when nothing fits).  Preference order:
-// R2 resident (no streaming at all), then two z buffers (one R2 sweep per tile) with at
-// least 3 X stages, then one z buffer (two sweeps per tile); more X stages first.
+// R2 resident (no streaming at all); then two z buffers (one R2 sweep per tile) with at least
+// 3 R2 stages; then one z buffer (two sweeps per tile) with at least 3 R2 stages; then 2 R2
+// stages.  Within each, more X stages first, then more R2 stages.
 template <int R, int KCAP>
 uint32_t plan(Params& p) {
   struct Try {
@@ -1206,7 +1207,7 @@ uint32_t plan(Params& p) {
         }
       }
   }
-  const Try tries[] = {{2, 3, 3}, {1, 2, 2}, {2, 2, 2}};
+  const Try tries[] = {{2, 2, 3}, {1, 2, 3}, {1, 2, 2}, {2, 2, 2}};
   for (const Try& tr : tries) {
     for (int xs = 4; xs >= tr.xs_min; --xs) {
       for (int r2n = 8; r2n >= tr.r2_min; --r2n) {
