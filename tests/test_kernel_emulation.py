@@ -152,7 +152,8 @@ def route_with(e, entry, X, R1, R2, N, h, r, M, k, exact=False):
 
 @pytest.mark.parametrize("entry", ["small_n", "unfused"])
 @pytest.mark.parametrize("N,h,r,M,k", [(7, 2048, 32, 4096, 8), (33, 136, 48, 64, 8), (20, 72, 16, 200, 1),
-                                       (9, 256, 64, 16, 16)])
+                                       (9, 256, 64, 16, 16), (11, 128, 32, 304, 3), (13, 96, 16, 128, 5),
+                                       (6, 64, 32, 512, 12)])
 def test_routing_kernels_match_oracle(emu, entry, N, h, r, M, k):
     X, R1, R2 = syn.router_inputs(N, h, r, M, seed=N)
     route_with(emu, entry, X, R1, R2, N, h, r, M, k)
