@@ -93,11 +93,14 @@ more_status more_route(const void* X, const void* R1, const void* R2, int64_t N,
 /*
  * The kernel AUTO runs for this shape (a more_variant value), or MORE_VARIANT_AUTO if the shape
  * fails the argument requirements.  The choice follows per-call times measured on a B200:
- *   - N <= 148: MORE_VARIANT_SMALL_N (one CTA per token, a single wave on a B200's 148 SMs);
+ *   - N <= 148: MORE_VARIANT_SMALL_N (one CTA per token, a single wave on a B200's 148 SMs),
+ *     except where the weights one CTA would read, r * (h + M) values, reach 196608 with
+ *     N <= 64 or 393216 at any N <= 148: there MORE_VARIANT_CLUSTER, which spreads them over
+ *     eight SMs (at h = 2048, M = 4096: r = 32 with N <= 64, and r >= 64);
  *   - otherwise MORE_VARIANT_CLUSTER while its time, which grows with N, stays below the fused
  *     kernel's floor (the latency of one 128-token tile: Z over h, then two sweeps over the
  *     M / 128 expert tiles); MORE_VARIANT_FUSED_TC beyond.  At h = 2048, M = 4096 the switch
- *     falls near N = 1,300 (r = 32) and N = 2,000 (r = 16);
+ *     falls near N = 1,440 (r = 32) and N = 1,920 (r = 16);
  *   - MORE_VARIANT_CLUSTER at any N > 148 for shapes the fused kernel's shared-memory plan
  *     cannot hold: r = 128 with k > 8 (any M), r = 128 with 4 < k <= 8 and M >= 11752,
  *     r = 128 with k <= 4 and M >= 28136, r = 64 with k > 8 and M >= 28136, every r not in

@@ -51,10 +51,15 @@ RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, in
 
 // AUTO's choice of kernel, from per-call times measured on a B200 (CUDA-graph replays of
 // back-to-back calls; h = 2048, M = 4096 with r = 16, 32 and 128):
-// - up to 148 tokens the small-N kernel (one CTA per token, one CTA per SM: a single wave on
-//   the 148 SMs of a B200) is fastest or level;
-// - beyond, it needs a second wave and the cluster kernel overtakes it.  Its time grows linearly,
-//   about 12 us + N * 2.3e-7 us * r * (h + M) (r = 32: 58 us at N = 1024, 104 us at 2048);
+// - up to 148 tokens the small-N kernel runs one CTA per token, one CTA per SM: a single wave
+//   on the 148 SMs of a B200.  Its time follows the weights one SM reads, r * (h + M) bf16
+//   values: 7.3 us at r = 16, 13.1 us at r = 32, 48 us at r = 128.  The cluster kernel spreads
+//   them over eight SMs and wins from r * (h + M) = 196608 (r = 32 at this shape: 12.6 against
+//   13.2 us at N = 1) while it holds at most 8 clusters (N <= 64), and from twice that at any
+//   N (r = 128: 36 against 49 us at N = 64);
+// - beyond 148 tokens the small-N kernel needs a second wave and the cluster kernel overtakes it.
+//   Its time grows linearly, about 9 us + N * (0.013 us + 1.53e-7 us * r * (h + M)) (r = 16:
+//   35 us at N = 1024, 121 us at 4096; r = 32: 56 us at 1024, 188 us at 4096);
 // - the fused kernel's time has a floor until every SM holds a tile: the chain of one
 //   128-token tile (Z over h, then two sweeps over the M / 128 expert tiles), about
 //   5 us + 0.0056 us * h + 0.0133 us * M * (0.7 + 0.3 r / 32) (r = 32: 74 us; r = 16: 58 us).
@@ -64,15 +69,21 @@ RouteArgs make_args(const void* X, const void* R1, const void* R2, int64_t N, in
 constexpr int64_t kClusterMinTokens = 149;
 
 double cluster_estimate_us(int64_t N, int h, int r, int M) {
-  return 12.0 + (double)N * 2.3e-7 * r * ((double)h + M);
+  return 9.0 + (double)N * (0.013 + 1.53e-7 * r * ((double)h + M));
 }
 
 double fused_floor_us(int h, int r, int M) {
   return 5.0 + 0.0056 * h + 0.0133 * M * (0.7 + 0.3 * r / 32.0);
 }
 
+constexpr double kClusterWeights = 196608.0;  // r * (h + M) from which the cluster kernel wins at N <= 64
+
 int auto_variant(const RouteArgs& a) {
-  if (a.N < kClusterMinTokens) return MORE_VARIANT_SMALL_N;
+  if (a.N < kClusterMinTokens) {
+    const double w = (double)a.r * ((double)a.h + a.M);
+    return (a.N <= 64 && w >= kClusterWeights) || w >= 2 * kClusterWeights ? MORE_VARIANT_CLUSTER
+                                                                            : MORE_VARIANT_SMALL_N;
+  }
   if (!fused_tc_fits(a)) return MORE_VARIANT_CLUSTER;
   return cluster_estimate_us(a.N, a.h, a.r, a.M) < fused_floor_us(a.h, a.r, a.M) ? MORE_VARIANT_CLUSTER
                                                                                   : MORE_VARIANT_FUSED_TC;
@@ -146,8 +157,10 @@ more_status more_route_variant(const void* X, const void* R1, const void* R2, in
   a.status = status_word();
   if (!a.status) return MORE_ERR_CUDA;
   if (N > 0 && variant == MORE_VARIANT_AUTO) variant = auto_variant(a);
-  // a single token routed by the small-N kernel runs on one CTA, which zeroes the counts itself
-  a.zero_counts = (N == 1 && variant == MORE_VARIANT_SMALL_N) ? 1 : 0;
+  // a single token on the small-N kernel (one CTA), or up to 8 on the cluster kernel (one
+  // cluster), is routed by a launch that zeroes the counts itself
+  a.zero_counts = ((N == 1 && variant == MORE_VARIANT_SMALL_N) || (N >= 1 && N <= 8 && variant == MORE_VARIANT_CLUSTER))
+                      ? 1 : 0;
   if (!a.zero_counts && cudaMemsetAsync(out_expert_count, 0, sizeof(int32_t) * (size_t)M, a.stream) != cudaSuccess)
     return MORE_ERR_CUDA;
   if (N == 0) return MORE_OK;

@@ -153,6 +153,8 @@ class Emulated:
         lib.emu_unfused_scratch_bytes.argtypes = [I64, I, I]
         lib.emu_route_unfused.restype = I
         lib.emu_route_unfused.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, P, P, P]
+        lib.emu_route_cluster_self_zero.restype = I
+        lib.emu_route_cluster_self_zero.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, P, P]
         lib.emu_route_small_self_zero.restype = I
         lib.emu_route_small_self_zero.argtypes = [P, P, P, I, I, I, I, P, P, P, P, P]
         lib.emu_threshold_topk.restype = I

@@ -88,6 +88,21 @@ extern "C" int emu_route_small(const void* X, const void* R1, const void* R2, in
   return (int)more::launch_small_n(route_args(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits, status));
 }
 
+// Up to 8 tokens on the cluster kernel with the counts zeroed by its single cluster (as
+// more_route does for N <= 8): the counts start as garbage here.
+extern "C" int emu_route_cluster_self_zero(const void* X, const void* R1, const void* R2, int64_t N, int h, int r,
+                                           int M, int k, int32_t* idx, float* gate, int32_t* cnt, float* logits,
+                                           unsigned* status) {
+  more::RouteArgs a = route_args(X, R1, R2, N, h, r, M, k, idx, gate, nullptr, logits, status);
+  a.out_count = cnt;
+  for (int e = 0; e < M; ++e) cnt[e] = 7;
+  a.zero_counts = 1;
+  emu::cluster_size = 8;
+  const int rc = (int)more::launch_cluster(a);
+  emu::cluster_size = 1;
+  return rc;
+}
+
 // One token on the small-N kernel with the counts zeroed by the kernel itself (as more_route does
 // for N == 1): the counts start as garbage here.
 extern "C" int emu_route_small_self_zero(const void* X, const void* R1, const void* R2, int h, int r, int M, int k,

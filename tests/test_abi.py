@@ -78,10 +78,16 @@ def test_unfused_scratch_size_and_checks(lib):
 
 
 @pytest.mark.parametrize("shape,expected", [
-    ((1, 2048, 32, 4096, 8), "small_n"), ((148, 2048, 32, 4096, 8), "small_n"),
+    ((1, 2048, 16, 4096, 4), "small_n"), ((148, 2048, 16, 4096, 4), "small_n"),
+    ((1, 2048, 32, 4096, 8), "cluster"), ((64, 2048, 32, 4096, 8), "cluster"),   # r (h + M) = 196608
+    ((65, 2048, 32, 4096, 8), "small_n"), ((148, 2048, 32, 4096, 8), "small_n"),
+    ((1, 2048, 32, 4088, 8), "small_n"),            # just below 196608
+    ((148, 2048, 128, 4096, 16), "cluster"),        # r (h + M) >= 393216 at any N
     ((149, 2048, 32, 4096, 8), "cluster"), ((1024, 2048, 32, 4096, 8), "cluster"),
     ((2048, 2048, 32, 4096, 8), "fused_tc"), ((262144, 2048, 32, 4096, 8), "fused_tc"),
-    ((2048, 2048, 16, 4096, 4), "cluster"), ((4096, 2048, 16, 4096, 4), "fused_tc"),
+    ((1900, 2048, 16, 4096, 4), "cluster"), ((1940, 2048, 16, 4096, 4), "fused_tc"),
+    ((1430, 2048, 32, 4096, 8), "cluster"), ((1450, 2048, 32, 4096, 8), "fused_tc"),
+    ((4096, 2048, 16, 4096, 4), "fused_tc"),
     ((262144, 2048, 128, 4096, 16), "cluster"),     # the fused kernel's plan does not hold r = 128, k > 8
     ((262144, 2048, 128, 8192, 8), "fused_tc"), ((262144, 2048, 128, 11752, 8), "cluster"),
     ((262144, 2048, 48, 4096, 8), "cluster"),       # r outside the fused kernel's ranks
@@ -89,7 +95,8 @@ def test_unfused_scratch_size_and_checks(lib):
     ((16, 64, 32, 64, 0), None), ((16, 64, 24, 64, 4), None),
 ])
 def test_auto_variant_follows_the_measured_crossovers(shape, expected):
-    """AUTO's choice (host-only, no GPU): small-N up to 148 tokens, the cluster kernel up to the
+    """AUTO's choice (host-only, no GPU): small-N up to 148 tokens unless the weights one CTA
+    would read are large (then the cluster kernel), the cluster kernel up to the
     fused kernel's one-tile floor, the fused kernel beyond, and the cluster kernel for shapes the
     fused kernel's shared-memory plan cannot hold."""
     import mixture_experts_rank_b200 as m

@@ -29,7 +29,7 @@ def test_expert_sweep_sampled():
 
 
 def test_many_experts_sampled():
-    """M = 65,536: 8,192 experts per CTA, 32 passes of the running top-k."""
+    """M = 65,536: 8,192 experts per CTA, 16 passes of 512 with a running top-k."""
     P.test_many_experts_sampled(V)
 
 

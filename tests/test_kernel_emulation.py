@@ -96,6 +96,10 @@ def cluster(e, X, R1, R2, N, h, r, M, k, exact=False):
     (9, 64, 16, 8, 8),        # M = 8: seven of the eight CTAs hold no expert; k = M
     (20, 200, 48, 200, 1),    # r = 48, ragged M, k = 1
     (5, 64, 128, 16, 16),     # r = 128, k = M = 16
+    (1, 2048, 32, 4096, 8),   # one token
+    (3, 4096, 64, 1024, 4),   # 512 hidden rows per CTA: two staged chunks
+    (7, 136, 16, 64, 2),      # 24-row slices: the last CTAs hold no hidden row
+    (2, 64, 32, 8192, 8),     # 1024 experts per CTA: two 512-expert passes
 ])
 def test_cluster_routing_matches_oracle(emu, N, h, r, M, k):
     X, R1, R2 = syn.router_inputs(N, h, r, M, seed=N)
@@ -231,6 +235,23 @@ def test_small_n_single_token_zeroes_its_counts(emu, h, r, M, k):
     e.free_all()
     assert status.value == 0
     parity.compare(X, R1, R2, 1, h, r, M, k, idx, gate, cnt, logits)
+
+
+@pytest.mark.parametrize("N,h,r,M,k", [(1, 2048, 32, 4096, 8), (8, 136, 48, 64, 8), (5, 72, 16, 200, 1)])
+def test_cluster_single_cluster_zeroes_its_counts(emu, N, h, r, M, k):
+    """Up to 8 tokens run on one cluster, whose CTAs zero the counts themselves (no memset is
+    issued): counts that start as garbage end as the bincount of the selections."""
+    e = emu
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=N + h)
+    out = [e.empty(N * k * 4), e.empty(N * k * 4), e.empty(M * 4), e.empty(N * k * 4)]
+    status = ctypes.c_uint(0)
+    assert e.lib.emu_route_cluster_self_zero(e.put(X), e.put(R1), e.put(R2), N, h, r, M, k, *out,
+                                             ctypes.addressof(status)) == 0
+    idx, gate = e.get(out[0], (N, k), np.int32), e.get(out[1], (N, k), np.float32)
+    cnt, logits = e.get(out[2], (M,), np.int32), e.get(out[3], (N, k), np.float32)
+    e.free_all()
+    assert status.value == 0
+    parity.compare(X, R1, R2, N, h, r, M, k, idx, gate, cnt, logits)
 
 
 @pytest.mark.parametrize("N,h,r,M", [(23, 128, 32, 192), (6, 512, 16, 1000), (1, 64, 128, 64)])
