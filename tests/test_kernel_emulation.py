@@ -117,12 +117,14 @@ def test_cluster_routing_tie_heavy_exact(emu):
 @pytest.mark.parametrize("name,old,new", [
     ("backward.cu", "(pbt[e] - tg[t])", "(pbt[e] + tg[t])"),                   # the sign of g in ybar
     ("route_cluster.cu", "for (int p = 0; p < kCluster; ++p) z +=", "for (int p = 1; p < kCluster; ++p) z +="),
+    ("route_cluster.cu", "acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);", "acc[t] += 0.f;"),  # half-warp rows lost
     ("route_scores_topk.cu", "lane < k && lv >= xv", "lane < k && lv > xv"),  # equal values: later expert first
     ("route_scores_topk.cu", "first ? lmax >= floor0", "first ? lmax > floor0"),  # drops values at the floor
 ])
 def test_planted_kernel_mistake_is_caught(tmp_path, name, old, new):
-    """A mistake planted in a kernel source fails these checks (a dropped partial z, a sign, the
-    order of equal scores, a first-chunk filter that drops values at its floor)."""
+    """A mistake planted in a kernel source fails these checks (a dropped partial z, the lost rows
+    of a half warp, a sign, the order of equal scores, a first-chunk filter that drops values at
+    its floor)."""
     reason = emulation.available()
     if reason:
         pytest.skip(reason)
@@ -134,8 +136,8 @@ def test_planted_kernel_mistake_is_caught(tmp_path, name, old, new):
             ties = np.random.default_rng(0).integers(-3, 4, size=(40, 520)).astype(np.float32)
             check_threshold_topk(e, ties, 4)
         else:
-            X, R1, R2 = syn.router_inputs(13, 256, 32, 512, seed=13)
-            cluster(e, X, R1, R2, 13, 256, 32, 512, 8)
+            X, R1, R2 = syn.router_inputs(13, 256, 48, 512, seed=13)  # r = 48: a full and a half column block
+            cluster(e, X, R1, R2, 13, 256, 48, 512, 8)
     e.free_all()
 
 
