@@ -102,11 +102,10 @@ more_status more_route(const void* X, const void* R1, const void* R2, int64_t N,
  *     M / 128 expert tiles); MORE_VARIANT_FUSED_TC beyond.  At h = 2048, M = 4096 the switch
  *     falls near N = 1,440 (r = 32) and N = 1,920 (r = 16);
  *   - MORE_VARIANT_CLUSTER at any N > 148 for shapes the fused kernel's shared-memory plan
- *     cannot hold: r = 128 with k > 8 (any M), r = 128 with 4 < k <= 8 and M >= 11752,
- *     r = 128 with k <= 4 and M >= 28136, r = 64 with k > 8 and M >= 28136, every r not in
- *     {16, 32, 64, 128}, and M > 65536.  Those shapes run on CUDA cores, far slower per token
- *     at prefill sizes than the fused kernel (r = 128, k = 16, M = 4096: about 0.26 us per
- *     token against 2.3 ns for the fused kernel at r = 32).
+ *     cannot hold: r = 128 with k > 8 (any M), every r not in {16, 32, 64, 128}, and
+ *     M > 65536.  Those shapes run on CUDA cores, far slower per token at prefill sizes than
+ *     the fused kernel (r = 128, k = 16, M = 4096: about 0.26 us per token against 2.1 ns for
+ *     the fused kernel at r = 32).
  * Host-only; makes no CUDA call.
  */
 int more_route_auto_variant(int64_t N, int h, int r, int M, int k);

@@ -16,30 +16,31 @@
 //           double-buffered TMEM accumulator (the next tiles stream while the
 //           current ones are routed, so HBM never waits on the top-k).
 //   warp 2  MMA issuer of pass A: D[tok, exp] = z_hi R2 (K = r), 128 experts a job.
-//   warp 3  MMA issuer of pass B: D^T[exp, tok] = R2^T [z_hi | z_lo]^T (K = 2r, exact
-//           to ~16 bits of z), 128 experts a job.
+//   warp 3  MMA issuer of pass B: D[tok, exp] = [z_hi | z_lo] [R2 ; R2] (K = 2r, exact to
+//           ~16 bits of z), 128 experts a job.
 //   warps 4-11   group A (two warps per TMEM lane group): per tile
 //     epilogue  Z from TMEM -> (z_hi, z_lo) bf16 pair -> shared memory (K-major),
 //               plus |z_hi|, |z_lo| per token and (first tile) the largest column norm
 //               of R2.
 //     pass A    every 32-expert chunk of a token is reduced to the maximum of its z_hi
 //               logits, packed into a 32-bit key (order-preserving value bits above the
-//               chunk id); a branch-free sorted list keeps the best k + 6 keys per warp.
+//               chunk id); a branch-free sorted list keeps the best k keys per warp.
 //     select    the two lists of a token are merged.  z_hi logits differ from the exact
 //               ones by at most eps (|z_lo| times the largest R2 column norm, plus fp32
-//               rounding), so the exact k-th logit is at least tlow - eps (tlow: the
-//               k-th chunk maximum) and only chunks whose maximum reaches tlow - 2 eps
-//               can hold a top-k expert.  (token, chunk) pairs are bucketed by chunk
-//               with a counting sort into one of two pair buffers, handed to group B.
+//               rounding), and the k chunks with the largest z_hi maxima (>= tlow) hold k
+//               experts whose exact logit is >= tlow - eps, so the exact k-th logit is at
+//               least the cut tlow - eps.  The cut of every token is handed to group B.
 //   warps 12-19  group B (two warps per TMEM lane group): per tile
-//     pass B    the two warps of a lane group split the pairs of their chunk, read each
-//               pair's token column and ballot the experts whose exact logit reaches
-//               tlow - eps (the candidates).
+//     pass B    each warp reads its 64 columns of every exact tile, reduces each 8-expert
+//               octet to its maximum, and appends the experts whose exact logit reaches the
+//               token's cut (the candidates, about k + 1 per token) to the token's list in
+//               shared memory; octets without such an expert in any lane of the warp are
+//               skipped by a vote.
 //     finalize  two threads per token rank its few candidates in routing order (larger
 //               logit, then lower expert) into a shared-memory staging of the outputs,
-//               which the tile writes with coalesced stores; softmax, counts.  A list too
-//               short to certify the cut, or more candidates than the slots hold, sends
-//               the token to an exact recomputation on CUDA cores shared by the group.
+//               which the tile writes with coalesced stores; softmax, counts.  More
+//               candidates than the lists hold sends the token to an exact recomputation
+//               on CUDA cores shared by the group.
 // The logit MMAs run in sweeps over the expert tiles: each sweep streams R2 once and every
 // R2 tile feeds pass B of tile t and pass A of tile t + 1 (with two z buffers; otherwise a
 // sweep carries one pass), so group B works on tile t while group A works on tile t + 1.
@@ -51,6 +52,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cfloat>
 
 #include "more_internal.cuh"
 #include "mbar_wait.cuh"
@@ -71,13 +73,12 @@ constexpr int kRoleWarps = 4;
 constexpr int kWarpsA = 8;                       // group A: two warps per TMEM lane group
 constexpr int kWarpsB = MORE_GROUP_B_WARPS;      // group B: kWarpsB / 4 warps per TMEM lane group
 constexpr int kThreadsA = kWarpsA * 32, kThreadsB = kWarpsB * 32;
-constexpr int kPerTokB = kWarpsB / 4;            // group B threads per token in the finalize
 constexpr int kWarpA0 = kRoleWarps, kWarpB0 = kRoleWarps + kWarpsA;
 constexpr int kThreads = (kRoleWarps + kWarpsA + kWarpsB) * 32;
 constexpr int kNamedBarA = 1, kNamedBarB = 2;    // bar.sync ids of the groups
 static_assert(kWarpsB % 4 == 0, "group B covers the four TMEM lane groups evenly");
 static_assert((kWarpsB & (kWarpsB - 1)) == 0, "fallback teams divide group B evenly");
-constexpr int kPairBatch = 4;   // TMEM column loads in flight per warp in pass B
+static_assert(kWarpsB == 8, "pass B splits each 128-expert tile into two 64-column halves per lane group");
 constexpr int kFbBatch = 8;     // fallback tokens ranked per round of the cooperative fallback
 static_assert(kFbBatch <= kWarpsB, "one merging warp per fallback token of a batch");
 constexpr uint32_t kTmemCols = 512;
@@ -90,7 +91,6 @@ struct Params {
   int num_tiles;     // token tiles
   int kb_count;      // hidden blocks of kBK
   int p_count;       // expert tiles of kBE
-  int nchunks;       // 32-expert chunks
   uint32_t low_mask; // chunk-id bits of a key
   int x_stages;
   int r2_stages;
@@ -98,26 +98,30 @@ struct Params {
   int interleave;    // two z buffers: a sweep carries pass B of one tile and pass A of the next
   uint32_t off_x, off_r1, off_r2, off_zs;
   // group A only
-  uint32_t off_lists, off_ccount, off_scan, off_znorm, off_cnorm;
-  // handed from group A to group B, two buffers each
-  uint32_t off_pairs, off_cbase, off_flag, off_nq;
+  uint32_t off_lists, off_znorm, off_cnorm;
+  // handed from group A to group B, two buffers each: the cut and flags of every token
+  uint32_t off_cut, off_flag;
   // group B only
-  uint32_t off_cand, off_pc, off_pool, off_poolcnt, off_fb, off_part;
+  uint32_t off_slots, off_ids, off_hcnt, off_stage, off_fb, off_part;
   int fb_groups;  // warps per fallback token: min(kWarpsB, 256-expert blocks rounded up to a power of two)
   uint32_t off_bar;
 };
 
 template <int R, int KCAP>
 struct Cfg {
-  static constexpr int KL = KCAP + 6;                  // chunk keys kept per token and warp
-  static constexpr int KLP = (KL + 15) & ~15;          // row stride of the candidate slots and counts
-  // per-token slots for candidates beyond the first of a chunk: at k <= 4 the few chunks of a
-  // small expert pool hold several candidates each, so eight (an overflow sends the token to the
-  // exact fallback)
-  static constexpr int POOL = KCAP <= 4 ? 8 : 4;
+  static constexpr int KA = KCAP;                      // chunk keys kept per token and warp in pass A
+  // octet slots of pass B: every 8-expert octet that holds an expert at or above the token's cut
+  // is stored whole (its eight exact logits and its index), up to OCT per token; a token with
+  // more goes to the exact fallback
+  static constexpr int OCT = R >= 128 ? KCAP + 4 : KCAP + 6;
+  // In the finalize the octet slots take, in order: the output staging, the fallback's partial
+  // lists, and (in odd slot rows from XS0 on, which only the second thread of a token reads)
+  // the list that this thread hands to the first.
+  static constexpr uint32_t STAGE_BYTES = (3 * kBT * KCAP * 4 + 15) / 16 * 16;
+  static constexpr uint32_t PART_BYTES = kFbBatch * kWarpsB * KCAP * 8;
+  static constexpr int XS0 = (int)((STAGE_BYTES + PART_BYTES + kBT * 32 - 1) / (kBT * 32)) | 1;
+  static_assert(XS0 + 2 * ((KCAP - 1) / 4) < OCT, "the exchanged list fits the odd slot rows");
   static constexpr int RK = 2 * R;                     // z_hi | z_lo columns of the z buffer
-  // one pair buffer: the (token, chunk) pairs of a tile, later its output staging (3 x 128 x k words)
-  static constexpr uint32_t PAIR_BYTES = kBT * KL * 8 > 3 * kBT * KCAP * 4 ? kBT * KL * 8 : 3 * kBT * KCAP * 4;
   static constexpr int BK = R >= 128 ? 32 : 64;        // hidden elements per X stage
   static constexpr uint32_t X_STAGE = kBT * BK * 2;    // 16 KB (8 KB at BK = 32)
   static constexpr uint32_t X_LAYOUT = BK == 64 ? kSwizzle128B : kSwizzle64B;
@@ -134,12 +138,14 @@ struct Cfg {
   static constexpr uint32_t ZS_SBO = (RK / 8) * 128;   // byte stride of 8-token groups
   static constexpr int ZCOLS = R < 32 ? 32 : R;        // TMEM columns per Z accumulator
   static constexpr int NBUF = (512 - 2 * ZCOLS) / 128 < 3 ? (512 - 2 * ZCOLS) / 128 : 3;
-  static constexpr int NA = 1;                         // TMEM buffers of pass A jobs
+#ifndef MORE_PASS_A_BUFS
+#define MORE_PASS_A_BUFS 1
+#endif
+  static constexpr int NA = MORE_PASS_A_BUFS < NBUF ? MORE_PASS_A_BUFS : 1;  // TMEM buffers of pass A jobs
   static constexpr int NB = NBUF - NA;                 // TMEM buffers of pass B jobs (longer MMAs)
   static constexpr int ZCOL0 = NBUF * 128;             // first TMEM column of the Z accumulators
   static constexpr uint32_t IDESC_Z = idesc_bf16_f32(128, R, 0, 1);    // A = X (K-major), B = R1 (MN-major)
-  static constexpr uint32_t IDESC_PA = idesc_bf16_f32(128, 128, 0, 1); // A = z pair, B = R2 tile
-  static constexpr uint32_t IDESC_PB = idesc_bf16_f32(128, 128, 1, 0); // A = R2 tile^T, B = z pair^T
+  static constexpr uint32_t IDESC_P = idesc_bf16_f32(128, 128, 0, 1);  // A = z pair, B = R2 tile
   static_assert(NB >= 1, "TMEM holds at least one buffer per pass");
 };
 
@@ -441,10 +447,7 @@ __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t
         for (int kk = 0; kk < KSTEPS; ++kk) {
           const uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
           const uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
-          if (PASS_B)
-            mma_bf16(dt, rd, zd, C::IDESC_PB, kk != 0);
-          else
-            mma_bf16(dt, zd, rd, C::IDESC_PA, kk != 0);
+          mma_bf16(dt, zd, rd, C::IDESC_P, kk != 0);
         }
         mma_commit(&full[d.i]);
         d.next(NBUF);
@@ -472,7 +475,7 @@ done:
 template <int R, int KCAP>
 __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  constexpr int KL = C::KL;
+  constexpr int KL = C::KA;
   const RouteArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int aw = warp - kWarpA0;        // 0..7
@@ -484,9 +487,7 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
   const uint32_t low = p.low_mask;
   uint8_t* zs0 = smem + p.off_zs;
   const uint8_t* r2s = smem + p.off_r2;
-  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);  // merge exchange, then stage
-  int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
-  int* scan = reinterpret_cast<int*>(smem + p.off_scan);
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + p.off_lists);  // merge exchange
   float* znorm = reinterpret_cast<float*>(smem + p.off_znorm);  // [hi h0 | hi h1 | lo h0 | lo h1][token]
   float* cnorm = reinterpret_cast<float*>(smem + p.off_cnorm);  // [8] per warp, [8] = result
   uint32_t gph = 0;
@@ -608,14 +609,12 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       }
     }
 
-    // ---------------- select: merge the lists, certified window, needed pairs --------------
-    const int pb = j & 1, pu = j >> 1;  // pair buffer and its use count
-    // the pair buffer's previous tile (j - 2) is finalized by group B
+    // ---------------- select: merge the lists, the candidate cut -------------------------
+    const int pb = j & 1, pu = j >> 1;  // hand-off buffer and its use count
+    // the hand-off buffer's previous tile (j - 2) is finalized by group B
     if (pu > 0 && !bounded_wait(&b.pairs_empty[pb], (pu - 1) & 1, b.abort_flag, a.status)) return;
-    uint2* pairs = reinterpret_cast<uint2*>(smem + p.off_pairs + pb * C::PAIR_BYTES);
-    int* cbase = reinterpret_cast<int*>(smem + p.off_cbase) + pb * (p.nchunks + 1);
+    float* cut = reinterpret_cast<float*>(smem + p.off_cut) + pb * kBT;
     uint8_t* flag = smem + p.off_flag + pb * kBT;
-    uint8_t* nq = smem + p.off_nq + pb * kBT;
     if (hh == 1) {
 #pragma unroll
       for (int i = 0; i < KL; ++i) lists[i * kBT + t] = kl[i];
@@ -637,13 +636,10 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
       cnorm[kWarpsA] = sqrtf(m) * (1.f + 0x1p-20f);  // max column norm of R2, rounded up
     }
     group_bar(kNamedBarA, kThreadsA);  // the merge has read the exchanged lists; cnorm is final
-    uint32_t* stage = lists;  // (chunk, rank) of each needed pair of token t
-    float ccut = -INFINITY;   // candidates: exact logit >= ccut
-    int needed = 0;
     if (hh == 0) {
       const bool active = n0 + t < a.N;
-      // Certified window: values from z_hi differ from the z_hi + z_lo values by at most
-      // eps = |z_lo| cmax (Cauchy-Schwarz) plus a bound on fp32 accumulation differences.
+      // z_hi logits differ from the z_hi + z_lo values by at most eps = |z_lo| cmax
+      // (Cauchy-Schwarz) plus a bound on fp32 accumulation differences.
       const float cmax = cnorm[kWarpsA];
       const float zh = sqrtf(znorm[t] + znorm[kBT + t]);
       const float zl = sqrtf(znorm[2 * kBT + t] + znorm[3 * kBT + t]);
@@ -652,71 +648,16 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
 #pragma unroll
       for (int i = 0; i < KL; ++i)
         if (i == a.k - 1) kth = kl[i];
-      int f = active ? 0 : 2;
-      // The k chunks with the largest z_hi maxima (>= tlow) hold k elements whose exact logit
-      // is >= tlow - eps, so the exact k-th logit is >= tlow - eps (the candidate cut), and an
-      // element reaching it has a z_hi logit >= tlow - 2 eps (the chunk cut).
-      uint32_t cut_key = 0u;  // chunks whose key range reaches cut_key are needed
-      if ((kth & ~low) >= kRealKey) {
-        const float tlow = ord_inv(kth & ~low);  // <= the k-th largest z_hi chunk maximum
-        ccut = __fsub_rd(tlow, eps);
-        cut_key = ord_key(__fsub_rd(tlow, __fmul_ru(2.f, eps)));
-        if ((kl[KL - 1] & ~low) >= kRealKey && (kl[KL - 1] | low) >= cut_key) f |= 1;  // list too short
-      }
-      if (f == 0) {
-#pragma unroll
-        for (int i = 0; i < KL; ++i) {
-          if ((kl[i] & ~low) >= kRealKey && (kl[i] | low) >= cut_key) {
-            const uint32_t cid = kl[i] & low;
-            const int rank = atomicAdd(&ccount[cid], 1);
-            stage[i * kBT + t] = cid | ((uint32_t)rank << 16);  // until the bucket bases are known
-            needed = i + 1;
-          }
-        }
-      }
-      flag[t] = (uint8_t)f;
-      nq[t] = (uint8_t)needed;
+      // The k chunks with the largest z_hi maxima (>= tlow) hold k experts whose exact logit is
+      // >= tlow - eps, so the exact k-th logit is >= tlow - eps: every top-k expert reaches the
+      // cut.  With fewer than k real chunks every in-range expert is a candidate (the
+      // out-of-range ones are at -infinity, below the lowest finite cut).
+      float ccut = -FLT_MAX;
+      if ((kth & ~low) >= kRealKey) ccut = __fsub_rd(ord_inv(kth & ~low), eps);
+      cut[t] = active ? ccut : __int_as_float(0x7fffffff);  // NaN: no expert reaches it
+      flag[t] = (uint8_t)(active ? 0 : 2);
     }
-    group_bar(kNamedBarA, kThreadsA);
-    // exclusive prefix of the per-chunk pair counts (chunks 0 .. nchunks; the last is empty),
-    // eight chunks per thread
-    {
-      int vals[8], run = 0;
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int i = gt * 8 + jj;
-        vals[jj] = (i < p.nchunks) ? ccount[i] : 0;
-        run += vals[jj];
-      }
-      int incl = run;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
-      }
-      if (lane == 31) scan[aw] = incl;
-      group_bar(kNamedBarA, kThreadsA);
-      int before = incl - run;
-      for (int w = 0; w < aw; ++w) before += scan[w];
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int i = gt * 8 + jj;
-        if (i <= p.nchunks) cbase[i] = before;
-        if (i < p.nchunks) ccount[i] = 0;
-        before += vals[jj];
-      }
-      // the end of the last bucket (index nchunks lies past the 8 x 256 slots when nchunks == 2048)
-      if (gt == kThreadsA - 1) cbase[p.nchunks] = before;
-    }
-    group_bar(kNamedBarA, kThreadsA);
-    if (hh == 0) {
-      for (int i = 0; i < needed; ++i) {
-        const uint32_t st = stage[i * kBT + t];
-        // {token | needed-chunk index << 8, candidate cut}
-        pairs[cbase[st & 0xffffu] + (st >> 16)] = make_uint2((uint32_t)t | ((uint32_t)i << 8), __float_as_uint(ccut));
-      }
-    }
-    group_bar(kNamedBarA, kThreadsA);  // the pairs are written; the stage area may be reused
+    group_bar(kNamedBarA, kThreadsA);  // the cuts are written; the exchange area may be reused
     if (gt == 0) mbar_arrive(&b.pairs_full[pb]);
   }
 }
@@ -799,24 +740,40 @@ __device__ __forceinline__ void fallback_merge(const RouteArgs& a, const uint2* 
   warp_write_selection(a, n, lane, v, e);
 }
 
+// Branch-free insertion of the 64-bit key x into the descending list kl[0..L).
+template <int L>
+__device__ __forceinline__ void key_insert64(uint64_t* kl, uint64_t x) {
+#pragma unroll
+  for (int i = L - 1; i > 0; --i) kl[i] = max(kl[i], min(kl[i - 1], x));
+  kl[0] = max(kl[0], x);
+}
+
+// Routing-order key of (logit, expert): larger logit first, then lower expert; 0 is below
+// every real key.  -0 and +0 are equal in routing order: both take the key of +0.
+__device__ __forceinline__ uint64_t route_key(uint32_t logit_bits, uint32_t expert) {
+  return ((uint64_t)ord_key(__uint_as_float(logit_bits) + 0.f) << 32) | (uint64_t)(~expert);
+}
+
 template <int R, int KCAP>
 __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
-  constexpr int KL = C::KL;
-  constexpr int NC = KL + C::POOL;
   const RouteArgs& a = p.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bw = warp - kWarpB0;        // 0 .. kWarpsB - 1
   const int sp = warp & 3;              // TMEM lane group: lanes 32 sp .. 32 sp + 31
-  const int hh = bw >> 2;               // which of the lane group's kPerTokB warps
+  const int hh = bw >> 2;               // which 64-column half of every tile
   const int gt = bw * 32 + lane;        // 0 .. kThreadsB - 1
-  const int t = sp * 32 + lane;         // token of this thread in the finalize
+  const int t = sp * 32 + lane;         // token of this thread
   const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
   uint8_t* zs0 = smem + p.off_zs;
-  uint2* cand = reinterpret_cast<uint2*>(smem + p.off_cand);
-  uint8_t* pc = smem + p.off_pc;
-  uint2* pool = reinterpret_cast<uint2*>(smem + p.off_pool);
-  int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
+  uint4* slots = reinterpret_cast<uint4*>(smem + p.off_slots);       // [slot][token][2]: eight logits
+  uint16_t* ids = reinterpret_cast<uint16_t*>(smem + p.off_ids);     // [slot][token]: octet index
+  int* hcnt = reinterpret_cast<int*>(smem + p.off_hcnt);             // [token]: octets stored
+  // the list thread 1 hands to thread 0: entry i in slot row XS0 + 2 (i / 4), word i % 4
+  uint64_t* xchg = reinterpret_cast<uint64_t*>(slots + 2 * (C::XS0 * kBT + t));
+  int32_t* sidx = reinterpret_cast<int32_t*>(smem + p.off_stage);    // [token][k]
+  float* sex = reinterpret_cast<float*>(sidx + kBT * KCAP);
+  float* slog = sex + kBT * KCAP;
   int* fbcount = reinterpret_cast<int*>(smem + p.off_fb);
   uint8_t* fblist = smem + p.off_fb + 4;
   uint8_t* fbmark = smem + p.off_fb + 4 + kBT;  // 1: the token's outputs come from the fallback
@@ -829,149 +786,116 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     const int64_t n0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kBT;
     const int pb = j & 1, pu = j >> 1;
     if (!bounded_wait(&b.pairs_full[pb], pu & 1, b.abort_flag, a.status)) return;
-    const uint2* pairs = reinterpret_cast<const uint2*>(smem + p.off_pairs + pb * C::PAIR_BYTES);
-    const int* cbase = reinterpret_cast<const int*>(smem + p.off_cbase) + pb * (p.nchunks + 1);
-    const uint8_t* flag = smem + p.off_flag + pb * kBT;
-    const uint8_t* nq = smem + p.off_nq + pb * kBT;
+    const float ccut = reinterpret_cast<const float*>(smem + p.off_cut)[pb * kBT + t];
+    const bool active = (smem[p.off_flag + pb * kBT + t] & 2) == 0;
 
-    // ---------------- pass B: candidates of the needed chunks (exact z_hi + z_lo logits) ----
-    // Lane group sp of the transposed tile is chunk 4 pt + sp; its kPerTokB warps split the
-    // chunk's pairs.
+    // ---------------- pass B: octets of the token that reach its cut (exact logits) ----------
+    // Warp hh of a lane group reads columns 64 hh .. 64 hh + 63 of every tile, reduces each
+    // octet to its maximum and stores the octets that reach its lane's cut.
     for (int pt = 0; pt < p.p_count; ++pt) {
-      const int c = pt * 4 + sp;
-      int lo = 0, hi = 0;
-      if (c < p.nchunks) {
-        const int c_lo = cbase[c], n = cbase[c + 1] - c_lo;
-        lo = c_lo + (n * hh) / kPerTokB;
-        hi = c_lo + (n * (hh + 1)) / kPerTokB;
-      }
       if (!bounded_wait(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
-      const int e = 32 * c + lane;
-      const bool e_ok = e < a.M;
-      const uint32_t col0 = tmem_base + lane_base + (C::NA + bd.i) * 128;
-      const uint32_t lt_mask = (1u << lane) - 1u;
-      for (int pi = lo; pi < hi; pi += kPairBatch) {
-        const int nb = hi - pi < kPairBatch ? hi - pi : kPairBatch;
-        uint2 ent[kPairBatch];
-        uint32_t val[kPairBatch];
+      const uint32_t col = tmem_base + lane_base + (C::NA + bd.i) * 128 + hh * 64;
 #pragma unroll
-        for (int q = 0; q < kPairBatch; ++q)
-          if (q < nb) ent[q] = pairs[pi + q];  // {token | slot << 8, candidate cut}
-#pragma unroll
-        for (int q = 0; q < kPairBatch; ++q)
-          if (q < nb) val[q] = tmem_ld_x1(col0 + (ent[q].x & 0xffu));
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld_x32(col + 32 * half, v);
         tmem_wait_ld();
-        reg_fence<kPairBatch>(val);
-        // per pair: ballot the experts at or above the cut; the first one takes the
-        // pair's slot, lane 0 records the count, any further ones go to the pool below
-        uint32_t bal[kPairBatch];
-        uint32_t extra = 0u;
-#pragma unroll
-        for (int q = 0; q < kPairBatch; ++q) {
-          const bool take = q < nb && e_ok && __uint_as_float(val[q]) >= __uint_as_float(ent[q].y);
-          bal[q] = __ballot_sync(0xffffffffu, take);
-          const uint32_t tq = ent[q].x & 0xffu, iq = ent[q].x >> 8;
-          const uint32_t before = bal[q] & lt_mask;
-          if (take && before == 0u) cand[iq * kBT + tq] = make_uint2(val[q], (uint32_t)e);
-          if (lane == 0 && q < nb) pc[tq * C::KLP + iq] = (uint8_t)__popc(bal[q]);
-          extra |= bal[q] & (bal[q] - 1u);  // set iff the pair has two or more candidates
+        reg_fence<32>(v);
+        if (half == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b.b_empty[bd.i]);
         }
-        if (extra) {  // rare: more candidates than the pair's slot
+        const int e0 = kBE * pt + 64 * hh + 32 * half;
+        if (e0 + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1): below every cut
 #pragma unroll
-          for (int q = 0; q < kPairBatch; ++q) {
-            if (((bal[q] >> lane) & 1u) && (bal[q] & lt_mask)) {
-              const int tok = ent[q].x & 0xff;
-              const int ps = atomicAdd(&poolcnt[tok], 1);
-              if (ps < C::POOL) pool[ps * kBT + tok] = make_uint2(val[q], (uint32_t)e);
+          for (int jj = 0; jj < 32; ++jj)
+            if (e0 + jj >= a.M) v[jj] = 0xff800000u;
+        }
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+          const uint32_t* w = v + 8 * o;
+          const float om = max3f(max3f(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2])),
+                                 max3f(__uint_as_float(w[3]), __uint_as_float(w[4]), __uint_as_float(w[5])),
+                                 fmaxf(__uint_as_float(w[6]), __uint_as_float(w[7])));
+          if (om >= ccut) {  // rare per lane: about k + 1 octets of a token in all
+            const int sl = atomicAdd(&hcnt[t], 1);
+            if (sl < C::OCT) {
+              uint4* dst = slots + 2 * (sl * kBT + t);
+              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              ids[sl * kBT + t] = (uint16_t)((e0 >> 3) + o);
             }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&b.b_empty[bd.i]);
       bd.next(C::NB);
     }
 
     // ---------------- finalize: order, softmax, store, count ---------------------------
-    // kPerTokB threads per token (the lane group's warps).  Every thread loads all of the
-    // token's candidates (the slots of its needed chunks, then its pool entries) into
-    // registers; thread hh ranks candidates hh, hh + kPerTokB, ... in routing order (larger
-    // logit, then lower expert) and the ones of rank < k go to the output staging at their rank,
-    // with exp(logit - max).  The staging reuses the tile's pair buffer, which pass B has
-    // finished reading.
+    // Two threads per token (the lane group's warps): thread hh keeps the best k of the
+    // candidates in the token's octets hh, hh + 2, ... as sorted 64-bit routing keys; thread 1
+    // hands its list to thread 0, which merges it and writes the token's outputs to the
+    // staging with the softmax gates.
     if (!group_enter(&b.gbar[1], gph, b.abort_flag, a.status)) return;
     // from here to the hand-off nothing waits on another role
-    int32_t* sidx = reinterpret_cast<int32_t*>(smem + p.off_pairs + pb * C::PAIR_BYTES);  // [token][k]
-    float* sex = reinterpret_cast<float*>(sidx + kBT * a.k);
-    float* slog = sex + kBT * a.k;
-    const int f = flag[t];
-    bool fb = false;
-    if ((f & 2) == 0) {
-      uint32_t o[NC], e[NC];
-      const int jn = nq[t], np = poolcnt[t];
-      uint32_t cnt[C::KLP / 4];
+    const int n = active ? hcnt[t] : 0;
+    const bool over = n > C::OCT;
+    uint64_t kl[KCAP];
 #pragma unroll
-      for (int w = 0; w < C::KLP / 16; ++w) {
-        const uint4 q4 = *reinterpret_cast<const uint4*>(pc + t * C::KLP + 16 * w);
-        cnt[4 * w] = q4.x;
-        cnt[4 * w + 1] = q4.y;
-        cnt[4 * w + 2] = q4.z;
-        cnt[4 * w + 3] = q4.w;
+    for (int i = 0; i < KCAP; ++i) kl[i] = 0ull;
+    if (!over) {
+      for (int sl = hh; sl < n; sl += 2) {
+        const uint4 q0 = slots[2 * (sl * kBT + t)], q1 = slots[2 * (sl * kBT + t) + 1];
+        const uint32_t eb = 8u * ids[sl * kBT + t];
+        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+          key_insert64<KCAP>(kl, __uint_as_float(w[jj]) >= ccut ? route_key(w[jj], eb + jj) : 0ull);
       }
-      // -0 and +0 are equal in routing order: both take the key of +0.  Empty slots take
-      // key 0, below every real value, so they never outrank a candidate.
-      int total = 0;
+    }
+    if (hh == 1) {
 #pragma unroll
-      for (int q = 0; q < NC; ++q) {
-        bool has;
-        uint2 cv = make_uint2(0u, 0u);
-        if (q < KL) {
-          const int nc = q < jn ? (int)((cnt[q >> 2] >> (8 * (q & 3))) & 0xffu) : 0;
-          total += nc;
-          has = nc > 0;
-          if (has) cv = cand[q * kBT + t];
-        } else {
-          has = q - KL < np;
-          if (has) cv = pool[(q - KL) * kBT + t];
+      for (int i = 0; i < KCAP; ++i) xchg[(i >> 2) * (2 * kBT * 4) + (i & 3)] = kl[i];
+    }
+    group_bar(kNamedBarB, kThreadsB);  // the lists are exchanged; every other octet slot is read
+    if (hh == 0) {
+      if (active) {
+        if (!over) {
+#pragma unroll
+          for (int i = 0; i < KCAP; ++i) key_insert64<KCAP>(kl, xchg[(i >> 2) * (2 * kBT * 4) + (i & 3)]);
         }
-        o[q] = has ? ord_key(__uint_as_float(cv.x) + 0.f) : 0u;
-        e[q] = cv.y;
-      }
-      fb = (f & 1) || np > C::POOL || total < a.k;
-      if (hh == 0) {
+        uint64_t kth = 0ull;
+#pragma unroll
+        for (int i = 0; i < KCAP; ++i)
+          if (i == a.k - 1) kth = kl[i];
+        const bool fb = over || kth == 0ull;  // too many octets, or fewer than k candidates
         fbmark[t] = fb ? 1 : 0;
-        if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
-      }
-      if (!fb) {
-        uint32_t top = 0u;
+        if (fb) {
+          fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
+        } else {
+          const float vtop = ord_inv((uint32_t)(kl[0] >> 32));
+          float ex[KCAP], sum = 0.f;
 #pragma unroll
-        for (int q = 0; q < NC; ++q) top = max(top, o[q]);
-        const float vtop = ord_inv(top);
+          for (int i = 0; i < KCAP; ++i) {
+            ex[i] = i < a.k ? expf(ord_inv((uint32_t)(kl[i] >> 32)) - vtop) : 0.f;
+            sum += ex[i];
+          }
+          const float inv = 1.f / sum;
 #pragma unroll
-        for (int q = 0; q < NC; ++q) {
-          if ((q % kPerTokB) != hh || o[q] == 0u) continue;  // this thread's share; empty slots
-          int rank = 0;
-#pragma unroll
-          for (int jj = 0; jj < NC; ++jj) rank += (o[jj] > o[q] || (o[jj] == o[q] && e[jj] < e[q])) ? 1 : 0;
-          if (rank < a.k) {
-            const float v = ord_inv(o[q]);
-            sidx[t * a.k + rank] = (int)e[q];
-            sex[t * a.k + rank] = expf(v - vtop);
-            slog[t * a.k + rank] = v;
-            if (e[q] < (uint32_t)a.M) atomicAdd(a.out_count + e[q], 1);
+          for (int i = 0; i < KCAP; ++i) {
+            if (i < a.k) {
+              const uint32_t e = ~(uint32_t)kl[i];
+              sidx[t * a.k + i] = (int)e;
+              sex[t * a.k + i] = ex[i] * inv;
+              slog[t * a.k + i] = ord_inv((uint32_t)(kl[i] >> 32));
+              if (e < (uint32_t)a.M) atomicAdd(a.out_count + e, 1);
+            }
           }
         }
       }
-    }
-    group_bar(kNamedBarB, kThreadsB);
-    // gates: each selected exp divided by its token's sum
-    if (hh == 0 && (f & 2) == 0 && !fb) {
-      float sum = 0.f;
-      for (int jj = 0; jj < a.k; ++jj) sum += sex[t * a.k + jj];
-      const float inv = 1.f / sum;
-      for (int jj = 0; jj < a.k; ++jj) sex[t * a.k + jj] *= inv;
+      hcnt[t] = 0;  // every thread of the token has read the count
     }
     group_bar(kNamedBarB, kThreadsB);
     // the tile's outputs are contiguous: copy the staging out with coalesced stores
@@ -985,7 +909,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     }
     // fallback tokens, kFbBatch at a time: teams of p.fb_groups warps rank the batch's tokens
     // over their 256-expert blocks, then warp jj merges the partial lists of the batch's token
-    // jj and writes it
+    // jj and writes it.  The partial lists lie past the staging, in the octet slots.
     const uint8_t* zs = zs0 + zs_buf(j, p.interleave) * C::ZS_BYTES;
     const int nfb = *fbcount;
     for (int fb0 = 0; fb0 < nfb; fb0 += kFbBatch) {
@@ -996,9 +920,9 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
         fallback_merge<KCAP>(a, part + bw * p.fb_groups * KCAP, p.fb_groups, n0 + fblist[fb0 + bw], lane);
       group_bar(kNamedBarB, kThreadsB);
     }
-    // reset the per-tile counters for the next tile
-    if (hh == 0) poolcnt[t] = 0;
-    group_bar(kNamedBarB, kThreadsB);  // every warp has read fbcount, the staging and the fallback lists
+    // every warp has read fbcount, the staging, the flags and the fallback lists: the next
+    // tile's pass B may write the octet slots again
+    group_bar(kNamedBarB, kThreadsB);
     if (gt == 0) {
       *fbcount = 0;
       mbar_arrive(&b.pairs_empty[pb]);
@@ -1056,14 +980,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(b.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= kWarpA0 && warp < kWarpB0) {  // clear the per-chunk pair counters
-    int* ccount = reinterpret_cast<int*>(smem + p.off_ccount);
-    for (int i = threadIdx.x - kWarpA0 * 32; i < p.nchunks; i += kThreadsA) ccount[i] = 0;
-  }
-  if (warp >= kWarpB0) {  // clear the per-token pool counters and the fallback count
-    int* poolcnt = reinterpret_cast<int*>(smem + p.off_poolcnt);
+  if (warp >= kWarpB0) {  // clear the per-token octet counts and the fallback count
     const int i = threadIdx.x - kWarpB0 * 32;
-    if (i < kBT) poolcnt[i] = 0;
+    if (i < kBT) reinterpret_cast<int*>(smem + p.off_hcnt)[i] = 0;
     if (i == 0) *reinterpret_cast<int*>(smem + p.off_fb) = 0;
   }
   tc_fence_before();
@@ -1142,44 +1061,31 @@ uint32_t layout(Params& p, int xs, int r2n, int nz) {
   off += r2n * C::R2_STAGE;
   p.off_zs = off = align_up(off, 1024);
   off += nz * C::ZS_BYTES;
-  // group A: list exchange, later the (chunk, rank) stage of the needed pairs
+  // group A: list exchange
   p.off_lists = off = align_up(off, 16);
-  off += C::KL * kBT * 4;
-  p.off_ccount = off;
-  off += p.nchunks * 4;
-  p.off_scan = off = align_up(off, 16);
-  off += kWarpsA * 4;
+  off += C::KA * kBT * 4;
   p.off_znorm = off;  // per token: |z_hi|^2 and |z_lo|^2 partial sums of both halves
   off += 4 * kBT * 4;
   p.off_cnorm = off;  // per warp: max squared column norm of R2; [8] = the result
   off += (kWarpsA + 1) * 4;
-  // group A -> group B, two buffers each; in the finalize a pair buffer holds the output
-  // staging
-  p.off_pairs = off = align_up(off, 16);
-  off += 2 * C::PAIR_BYTES;
-  p.off_cbase = off;
-  off += 2 * (p.nchunks + 1) * 4;
+  // group A -> group B, two buffers each: cut (fp32) and flags of every token
+  p.off_cut = off = align_up(off, 16);
+  off += 2 * kBT * 4;
   p.off_flag = off;
   off += 2 * kBT;
-  p.off_nq = off;
-  off += 2 * kBT;
-  // group B: candidate slots (later the output staging), counts, pool, fallback
-  p.off_cand = off = align_up(off, 16);
-  {
-    const uint32_t cand_bytes = kBT * C::KLP * 8, staging_bytes = 3 * kBT * KCAP * 4;
-    off += cand_bytes > staging_bytes ? cand_bytes : staging_bytes;
-  }
-  p.off_pc = off = align_up(off, 16);
-  off += kBT * C::KLP;
-  p.off_pool = off = align_up(off, 8);
-  off += kBT * C::POOL * 8;
-  p.off_poolcnt = off;
+  // group B: octet slots, their indices and counts, the list exchange, fallback
+  p.off_slots = off = align_up(off, 16);
+  off += C::OCT * kBT * 32;
+  p.off_ids = off;
+  off += C::OCT * kBT * 2;
+  p.off_hcnt = off = align_up(off, 16);
   off += kBT * 4;
   p.off_fb = off;  // fallback count, the tile's fallback tokens, per-token mark
   off += 4 + 2 * kBT;
-  // the fallback's partial lists reuse the candidate slots: the finalize has read them by then
-  static_assert(kFbBatch * kWarpsB * KCAP * 8 <= kBT * C::KLP * 8, "partial lists fit the slots");
-  p.off_part = p.off_cand;
+  // the output staging and, after it, the fallback's partial lists reuse the octet slots: the
+  // finalize has read them by then
+  p.off_stage = p.off_slots;
+  p.off_part = p.off_slots + C::STAGE_BYTES;
   p.off_bar = off = align_up(off, 8);
   off += kBarBytes;
   return off + 1024;  // alignment slack of the dynamic base
@@ -1231,7 +1137,6 @@ bool fill_params(const RouteArgs& a, Params& p, uint32_t& smem) {
   p.num_tiles = (int)((a.N + kBT - 1) / kBT);
   p.kb_count = (a.h + Cfg<R, KCAP>::BK - 1) / Cfg<R, KCAP>::BK;
   p.p_count = (a.M + kBE - 1) / kBE;
-  p.nchunks = (a.M + 31) / 32;
   p.fb_groups = 1;
   while (p.fb_groups < kWarpsB && 256 * p.fb_groups < a.M) p.fb_groups *= 2;
   int bits = 1;  // chunk ids run up to 4 p_count - 1 (the padded last tile)
@@ -1297,7 +1202,7 @@ bool supports_r(const RouteArgs& a) {
 }  // namespace tc
 
 bool fused_tc_fits(const RouteArgs& a) {
-  // 65536 experts = 2048 chunks: the pair-count scan covers 8 chunks per group-A thread
+  // up to 65536 experts = 2048 chunks: the chunk id takes at most 11 low bits of a pass-A key
   if (a.M > 65536 || a.k > 16 || a.N < 1 || a.N > 0x7fffffffLL - tc::kBT) return false;
   switch (a.r) {
     case 16: return tc::supports_r<16>(a);

@@ -89,7 +89,7 @@ def test_unfused_scratch_size_and_checks(lib):
     ((1430, 2048, 32, 4096, 8), "cluster"), ((1450, 2048, 32, 4096, 8), "fused_tc"),
     ((4096, 2048, 16, 4096, 4), "fused_tc"),
     ((262144, 2048, 128, 4096, 16), "cluster"),     # the fused kernel's plan does not hold r = 128, k > 8
-    ((262144, 2048, 128, 8192, 8), "fused_tc"), ((262144, 2048, 128, 11752, 8), "cluster"),
+    ((262144, 2048, 128, 8192, 8), "fused_tc"), ((262144, 2048, 128, 65536, 8), "fused_tc"),
     ((262144, 2048, 48, 4096, 8), "cluster"),       # r outside the fused kernel's ranks
     ((32768, 4096, 64, 65536, 8), "fused_tc"),
     ((16, 64, 32, 64, 0), None), ((16, 64, 24, 64, 4), None),
