@@ -113,7 +113,7 @@ struct Cfg {
   // octet slots of pass B: every 8-expert octet that holds an expert at or above the token's cut
   // is stored whole (its eight exact logits and its index), up to OCT per token; a token with
   // more goes to the exact fallback
-  static constexpr int OCT = R >= 128 ? KCAP + 4 : KCAP + 6;
+  static constexpr int OCT = R >= 128 ? KCAP + 4 : (R >= 64 ? KCAP + 5 : KCAP + 6);
   // In the finalize the octet slots take, in order: the output staging, the fallback's partial
   // lists, and (in odd slot rows from XS0 on, which only the second thread of a token reads)
   // the list that this thread hands to the first.
