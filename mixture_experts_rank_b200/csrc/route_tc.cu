@@ -112,15 +112,14 @@ struct Cfg {
   static constexpr int KA = KCAP;                      // chunk keys kept per token and warp in pass A
   // octet slots of pass B: every 8-expert octet that holds an expert at or above the token's cut
   // is stored whole (its eight exact logits and its index), up to OCT per token; a token with
-  // more goes to the exact fallback
+  // more goes to the exact fallback.  The warp of the low column half fills a token's slots from
+  // the first up, the other from the last down, so neither needs the other's count.
   static constexpr int OCT = R >= 128 ? KCAP + 4 : (R >= 64 ? KCAP + 5 : KCAP + 6);
-  // In the finalize the octet slots take, in order: the output staging, the fallback's partial
-  // lists, and (in odd slot rows from XS0 on, which only the second thread of a token reads)
-  // the list that this thread hands to the first.
+  // In the finalize the octet slots take the output staging and, after it, the fallback's
+  // partial lists.
   static constexpr uint32_t STAGE_BYTES = (3 * kBT * KCAP * 4 + 15) / 16 * 16;
   static constexpr uint32_t PART_BYTES = kFbBatch * kWarpsB * KCAP * 8;
-  static constexpr int XS0 = (int)((STAGE_BYTES + PART_BYTES + kBT * 32 - 1) / (kBT * 32)) | 1;
-  static_assert(XS0 + 2 * ((KCAP - 1) / 4) < OCT, "the exchanged list fits the odd slot rows");
+  static_assert(STAGE_BYTES + PART_BYTES <= OCT * kBT * 32, "staging and partial lists fit the octet slots");
   static constexpr int RK = 2 * R;                     // z_hi | z_lo columns of the z buffer
   static constexpr int BK = R >= 128 ? 32 : 64;        // hidden elements per X stage
   static constexpr uint32_t X_STAGE = kBT * BK * 2;    // 16 KB (8 KB at BK = 32)
@@ -768,9 +767,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
   uint8_t* zs0 = smem + p.off_zs;
   uint4* slots = reinterpret_cast<uint4*>(smem + p.off_slots);       // [slot][token][2]: eight logits
   uint16_t* ids = reinterpret_cast<uint16_t*>(smem + p.off_ids);     // [slot][token]: octet index
-  int* hcnt = reinterpret_cast<int*>(smem + p.off_hcnt);             // [token]: octets stored
-  // the list thread 1 hands to thread 0: entry i in slot row XS0 + 2 (i / 4), word i % 4
-  uint64_t* xchg = reinterpret_cast<uint64_t*>(slots + 2 * (C::XS0 * kBT + t));
+  int* hcnt = reinterpret_cast<int*>(smem + p.off_hcnt);             // [half][token]: octets found
   int32_t* sidx = reinterpret_cast<int32_t*>(smem + p.off_stage);    // [token][k]
   float* sex = reinterpret_cast<float*>(sidx + kBT * KCAP);
   float* slog = sex + kBT * KCAP;
@@ -792,6 +789,7 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     // ---------------- pass B: octets of the token that reach its cut (exact logits) ----------
     // Warp hh of a lane group reads columns 64 hh .. 64 hh + 63 of every tile, reduces each
     // octet to its maximum and stores the octets that reach its lane's cut.
+    int cnt = 0;  // octets of the lane's token that reach the cut in this warp's columns
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!bounded_wait(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
@@ -820,82 +818,81 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
                                  max3f(__uint_as_float(w[3]), __uint_as_float(w[4]), __uint_as_float(w[5])),
                                  fmaxf(__uint_as_float(w[6]), __uint_as_float(w[7])));
           if (om >= ccut) {  // rare per lane: about k + 1 octets of a token in all
-            const int sl = atomicAdd(&hcnt[t], 1);
-            if (sl < C::OCT) {
+            if (cnt < C::OCT) {
+              const int sl = hh ? C::OCT - 1 - cnt : cnt;
               uint4* dst = slots + 2 * (sl * kBT + t);
               dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
               dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
               ids[sl * kBT + t] = (uint16_t)((e0 >> 3) + o);
             }
+            ++cnt;
           }
         }
       }
       bd.next(C::NB);
     }
 
+    hcnt[hh * kBT + t] = cnt;
+
     // ---------------- finalize: order, softmax, store, count ---------------------------
-    // Two threads per token (the lane group's warps): thread hh keeps the best k of the
-    // candidates in the token's octets hh, hh + 2, ... as sorted 64-bit routing keys; thread 1
-    // hands its list to thread 0, which merges it and writes the token's outputs to the
-    // staging with the softmax gates.
+    // Thread 0 of a token (warp hh = 0) walks the token's stored octets, keeps the best k of
+    // the logits that reach the cut as sorted 64-bit routing keys, and writes the token's
+    // outputs to the staging with the softmax gates.
     if (!group_enter(&b.gbar[1], gph, b.abort_flag, a.status)) return;
     // from here to the hand-off nothing waits on another role
-    const int n = active ? hcnt[t] : 0;
-    const bool over = n > C::OCT;
     uint64_t kl[KCAP];
 #pragma unroll
     for (int i = 0; i < KCAP; ++i) kl[i] = 0ull;
-    if (!over) {
-      for (int sl = hh; sl < n; sl += 2) {
-        const uint4 q0 = slots[2 * (sl * kBT + t)], q1 = slots[2 * (sl * kBT + t) + 1];
-        const uint32_t eb = 8u * ids[sl * kBT + t];
-        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
-          key_insert64<KCAP>(kl, __uint_as_float(w[jj]) >= ccut ? route_key(w[jj], eb + jj) : 0ull);
-      }
-    }
-    if (hh == 1) {
-#pragma unroll
-      for (int i = 0; i < KCAP; ++i) xchg[(i >> 2) * (2 * kBT * 4) + (i & 3)] = kl[i];
-    }
-    group_bar(kNamedBarB, kThreadsB);  // the lists are exchanged; every other octet slot is read
-    if (hh == 0) {
-      if (active) {
-        if (!over) {
-#pragma unroll
-          for (int i = 0; i < KCAP; ++i) key_insert64<KCAP>(kl, xchg[(i >> 2) * (2 * kBT * 4) + (i & 3)]);
+    bool fb = false;
+    if (hh == 0 && active) {
+      const int c0 = hcnt[t], c1 = hcnt[kBT + t];
+      fb = c0 + c1 > C::OCT;  // the two ends of the slots met: an octet was not stored
+      if (!fb) {
+        for (int q = 0; q < c0 + c1; ++q) {
+          const int sl = q < c0 ? q : C::OCT - 1 - (q - c0);
+          const uint4* src = slots + 2 * (sl * kBT + t);
+          const uint4 q0 = src[0], q1 = src[1];
+          uint32_t m = (uint32_t)(__uint_as_float(q0.x) >= ccut) | ((uint32_t)(__uint_as_float(q0.y) >= ccut) << 1) |
+                       ((uint32_t)(__uint_as_float(q0.z) >= ccut) << 2) | ((uint32_t)(__uint_as_float(q0.w) >= ccut) << 3) |
+                       ((uint32_t)(__uint_as_float(q1.x) >= ccut) << 4) | ((uint32_t)(__uint_as_float(q1.y) >= ccut) << 5) |
+                       ((uint32_t)(__uint_as_float(q1.z) >= ccut) << 6) | ((uint32_t)(__uint_as_float(q1.w) >= ccut) << 7);
+          const uint32_t eb = 8u * ids[sl * kBT + t];
+          const uint32_t* sv = reinterpret_cast<const uint32_t*>(src);
+          while (m) {  // the logits of the octet that reach the cut: usually one
+            const int jj = __ffs(m) - 1;
+            m &= m - 1u;
+            key_insert64<KCAP>(kl, route_key(sv[jj], eb + (uint32_t)jj));
+          }
         }
         uint64_t kth = 0ull;
 #pragma unroll
         for (int i = 0; i < KCAP; ++i)
           if (i == a.k - 1) kth = kl[i];
-        const bool fb = over || kth == 0ull;  // too many octets, or fewer than k candidates
-        fbmark[t] = fb ? 1 : 0;
-        if (fb) {
-          fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
-        } else {
-          const float vtop = ord_inv((uint32_t)(kl[0] >> 32));
-          float ex[KCAP], sum = 0.f;
+        fb = kth == 0ull;  // fewer than k candidates
+      }
+      fbmark[t] = fb ? 1 : 0;
+      if (fb) fblist[atomicAdd(fbcount, 1)] = (uint8_t)t;
+    }
+    group_bar(kNamedBarB, kThreadsB);  // every octet slot is read: the staging may overwrite them
+    if (hh == 0 && active && !fb) {
+      const float vtop = ord_inv((uint32_t)(kl[0] >> 32));
+      float ex[KCAP], sum = 0.f;
 #pragma unroll
-          for (int i = 0; i < KCAP; ++i) {
-            ex[i] = i < a.k ? expf(ord_inv((uint32_t)(kl[i] >> 32)) - vtop) : 0.f;
-            sum += ex[i];
-          }
-          const float inv = 1.f / sum;
+      for (int i = 0; i < KCAP; ++i) {
+        ex[i] = i < a.k ? expf(ord_inv((uint32_t)(kl[i] >> 32)) - vtop) : 0.f;
+        sum += ex[i];
+      }
+      const float inv = 1.f / sum;
 #pragma unroll
-          for (int i = 0; i < KCAP; ++i) {
-            if (i < a.k) {
-              const uint32_t e = ~(uint32_t)kl[i];
-              sidx[t * a.k + i] = (int)e;
-              sex[t * a.k + i] = ex[i] * inv;
-              slog[t * a.k + i] = ord_inv((uint32_t)(kl[i] >> 32));
-              if (e < (uint32_t)a.M) atomicAdd(a.out_count + e, 1);
-            }
-          }
+      for (int i = 0; i < KCAP; ++i) {
+        if (i < a.k) {
+          const uint32_t e = ~(uint32_t)kl[i];
+          sidx[t * a.k + i] = (int)e;
+          sex[t * a.k + i] = ex[i] * inv;
+          slog[t * a.k + i] = ord_inv((uint32_t)(kl[i] >> 32));
+          if (e < (uint32_t)a.M) atomicAdd(a.out_count + e, 1);
         }
       }
-      hcnt[t] = 0;  // every thread of the token has read the count
     }
     group_bar(kNamedBarB, kThreadsB);
     // the tile's outputs are contiguous: copy the staging out with coalesced stores
@@ -980,11 +977,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(b.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= kWarpB0) {  // clear the per-token octet counts and the fallback count
-    const int i = threadIdx.x - kWarpB0 * 32;
-    if (i < kBT) reinterpret_cast<int*>(smem + p.off_hcnt)[i] = 0;
-    if (i == 0) *reinterpret_cast<int*>(smem + p.off_fb) = 0;
-  }
+  if (threadIdx.x == kWarpB0 * 32) *reinterpret_cast<int*>(smem + p.off_fb) = 0;  // fallback count
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1079,7 +1072,7 @@ uint32_t layout(Params& p, int xs, int r2n, int nz) {
   p.off_ids = off;
   off += C::OCT * kBT * 2;
   p.off_hcnt = off = align_up(off, 16);
-  off += kBT * 4;
+  off += 2 * kBT * 4;
   p.off_fb = off;  // fallback count, the tile's fallback tokens, per-token mark
   off += 4 + 2 * kBT;
   // the output staging and, after it, the fallback's partial lists reuse the octet slots: the
