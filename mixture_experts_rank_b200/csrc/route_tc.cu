@@ -753,6 +753,20 @@ __device__ __forceinline__ uint64_t route_key(uint32_t logit_bits, uint32_t expe
   return ((uint64_t)ord_key(__uint_as_float(logit_bits) + 0.f) << 32) | (uint64_t)(~expert);
 }
 
+// Stores an octet of logits (32 bytes at dst) and its 16-bit index (at idst) in shared memory
+// when pred is nonzero; predicated stores, no branch.
+__device__ __forceinline__ void st_octet_if(uint32_t pred, uint32_t dst, const uint32_t* w, uint32_t idst,
+                                            uint32_t id) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+      "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
+      "@p st.shared.v4.b32 [%1+16], {%6, %7, %8, %9};\n\t"
+      "@p st.shared.u16 [%10], %11;\n\t}" ::"r"(pred),
+      "r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(idst),
+      "h"((unsigned short)id)
+      : "memory");
+}
+
 template <int R, int KCAP>
 __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t tmem_base) {
   using C = Cfg<R, KCAP>;
@@ -790,6 +804,11 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     // Warp hh of a lane group reads columns 64 hh .. 64 hh + 63 of every tile, reduces each
     // octet to its maximum and stores the octets that reach its lane's cut.
     int cnt = 0;  // octets of the lane's token that reach the cut in this warp's columns
+    // shared-memory addresses of the lane's next octet slot and index; each stored octet moves
+    // them one slot row up (warp 0) or down (warp 1)
+    uint32_t sdst = smem_u32(slots + 2 * ((hh ? C::OCT - 1 : 0) * kBT + t));
+    uint32_t idst = smem_u32(ids + (hh ? C::OCT - 1 : 0) * kBT + t);
+    const int sstep = hh ? -kBT * 32 : kBT * 32, istep = hh ? -kBT * 2 : kBT * 2;
     for (int pt = 0; pt < p.p_count; ++pt) {
       if (!bounded_wait(&b.b_full[bd.i], bd.phase, b.abort_flag, a.status)) return;
       tc_fence_after();
@@ -817,16 +836,12 @@ __device__ void group_b(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
           const float om = max3f(max3f(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2])),
                                  max3f(__uint_as_float(w[3]), __uint_as_float(w[4]), __uint_as_float(w[5])),
                                  fmaxf(__uint_as_float(w[6]), __uint_as_float(w[7])));
-          if (om >= ccut) {  // rare per lane: about k + 1 octets of a token in all
-            if (cnt < C::OCT) {
-              const int sl = hh ? C::OCT - 1 - cnt : cnt;
-              uint4* dst = slots + 2 * (sl * kBT + t);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              ids[sl * kBT + t] = (uint16_t)((e0 >> 3) + o);
-            }
-            ++cnt;
-          }
+          // rare per lane (about k + 1 octets of a token in all): predicated stores, no branch
+          const int hit = om >= ccut ? 1 : 0;
+          st_octet_if(hit & (cnt < C::OCT ? 1 : 0), sdst, w, idst, (uint32_t)((e0 >> 3) + o));
+          sdst += (uint32_t)(hit * sstep);
+          idst += (uint32_t)(hit * istep);
+          cnt += hit;
         }
       }
       bd.next(C::NB);
