@@ -69,8 +69,8 @@ BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X,
 # was captured: once route_tc.cu differs from that source the figure is stale and traffic is
 # reported null.  Workloads without a capture report traffic null.
 NCU_TRAFFIC = {    # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
-    "prefill_r32": ((269283328 + 5237504) / 65536,
-                    "7874d9a4fcdca8febaeb56b71af05e6d697b7afed060f77f1da0e4cffd1eb2ee"),
+    "prefill_r32": ((269119488 + 5748224) / 65536,
+                    "48f6c3a3ece330d1a12531d34f52c2a4673ead09ec300a7cd665e670cdd4a8b3"),
 }
 L2_BYTES = 126 * 1024 * 1024
 
