@@ -69,8 +69,8 @@ BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X,
 # was captured: once route_tc.cu differs from that source the figure is stale and traffic is
 # reported null.  Workloads without a capture report traffic null.
 NCU_TRAFFIC = {    # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
-    "prefill_r32": ((269119488 + 5748224) / 65536,
-                    "48f6c3a3ece330d1a12531d34f52c2a4673ead09ec300a7cd665e670cdd4a8b3"),
+    "prefill_r32": ((269128960 + 4530432) / 65536,
+                    "d40538d94b91d5f9d612af0602d13518a68bf79fd55c9b7584f1e1dba652ac0f"),
 }
 L2_BYTES = 126 * 1024 * 1024
 

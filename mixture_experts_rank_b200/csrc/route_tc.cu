@@ -137,18 +137,14 @@ struct Cfg {
   static constexpr uint32_t ZS_SBO = (RK / 8) * 128;   // byte stride of 8-token groups
   static constexpr int ZCOLS = R < 32 ? 32 : R;        // TMEM columns per Z accumulator
   static constexpr int NBUF = (512 - 2 * ZCOLS) / 128 < 3 ? (512 - 2 * ZCOLS) / 128 : 3;
-  // Pass A takes one 128-column TMEM region.  At r = 16 it holds two 64-column buffers, one
-  // 64-expert job each (two jobs per R2 stage), so that the MMAs of the next job run while the
-  // consumers read the current one; at larger r the longer MMA chains of the extra jobs cost
-  // more than that overlap saves (measured), and the region is one 128-expert buffer.
-  static constexpr int NA = 1;
-  static constexpr int AJOBS = R == 16 ? 2 : 1;        // pass A jobs per R2 stage (= its buffers)
-  static constexpr int AJC = 128 / AJOBS;              // TMEM columns of a pass A job
-  static constexpr int NB = NBUF - NA;                 // 128-column TMEM buffers of pass B jobs
+#ifndef MORE_PASS_A_BUFS
+#define MORE_PASS_A_BUFS 1
+#endif
+  static constexpr int NA = MORE_PASS_A_BUFS < NBUF ? MORE_PASS_A_BUFS : 1;  // TMEM buffers of pass A jobs
+  static constexpr int NB = NBUF - NA;                 // TMEM buffers of pass B jobs (longer MMAs)
   static constexpr int ZCOL0 = NBUF * 128;             // first TMEM column of the Z accumulators
   static constexpr uint32_t IDESC_Z = idesc_bf16_f32(128, R, 0, 1);    // A = X (K-major), B = R1 (MN-major)
   static constexpr uint32_t IDESC_P = idesc_bf16_f32(128, 128, 0, 1);  // A = z pair, B = R2 tile
-  static constexpr uint32_t IDESC_PA = idesc_bf16_f32(128, AJC, 0, 1);  // pass A: B = R2 tile or one box
   static_assert(NB >= 1, "TMEM holds at least one buffer per pass");
 };
 
@@ -420,9 +416,7 @@ __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t
   const uint32_t zs0 = smem_u32(smem + p.off_zs), r20 = smem_u32(smem + p.off_r2);
   uint64_t* full = PASS_B ? b.b_full : b.a_full;
   uint64_t* empty = PASS_B ? b.b_empty : b.a_empty;
-  constexpr int NBUF = PASS_B ? C::NB : C::AJOBS;  // ring of TMEM buffers
-  constexpr int JOBS = PASS_B ? 1 : C::AJOBS;      // jobs per R2 stage
-  constexpr int JCOLS = PASS_B ? 128 : C::AJC;     // TMEM columns (and experts) of a job
+  constexpr int NBUF = PASS_B ? C::NB : C::NA;
   constexpr int COL0 = PASS_B ? C::NA * 128 : 0;
   // pass A reads z_hi only (K = r); pass B reads z_hi | z_lo (K = 2r) for exact logits
   constexpr int KSTEPS = PASS_B ? C::RK / 16 : R / 16;
@@ -444,20 +438,18 @@ __device__ void mma_pass(const Params& p, const Bars& b, uint8_t* smem, uint32_t
         if (t == 0 && !bounded_wait(&b.zsm_full[zs_buf(j, p.interleave)], zs_use(j, p.interleave) & 1, b.abort_flag,
                                 p.a.status))
           goto done;
-        for (int h = 0; h < JOBS; ++h) {
-          if (!bounded_wait(&empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
-          tc_fence_after();
-          const uint32_t dt = tmem_base + COL0 + d.i * JCOLS;
-          const uint32_t r2 = r20 + st * C::R2_STAGE + h * C::R2_BOX_BYTES;
+        if (!bounded_wait(&empty[d.i], d.phase ^ 1u, b.abort_flag, p.a.status)) goto done;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + COL0 + d.i * 128;
+        const uint32_t r2 = r20 + st * C::R2_STAGE;
 #pragma unroll
-          for (int kk = 0; kk < KSTEPS; ++kk) {
-            const uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
-            const uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
-            mma_bf16(dt, zd, rd, PASS_B ? C::IDESC_P : C::IDESC_PA, kk != 0);
-          }
-          mma_commit(&full[d.i]);
-          d.next(NBUF);
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          const uint64_t zd = smem_desc(zs + kk * 256, 128, C::ZS_SBO, kSwizzleNone);
+          const uint64_t rd = smem_desc(r2 + (kk % (R / 16)) * 2048, C::R2_BOX_BYTES, 1024, kSwizzle128B);
+          mma_bf16(dt, zd, rd, C::IDESC_P, kk != 0);
         }
+        mma_commit(&full[d.i]);
+        d.next(NBUF);
       }
       if (!p.r2_resident) {
         if (j >= 0)
@@ -560,38 +552,34 @@ __device__ void group_a(const Params& p, const Bars& b, uint8_t* smem, uint32_t 
     }
 
     // ---------------- pass A: chunk maxima of z_hi . R2 -> top KL chunk keys -------------
-    // Each R2 stage is AJOBS jobs of AJC experts; warp hh of a lane group owns columns
-    // AJC / 2 * hh .. AJC / 2 * (hh + 1) - 1 of every job, read 32 at a time.
-    constexpr int WC = C::AJC / 2;  // columns of a warp in a job
+    // warp hh of a lane group owns columns 64 hh .. 64 hh + 63 (chunks 4 pt + 2 hh, + 1)
 #pragma unroll
     for (int i = 0; i < KL; ++i) kl[i] = 0u;
     for (int pt = 0; pt < p.p_count; ++pt) {
+      if (!bounded_wait(&b.a_full[ad.i], ad.phase, b.abort_flag, a.status)) return;
+      tc_fence_after();
+      const uint32_t col = tmem_base + lane_base + ad.i * 128 + hh * 64;
+      const int c0 = pt * 4 + 2 * hh;
 #pragma unroll
-      for (int h = 0; h < C::AJOBS; ++h) {
-        if (!bounded_wait(&b.a_full[ad.i], ad.phase, b.abort_flag, a.status)) return;
-        tc_fence_after();
-        const uint32_t col = tmem_base + lane_base + ad.i * C::AJC + hh * WC;
-#pragma unroll
-        for (int q = 0; q < WC / 32; ++q) {
-          uint32_t v[32];
-          tmem_ld_x32(col + 32 * q, v);
-          tmem_wait_ld();
-          reg_fence<32>(v);
-          if (q == WC / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&b.a_empty[ad.i]);
-          }
-          const int c = (kBE * pt + C::AJC * h + WC * hh) / 32 + q;
-          if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-              if (32 * c + jj >= a.M) v[jj] = 0xff800000u;
-          }
-          key_insert<KL>(kl, (ord_key(max32(v)) & ~low) | (uint32_t)c);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld_x32(col + 32 * half, v);
+        tmem_wait_ld();
+        reg_fence<32>(v);
+        if (half == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b.a_empty[ad.i]);
         }
-        ad.next(C::AJOBS);
+        const int c = c0 + half;
+        if (32 * c + 32 > a.M) {  // out-of-range experts at -infinity (Algorithm 1)
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (32 * c + jj >= a.M) v[jj] = 0xff800000u;
+        }
+        key_insert<KL>(kl, (ord_key(max32(v)) & ~low) | (uint32_t)c);
       }
+      ad.next(C::NA);
       if (first) {
         // squared column norms of R2 (experts 16 aw .. 16 aw + 15 of the stage)
         int st;
