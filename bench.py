@@ -70,7 +70,7 @@ BACKWARD_METRIC = "router backward tokens/s (App. F Algorithm 3: gradients of X,
 # reported null.  Workloads without a capture report traffic null.
 NCU_TRAFFIC = {    # workload -> (bytes per token, sha256 of route_tc.cu at capture time)
     "prefill_r32": ((269128960 + 4530432) / 65536,
-                    "d40538d94b91d5f9d612af0602d13518a68bf79fd55c9b7584f1e1dba652ac0f"),
+                    "6c8948233b0fcb6b5ca0c1295b3c677ff694bfefe8d374bfafbc5ae569f85503"),
 }
 L2_BYTES = 126 * 1024 * 1024
 

@@ -32,15 +32,16 @@
 //               least the cut tlow - eps.  The cut of every token is handed to group B.
 //   warps 12-19  group B (two warps per TMEM lane group): per tile
 //     pass B    each warp reads its 64 columns of every exact tile, reduces each 8-expert
-//               octet to its maximum, and appends the experts whose exact logit reaches the
-//               token's cut (the candidates, about k + 1 per token) to the token's list in
-//               shared memory; octets without such an expert in any lane of the warp are
-//               skipped by a vote.
-//     finalize  two threads per token rank its few candidates in routing order (larger
-//               logit, then lower expert) into a shared-memory staging of the outputs,
-//               which the tile writes with coalesced stores; softmax, counts.  More
-//               candidates than the lists hold sends the token to an exact recomputation
-//               on CUDA cores shared by the group.
+//               octet to its maximum, and stores the octets that reach the token's cut
+//               (about k + 1 per token) whole in the token's octet slots, with predicated
+//               shared-memory stores; the two warps of a lane group fill the slots from
+//               opposite ends, each counting in a register.
+//     finalize  one thread per token walks its stored octets and keeps the best k logits
+//               that reach the cut as sorted 64-bit routing keys (larger logit, then lower
+//               expert), writes them with the softmax gates to a shared-memory staging of
+//               the outputs, which the tile writes with coalesced stores, and counts them.
+//               A token whose octets overflowed the slots goes to an exact recomputation on
+//               CUDA cores shared by the group.
 // The logit MMAs run in sweeps over the expert tiles: each sweep streams R2 once and every
 // R2 tile feeds pass B of tile t and pass A of tile t + 1 (with two z buffers; otherwise a
 // sweep carries one pass), so group B works on tile t while group A works on tile t + 1.
