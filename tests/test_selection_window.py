@@ -63,6 +63,7 @@ def candidates(z, R2, k):
         ccut = float(ord_inv(kth & ~low)) - eps
     cand = np.flatnonzero(exact >= ccut)
     halves = np.bincount((cand % 128) // 64, minlength=2)
+    candidates.cut = ccut  # the cut of the last token, for the octet model below
     return cand, exact, halves
 
 
@@ -129,3 +130,75 @@ def test_cut_needs_its_margin():
         tlow = np.sort(np.max((z_hi @ R2f).reshape(-1, 32), axis=1))[::-1][7]
         missed += int(np.any(exact[true_topk(exact, 8)] < tlow))
     assert missed > 0
+
+
+def octet_route(exact, cut, k, oct_slots):
+    """The fused kernel's pass B and finalize, restated on one token's exact logits: the two
+    warps of a lane group see experts by 64-column halves of each 128-expert tile, store every
+    8-expert octet whose maximum reaches the cut into slots filled from opposite ends, and a
+    single thread ranks the stored logits that reach the cut with (logit desc, expert asc)
+    routing keys.  Returns the top-k expert ids, or None when the token goes to the fallback
+    (slots overflowed, or fewer than k candidates)."""
+    M = exact.size
+    Mp = (M + 127) // 128 * 128
+    pad = np.full(Mp, -np.inf)
+    pad[:M] = exact
+    counts = [0, 0]
+    slots = [None] * oct_slots
+    for e0 in range(0, Mp, 8):
+        half = (e0 % 128) // 64
+        octet = pad[e0:e0 + 8]
+        if octet.max() >= cut:
+            if counts[half] < oct_slots:
+                sl = counts[half] if half == 0 else oct_slots - 1 - counts[half]
+                slots[sl] = (e0, octet.copy())
+            counts[half] += 1
+    if counts[0] + counts[1] > oct_slots:
+        return None
+    cand = []
+    for q in range(counts[0] + counts[1]):
+        sl = q if q < counts[0] else oct_slots - 1 - (q - counts[0])
+        e0, octet = slots[sl]
+        cand += [(v, e0 + j) for j, v in enumerate(octet) if v >= cut]
+    if len(cand) < k:
+        return None
+    cand.sort(key=lambda c: (-c[0], c[1]))
+    return np.array([e for _, e in cand[:k]])
+
+
+@pytest.mark.parametrize("N,h,r,M,k,unit,max_fb", [(200, 2048, 32, 4096, 8, True, 0.02),
+                                                   (300, 128, 32, 192, 4, False, 0.02),
+                                                   (200, 512, 32, 1000, 8, False, 0.02),
+                                                   (150, 256, 64, 2048, 16, False, 0.1)])
+def test_octet_slots_reproduce_the_exact_top_k(N, h, r, M, k, unit, max_fb):
+    """Storing whole octets that reach the cut, with the kernel's slot counts, and ranking what
+    they hold gives the exact top-k on every token that does not overflow.  Overflow is rare at
+    k <= 8; at k = 16 with only 2048 experts about 7 % of tokens need more than 21 slots."""
+    X, R1, R2 = syn.router_inputs(N, h, r, M, seed=5, x_unit_rms=unit)
+    Z = oracle.projection(X, R1, N, h, r)
+    R2f = syn.bf16_bits_to_f64(R2)
+    kcap = 4 if k <= 4 else (8 if k <= 8 else 16)
+    oct_slots = kcap + (4 if r >= 128 else (5 if r >= 64 else 6))
+    fallbacks = 0
+    for z in Z:
+        _, exact, _ = candidates(z, R2f, k)
+        sel = octet_route(exact, candidates.cut, k, oct_slots)
+        if sel is None:
+            fallbacks += 1
+            continue
+        np.testing.assert_array_equal(sel, true_topk(exact, k))
+    assert fallbacks <= max_fb * N, fallbacks
+
+
+def test_octet_slots_tie_order_and_overflow():
+    """Equal logits go to the lower expert; a token whose qualifying octets exceed the slots is
+    sent to the fallback rather than ranked from a partial list."""
+    exact = np.zeros(256)
+    exact[[3, 70, 130, 200]] = 2.0       # four equal winners in four octets
+    exact[[9, 140]] = 1.0
+    sel = octet_route(exact, 0.5, 4, 6)
+    np.testing.assert_array_equal(sel, [3, 70, 130, 200])
+    sel = octet_route(exact, 0.5, 5, 6)
+    np.testing.assert_array_equal(sel, [3, 70, 130, 200, 9])
+    many = np.ones(256)                  # every octet qualifies: 32 octets > 6 slots
+    assert octet_route(many, 0.5, 4, 6) is None
